@@ -1,0 +1,457 @@
+#!/usr/bin/env python3
+"""Decode-step benchmark of the per-head latent-KV path on B200.
+
+One step = one autoregressive decode step of the attention layer of the
+LLaVA-7B-like workload (E=4096, 32 heads x H=128, rank 32 int8 latents, batch 1,
+4096-token context, 128 decode steps): latent projection + quantise + append
+of the new token (lk_latent_project_append) and latent flash-decode attention
+(lk_latent_decode_attn).  Inputs are resident in HBM before timing; L2 is
+flushed (a 256 MiB write) before every step; each step is timed with CUDA
+events on the launching stream, the max over ranks is taken, and rank 0
+prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 2]
+
+--impl reference times the CPU oracle (float64, K and V materialised) on the
+host cores, same workload and metric.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/s and latent-attn HBM GB/s (% of B200 peak) at 1 GPU"
+UNIT = "tokens/s"
+FLUSH_BYTES = 256 << 20
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------- ranks
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world, backend):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world, device="cpu"):
+    """Max of a float over all ranks (every rank takes this collective step)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks (NVML, read-only)
+
+_REASONS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+    0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons every few ms while running (read-only NVML)."""
+
+    def __init__(self, device_index, period_s=0.005):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                self.reasons |= int(self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if self._h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        reasons = [n for bit, n in _REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- workload state
+
+class DecodeState:
+    """Device state of the attention-layer decode workload (one layer)."""
+
+    def __init__(self, w, device):
+        import rank_latent_kv_lk_b200 as lk
+        from rank_latent_kv_lk_b200 import synth
+        self.lk, self.w = lk, w
+        rk, rv = synth.ranks(w)
+        self.rk, self.rv = rk[0], rv[0]
+        A, BK, BV = synth.factors(w, 0, self.rk, self.rv)
+        self.A, self.BK, self.BV = A.to(device), BK.to(device), BV.to(device)
+        self.ck = lk.LatentCache(w.batch, self.rk, w.capacity, w.kind, w.group, device)
+        self.cv = lk.LatentCache(w.batch, self.rv, w.capacity, w.kind, w.group, device)
+        self.seq = torch.zeros(w.batch, dtype=torch.int32, device=device)
+        x_ctx = synth.context_tokens(w, 0).to(device)
+        lk.latent_project_append(self.ck, self.cv, x_ctx.reshape(-1, w.embed_dim), self.A, self.seq,
+                                 [0] * w.batch)
+        del x_ctx
+        self.lens = w.context
+        self.x_dec = synth.decode_tokens(w, 0).to(device)          # [steps, B, E]
+        self.q = synth.queries(w, 0).to(device)                    # [steps, B, nh, H]
+        self.out = torch.empty(w.batch, w.n_heads, w.head_dim, dtype=torch.bfloat16, device=device)
+        torch.cuda.synchronize()
+        lk.device_status()
+
+    def rewind_if_full(self):
+        if self.lens >= self.w.context + self.w.steps:
+            self.seq.fill_(self.w.context)
+            self.lens = self.w.context
+
+    def project(self, i, x=None):
+        j = i % self.w.steps
+        self.lk.latent_project_append(self.ck, self.cv, self.x_dec[j] if x is None else x, self.A, self.seq,
+                                      [self.lens] * self.w.batch)
+        self.lens += 1
+
+    def attend(self, i, q=None, out=None):
+        j = i % self.w.steps
+        return self.lk.latent_decode_attn(self.ck, self.cv, self.q[j] if q is None else q, self.BK, self.BV,
+                                          self.seq, self.lens, out=self.out if out is None else out)
+
+    # algorithmic bytes (what the math must touch once)
+    def attn_bytes(self, length):
+        w = self.w
+        rb = lambda r: r if w.kind == "i8" else r // 2
+        sb = lambda r: 4 if w.kind == "i8" else 2 * (-(-r // min(w.group, r)))
+        per_tok = sum(rb(r) + sb(r) for r in self.rk) + sum(rb(r) + sb(r) for r in self.rv)
+        factors = (sum(self.rk) + sum(self.rv)) * w.head_dim * self.BK.element_size()
+        qo = 2 * w.batch * w.n_heads * w.head_dim * 2
+        return w.batch * length * per_tok + factors + qo
+
+    def proj_bytes(self):
+        w = self.w
+        rb = lambda r: r if w.kind == "i8" else r // 2
+        codes = w.batch * (sum(rb(r) for r in self.rk) + sum(rb(r) for r in self.rv))
+        return self.A.numel() * self.A.element_size() + w.batch * w.embed_dim * 2 + codes
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rank_latent_kv_lk_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu capture, if the kernels have not changed since."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            d = json.load(f)
+        e = d[f"{kernel}@{workload}"]
+        if e["source_hash"] != kernel_source_hash():
+            return None
+        return e["dram_bytes_per_launch"]
+    except Exception:
+        return None
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
+
+def oracle_session(w):
+    """Oracle state after the (untimed) context prefill; returns a step function."""
+    import oracle as O
+    from rank_latent_kv_lk_b200 import synth
+    rk, rv = synth.ranks(w)
+    rk, rv = rk[0], rv[0]
+    A, BK, BV = synth.factors(w, 0, rk, rv)
+    A64 = synth.as_numpy(A).T.astype(np.float64)
+    BK, BV = synth.as_numpy(BK).astype(np.float64), synth.as_numpy(BV).astype(np.float64)
+    offk, offv = np.cumsum([0] + rk), np.cumsum([0] + rv)
+    BKh = [BK[offk[h]:offk[h + 1]] for h in range(len(rk))]
+    BVh = [BV[offv[h]:offv[h + 1]] for h in range(len(rv))]
+    ck, cv = O.LatentCache(w.batch, rk, w.kind, w.group), O.LatentCache(w.batch, rv, w.kind, w.group)
+    nk = sum(rk)
+    x_ctx = synth.as_numpy(synth.context_tokens(w, 0))
+    for b in range(w.batch):
+        v = O.latent_project_float(x_ctx[b], A64)
+        ck.append(b, O.quantize_latents(v[:, :nk], rk, w.kind, w.group))
+        cv.append(b, O.quantize_latents(v[:, nk:], rv, w.kind, w.group))
+    x_dec = synth.as_numpy(synth.decode_tokens(w, 0))
+    q = synth.as_numpy(synth.queries(w, 0))
+    scale = 1.0 / math.sqrt(w.head_dim)
+
+    def step(i):
+        j = i % w.steps
+        v = O.latent_project_float(x_dec[j], A64)
+        for b in range(w.batch):
+            ck.append(b, O.quantize_latents(v[b:b + 1, :nk], rk, w.kind, w.group))
+            cv.append(b, O.quantize_latents(v[b:b + 1, nk:], rv, w.kind, w.group))
+        return O.latent_attention(q[j], ck, cv, BKh, BVh, scale)
+
+    return step
+
+
+def blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, budget_s=15.0):
+    step = oracle_session(w)
+    t0 = time.perf_counter()
+    step(0)
+    t1 = time.perf_counter() - t0
+    n = int(max(1, min(w.steps - 1, budget_s / max(t1, 1e-6))))
+    t0 = time.perf_counter()
+    for i in range(1, n + 1):
+        step(i)
+    dt = time.perf_counter() - t0
+    return {"value": w.batch * n / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} decode steps of the workload after its context prefill (prefill untimed; "
+                      f"float64, K and V materialised)"}
+
+
+# ---------------------------------------------------------------- arms
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from rank_latent_kv_lk_b200.configs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    step = oracle_session(w)
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.warmup, args.warmup + args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    value = w.batch * args.steps / dt
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)",
+            "config": {"workload": w.name, "batch": w.batch, "context": w.context},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} timed oracle decode steps after {args.warmup} warm-up "
+                                       "steps and an untimed context prefill"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    from rank_latent_kv_lk_b200.configs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    st = DecodeState(w, device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def flush_l2():
+        flush.fill_(1)
+
+    # warm-up (untimed)
+    for i in range(max(3, args.warmup)):
+        st.rewind_if_full()
+        st.project(i)
+        st.attend(i)
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    lens_at = []
+    barrier(world)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(1e8))  # let the host queue run ahead of the device
+    with ClockSampler(local) as clocks:
+        for i in range(K):
+            st.rewind_if_full()
+            flush_l2()
+            ev[i][0].record(stream)
+            st.project(i)
+            ev[i][1].record(stream)
+            st.attend(i)
+            ev[i][2].record(stream)
+            lens_at.append(st.lens)
+        torch.cuda.synchronize()
+    barrier(world)
+    st.lk.device_status()
+    proj_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    attn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    step_ms = [p + a for p, a in zip(proj_ms, attn_ms)]
+    total_ms = max_over_ranks(sum(step_ms), world, device)
+    value = w.batch * K * world / (total_ms / 1e3)
+
+    # e2e: host buffers through the C ABI, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        xh = st.x_dec.cpu().pin_memory()
+        qh = st.q.cpu().pin_memory()
+        oh = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+        xd = torch.empty_like(st.x_dec[0])
+        qd = torch.empty_like(st.q[0])
+        e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        barrier(world)
+        torch.cuda.synchronize()
+        torch.cuda._sleep(int(1e8))
+        for i in range(K):
+            j = i % w.steps
+            st.rewind_if_full()
+            flush_l2()
+            e_ev[i][0].record(stream)
+            xd.copy_(xh[j], non_blocking=True)
+            qd.copy_(qh[j], non_blocking=True)
+            st.project(i, x=xd)
+            st.attend(i, q=qd)
+            oh.copy_(st.out, non_blocking=True)
+            e_ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e_ms = max_over_ranks(sum(e_ev[i][0].elapsed_time(e_ev[i][1]) for i in range(K)), world, device)
+        e2e = {"value": w.batch * K * world / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": xd.numel() * xd.element_size() + qd.numel() * qd.element_size(),
+               "d2h_bytes_per_step": oh.numel() * oh.element_size()}
+
+    if rank != 0:
+        _finish(world)
+        return 0
+    hbm, peak_kind = peaks()
+    attn_avg_s = statistics.mean(attn_ms) / 1e3
+    proj_avg_s = statistics.mean(proj_ms) / 1e3
+    attn_bytes = statistics.mean(st.attn_bytes(L) for L in lens_at)
+    proj_bytes = st.proj_bytes()
+    attn_gbs = attn_bytes / attn_avg_s / 1e9
+    proj_gbs = proj_bytes / proj_avg_s / 1e9
+    dominant = "latent_decode_attn" if attn_avg_s >= proj_avg_s else "latent_project_append"
+    if dominant == "latent_decode_attn":
+        ach, traffic = attn_gbs, profiled_traffic("decode_attn_kernel", w.key)
+    else:
+        ach, traffic = proj_gbs, profiled_traffic("proj_gemv_kernel", w.key)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (seeded, shapes of the LLaVA-7B-like workload)",
+        "config": {"workload": w.name, "batch": w.batch, "context": w.context, "decode_steps": w.steps,
+                   "storage": f"{w.kind} latents + per-token scales, bf16 factors and activations",
+                   "l2": "flushed before every step (256 MiB write, untimed)",
+                   "timing": "CUDA events per step on the launching stream; max over ranks",
+                   "parallelism": f"replicas x{world} (independent decode problems, no collective)"},
+        "roofline": {"kernel": dominant, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                     "frac": ach / hbm, "peak_kind": peak_kind, "traffic": traffic},
+        "latent_attn": {"achieved_gbs": attn_gbs, "frac_of_measured_hbm": attn_gbs / hbm,
+                        "frac_of_8tbs": attn_gbs / 8000.0, "us_per_launch": attn_avg_s * 1e6,
+                        "algorithmic_bytes_per_launch": attn_bytes},
+        "latent_project": {"achieved_gbs": proj_gbs, "us_per_call": proj_avg_s * 1e6,
+                           "algorithmic_bytes_per_call": proj_bytes},
+        "gpu_launches": K * 3,
+        "clocks": clocks.summary(),
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+    _finish(world)
+    return 0
+
+
+def _finish(world):
+    if world > 1 and torch.distributed.is_initialized():
+        torch.distributed.destroy_process_group()
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

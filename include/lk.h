@@ -1,0 +1,259 @@
+/*
+ * lk.h — C ABI of the per-head latent-KV decode library (sm_100a).
+ *
+ * What it computes.  A transformer whose K and V projections are factored per
+ * head, W_K^h ~ A_K^h B_K^h and W_V^h ~ A_V^h B_V^h with rank r_h << head dim
+ * H, caches only the quantised latents c^h = quant(x A^h) ("WSVD: Weighted
+ * Low-Rank Approximation for Fast and Efficient Execution of Low-Precision
+ * Vision-Language Models", technical summary §2A per-head SVD and §2C W8A8 /
+ * W8A4 and the fused decode kernel; "LASER: Loss-Aware Singular-value
+ * Decomposition and Rank Allocation ...", technical summary §2 non-uniform
+ * per-head ranks).  A decode step computes softmax(q K^T / sqrt(H)) V with
+ * K = dequant(C_K) B_K and V = dequant(C_V) B_V without ever writing K or V
+ * to memory: q is absorbed into latent space (q~ = B_K q), scores are taken
+ * against the latent codes, and the probability-weighted latent sum is
+ * up-projected by B_V once per head.  The LASER hybrid FFN linear
+ * (technical summary §3) y = x[:,D] W_D + (x[:,not D] U) V is provided in
+ * W8A8 form.
+ *
+ * Conventions for every entry point.
+ *  - All tensor pointers are DEVICE pointers owned by the caller unless the
+ *    argument says "host".  The library never allocates, frees or
+ *    synchronises device memory; scratch space is passed in as `workspace`.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).
+ *  - Every call validates its arguments on the host first and returns an
+ *    error status WITHOUT launching anything or writing any output if a check
+ *    fails.  lk_last_error() then holds a one-line explanation (per host
+ *    thread).  A CUDA launch error is reported as LK_ERR_CUDA.
+ *  - Device pointers must be 16-byte aligned unless stated otherwise; the
+ *    latent cache planes and workspaces must be 256-byte aligned.
+ *  - Weight matrices are stored [out_features, in_features], row-major
+ *    (each output's weights contiguous), like torch.nn.Linear.weight.
+ *  - fp16 / bf16 values are passed as 16-bit storage (uint16_t bit patterns).
+ */
+#ifndef LK_H_
+#define LK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so callers need no CUDA header. */
+typedef struct CUstream_st* lk_stream_t;
+
+typedef enum {
+  LK_OK = 0,
+  LK_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad enum          */
+  LK_ERR_SHAPE = 2,       /* sizes inconsistent or outside supported range  */
+  LK_ERR_DTYPE = 3,       /* dtype not supported for this argument          */
+  LK_ERR_ALIGN = 4,       /* pointer or size not aligned as required        */
+  LK_ERR_CAPACITY = 5,    /* append would overrun the cache capacity        */
+  LK_ERR_UNSUPPORTED = 6, /* valid request this build does not implement    */
+  LK_ERR_WORKSPACE = 7,   /* workspace null or smaller than required        */
+  LK_ERR_CUDA = 8,        /* a CUDA call failed (text in lk_last_error)     */
+  LK_ERR_DEVICE = 9       /* a kernel reported a bounded wait that expired  */
+} lk_status;
+
+typedef enum {
+  LK_F32 = 0,
+  LK_BF16 = 1,
+  LK_F16 = 2,
+  LK_I8 = 3, /* int8 codes: r codes per (token, head), one fp32 scale        */
+  LK_I4 = 4  /* int4 codes: two per byte (low nibble = even dim), one fp16
+                scale per group of g consecutive dims                         */
+} lk_dtype;
+
+#define LK_MAX_HEADS 128 /* heads per layer                                   */
+#define LK_MAX_RANK 64   /* latent rank per head for attention               */
+#define LK_MAX_HEAD_DIM 256
+
+/*
+ * Latent cache of one layer, for K or for V (caller-owned device memory).
+ *
+ * Ranks: ranks[h] = r_h (HOST array, read during the call only).  int8 caches
+ * need r_h % 4 == 0, int4 caches r_h % 8 == 0, 4 <= r_h <= LK_MAX_RANK.  The K
+ * and V caches of a layer may have different ranks (LASER allocates them
+ * independently).
+ *
+ * Row bytes of head h: rb_h = r_h (int8) or r_h / 2 (int4).  Scale groups:
+ * ng_h = 1 (int8) or ceil(r_h / min(group, r_h)) (int4).
+ *
+ * codes: for batch row b and head h, one contiguous plane of capacity * rb_h
+ *   bytes at byte offset (b * sum_h rb_h + sum_{h' < h} rb_h') * capacity.
+ *   Inside a plane, tokens are kept in blocks of 16; with chunk size
+ *   cs = 16 if rb % 16 == 0, else 8 if rb % 8 == 0, else 4, byte k of token
+ *   t's code row sits at
+ *       (t / 16) * 16 * rb + (k / cs) * 16 * cs + (t % 16) * cs + (k % cs).
+ *   (Thread-per-token readers then touch consecutive 16-byte words.)
+ * scales: int8: fp32 [capacity] per (b, h) at element offset
+ *   (b * n_heads + h) * capacity.  int4: fp16 [capacity][ng_h] per (b, h)
+ *   at element offset (b * sum_h ng_h + sum_{h' < h} ng_h') * capacity.
+ * capacity must be a multiple of 16.
+ */
+typedef struct {
+  int32_t batch;        /* B                                                */
+  int32_t n_heads;      /* n_h <= LK_MAX_HEADS                              */
+  int32_t capacity;     /* T_max, multiple of 16                            */
+  lk_dtype code_dtype;  /* LK_I8 or LK_I4                                   */
+  int32_t group;        /* int4 group size along r (effective min(g, r_h))  */
+  const int32_t* ranks; /* HOST [n_heads]                                   */
+  void* codes;          /* device, 256-byte aligned                        */
+  void* scales;         /* device, 256-byte aligned                        */
+} lk_latent_cache;
+
+/* Bytes the caller must allocate for a cache's code and scale planes. */
+lk_status lk_latent_cache_bytes(const lk_latent_cache* cache, size_t* codes_bytes,
+                                size_t* scales_bytes);
+
+/*
+ * Latent projection + quantisation + append (WSVD §2A: the per-head latent
+ * x A^h is what is cached; §2C: it is stored in 8 or 4 bits; LASER §4 fuses
+ * projection, latent generation and quantisation).
+ *
+ * x: [B * n_new, embed_dim] row-major, row b * n_new + t is batch row b's
+ *   t-th new token.  x_dtype LK_F32, LK_BF16 or LK_I8 (then x_scale, fp32
+ *   [B * n_new], is the per-token dequantisation scale; else NULL).
+ * A: [N_tot, embed_dim] (K-major), N_tot = sum r_K + sum r_V: rows are the
+ *   K heads' latent dims in head order, then the V heads'.  a_dtype must
+ *   equal x_dtype; for LK_I8, a_scale is fp16 [N_tot] (per latent dim).
+ * For every new token and head the latent v^h (fp32) is quantised with the
+ *   cache's rule (see lk_quantize_latent) and written at position
+ *   seq_len[b] + t.  Float inputs: v is the fp32 dot product.  LK_I8 inputs:
+ *   v = fl32(fl32(fl32(sum x_q A_q) * x_scale) * a_scale), exact int32 sum.
+ * seq_len: device int32 [B], read as the write offset, then increased by
+ *   n_new once every token is written.  seq_len_host: HOST copy of the same
+ *   values, used for the capacity check seq_len + n_new <= capacity.
+ * workspace: lk_latent_project_workspace_bytes(...) bytes, 256-B aligned;
+ *   its first 256 bytes are an arrival counter that must be zero before the
+ *   first call and that every completed call leaves zero.
+ */
+lk_status lk_latent_project_append(const lk_latent_cache* k_cache, const lk_latent_cache* v_cache,
+                                   const void* x, lk_dtype x_dtype, const float* x_scale,
+                                   const void* A, lk_dtype a_dtype, const uint16_t* a_scale,
+                                   int32_t embed_dim, int32_t n_new, int32_t* seq_len,
+                                   const int32_t* seq_len_host, void* workspace,
+                                   size_t workspace_bytes, lk_stream_t stream);
+size_t lk_latent_project_workspace_bytes(const lk_latent_cache* k_cache,
+                                         const lk_latent_cache* v_cache, int32_t embed_dim,
+                                         int32_t n_new, lk_dtype x_dtype);
+
+/*
+ * Latent decode attention (WSVD §2C fused kernel; absorption form).
+ *
+ * For each batch row b and head h, over positions t in [0, seq_len[b]):
+ *   q~ = B_K^h q^h                                  (absorb q, r_K values)
+ *   s_t = softmax_scale * sigma_K[t] . (c_K[t] . q~)   (per group for int4)
+ *   p = softmax(s);  u = sum_t p_t * sigma_V[t] * c_V[t]   (r_V values)
+ *   out^h = u B_V^h                                  ([H])
+ * computed split-K over t (flash-decoding) with per-split partials
+ * (max, sum, u) merged in latent space.  K and V are never formed.
+ *
+ * q: [B, n_heads, head_dim], q_dtype LK_F32 or LK_BF16.
+ * B_K, B_V: per-head factors [r_h, head_dim] row-major, packed head after
+ *   head (head h starts at element sum_{h'<h} r_h' * head_dim); b_dtype
+ *   LK_F32 or LK_BF16.
+ * seq_len: device [B] (values may differ per row); max_seq_len: HOST upper
+ *   bound on those values (<= capacity); positions past it are not read.
+ *   A row with seq_len 0 gets a zero output.
+ * out: [B, n_heads, head_dim], LK_F32 or LK_BF16.
+ * n_split: number of sequence splits per (b, h); 0 picks one for the GPU.
+ *   The result does not depend on it beyond float rounding.
+ * workspace: lk_latent_decode_workspace_bytes(...) bytes, 256-B aligned; its
+ *   first region holds per-(b, h) arrival counters that must be zero before
+ *   the first call and that every completed call leaves zero.
+ */
+lk_status lk_latent_decode_attn(const lk_latent_cache* k_cache, const lk_latent_cache* v_cache,
+                                const void* q, lk_dtype q_dtype, const void* B_K,
+                                const void* B_V, lk_dtype b_dtype, int32_t head_dim,
+                                const int32_t* seq_len, int32_t max_seq_len,
+                                float softmax_scale, void* out, lk_dtype out_dtype,
+                                int32_t n_split, void* workspace, size_t workspace_bytes,
+                                lk_stream_t stream);
+size_t lk_latent_decode_workspace_bytes(const lk_latent_cache* k_cache,
+                                        const lk_latent_cache* v_cache, int32_t max_seq_len,
+                                        int32_t n_split);
+
+/*
+ * LASER hybrid dense + low-rank linear, W8A8 (LASER technical summary §3:
+ * selected input channels go through SVD factors, the rest stay dense; both
+ * branches RTN-quantised).
+ *
+ *   acc_D = x_q[:, dense_idx] W_D^T            (exact int32)
+ *   t     = fl32(fl32(fl32(x_q[:, lr_idx] U^T) * x_scale) * s_U)
+ *   (t_q, s_t) = per-token int8 absmax quantisation of t
+ *   acc_V = t_q V^T                            (exact int32)
+ *   y     = acc_D * x_scale * s_D + acc_V * s_t * s_V (+ residual), fp32,
+ *           stored as y_dtype.
+ * rank == 0 with n_dense == k_in is a plain W8A8 linear.
+ */
+typedef struct {
+  int32_t k_in;              /* input channels                                 */
+  int32_t n_out;             /* output channels                                */
+  int32_t rank;              /* low-rank width R (0 = no low-rank branch)      */
+  int32_t n_dense;           /* |D|                                            */
+  const int32_t* dense_idx;  /* device [n_dense], sorted, disjoint from lr_idx */
+  const int32_t* lr_idx;     /* device [k_in - n_dense], sorted                */
+  const int8_t* W_D;         /* [n_out, n_dense]                               */
+  const uint16_t* s_D;       /* fp16 [n_out]                                   */
+  const int8_t* U;           /* [rank, k_in - n_dense]                         */
+  const uint16_t* s_U;       /* fp16 [rank]                                    */
+  const int8_t* V;           /* [n_out, rank]                                  */
+  const uint16_t* s_V;       /* fp16 [n_out]                                   */
+} lk_lowrank_weight;
+
+/* x_q: int8 [m, k_in]; x_scale fp32 [m]; residual: bf16 [m, n_out] or NULL;
+ * y: [m, n_out] LK_BF16 or LK_F32; t_q_out / t_scale_out: optional
+ * ([m, rank] int8, [m] fp32) copies of the requantised latent;
+ * workspace: lk_lowrank_workspace_bytes(w, m) bytes. */
+lk_status lk_lowrank_linear(const lk_lowrank_weight* w, const int8_t* x_q, const float* x_scale,
+                            int32_t m, const uint16_t* residual, void* y, lk_dtype y_dtype,
+                            int8_t* t_q_out, float* t_scale_out, void* workspace,
+                            size_t workspace_bytes, lk_stream_t stream);
+size_t lk_lowrank_workspace_bytes(const lk_lowrank_weight* w, int32_t m);
+
+/*
+ * Stand-alone latent quantiser (the rule lk_latent_project_append applies),
+ * exposed for bit-exact testing.  v: fp32 [m, r].
+ *  LK_I8: scale = fl32(absmax / 127); code = clamp(rint(fl32(v / scale)),
+ *    -127, 127) (round half to even); scale 0 gives zero codes.
+ *    codes int8 [m, r]; scales fp32 [m].
+ *  LK_I4: per group of g = min(group, r) dims: scale16 = fp16_rn(fl32(absmax /
+ *    7)) saturated to 65504; code = clamp(rint(fl32(v / scale)), -7, 7);
+ *    codes packed [m, r / 2] (low nibble = even dim); scales fp16
+ *    [m, ceil(r / g)].  r must be even.
+ */
+lk_status lk_quantize_latent(const float* v, int32_t m, int32_t r, lk_dtype code_dtype,
+                             int32_t group, void* codes, void* scales, lk_stream_t stream);
+
+/* Per-row int8 absmax quantisation of activations (same rule as LK_I8
+ * above).  x: [m, k] LK_F32 or LK_BF16; x_q int8 [m, k]; x_scale fp32 [m]. */
+lk_status lk_quantize_rows_i8(const void* x, lk_dtype x_dtype, int32_t m, int32_t k,
+                              int8_t* x_q, float* x_scale, lk_stream_t stream);
+
+/* RMSNorm with unit weight, y = x / sqrt(mean(x^2) + eps), then per-row int8
+ * quantisation of y (fp32).  x: [m, k] LK_F32 or LK_BF16. */
+lk_status lk_rmsnorm_quant_i8(const void* x, lk_dtype x_dtype, int32_t m, int32_t k, float eps,
+                              int8_t* x_q, float* x_scale, lk_stream_t stream);
+
+/* SwiGLU h = silu(gate) * up in fp32 (LASER §4 fuses it into the FFN), then
+ * per-row int8 quantisation of h.  gate, up: [m, n] LK_F32 or LK_BF16. */
+lk_status lk_swiglu_quant_i8(const void* gate, const void* up, lk_dtype dtype, int32_t m,
+                             int32_t n, int8_t* h_q, float* h_scale, lk_stream_t stream);
+
+/* Synchronises the device, then reports (and with reset != 0 clears) the
+ * error word kernels set when a bounded wait expires: LK_OK or LK_ERR_DEVICE. */
+lk_status lk_device_status(int32_t reset);
+
+const char* lk_status_string(lk_status status);
+const char* lk_last_error(void);
+int32_t lk_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LK_H_ */

@@ -1,0 +1,201 @@
+"""Thin torch-facing wrappers over the C ABI (marshalling only).
+
+Tensors are device tensors allocated by torch; the library computes.  Every
+wrapper raises LkError when the library rejects its arguments.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import math
+
+import torch
+
+from ._lib import LK_BF16, LK_F16, LK_F32, LK_I4, LK_I8, LatentCacheDesc, LowrankWeightDesc, check, lib
+from .layout import CacheGeometry
+
+_DT = {torch.float32: LK_F32, torch.bfloat16: LK_BF16, torch.float16: LK_F16, torch.int8: LK_I8}
+
+
+def _dtype_code(t):
+    try:
+        return _DT[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}") from None
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+class _WorkspacePool:
+    """Zero-initialised per-device scratch buffers, one per purpose.
+
+    Each entry point keeps its own buffer because the arrival counters at the
+    start of a workspace must read zero at the start of every call (every
+    completed call leaves them zero)."""
+
+    def __init__(self):
+        self._bufs = {}
+
+    def get(self, purpose, nbytes, device):
+        key = (purpose, str(device))
+        buf = self._bufs.get(key)
+        if buf is None or buf.numel() < nbytes:
+            buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+            self._bufs[key] = buf
+        return buf
+
+
+workspaces = _WorkspacePool()
+
+
+class LatentCache:
+    """Device latent cache of one layer for K or V (codes + scales planes)."""
+
+    def __init__(self, batch, ranks, capacity, kind="i8", group=32, device="cuda"):
+        if kind not in ("i8", "i4"):
+            raise ValueError("kind must be 'i8' or 'i4'")
+        self.geom = CacheGeometry(batch, ranks, capacity, kind, group)
+        self.batch, self.ranks, self.capacity, self.kind, self.group = batch, list(ranks), capacity, kind, group
+        self.codes = torch.zeros(self.geom.codes_bytes, dtype=torch.uint8, device=device)
+        self.scales = torch.zeros(self.geom.scales_elems,
+                                  dtype=torch.float32 if kind == "i8" else torch.float16, device=device)
+        self._ranks = (C.c_int32 * len(self.ranks))(*self.ranks)
+        self._desc = LatentCacheDesc(batch, len(self.ranks), capacity, LK_I8 if kind == "i8" else LK_I4,
+                                     group, self._ranks, self.codes.data_ptr(), self.scales.data_ptr())
+
+    @property
+    def n_heads(self):
+        return len(self.ranks)
+
+    def desc(self):
+        return C.byref(self._desc)
+
+    def load(self, rows, scales):
+        """Fill from logical code rows (rows[b][h]: uint8 [T, rb]) and scales."""
+        c, s = self.geom.pack(rows, scales)
+        self.codes.copy_(torch.from_numpy(c))
+        self.scales.copy_(torch.from_numpy(s))
+
+    def read(self, lens):
+        """Logical code rows and scales of the first lens[b] tokens (host copies)."""
+        return self.geom.unpack(self.codes.cpu().numpy(), self.scales.cpu().numpy(), lens)
+
+
+def latent_project_append(k_cache, v_cache, x, A, seq_len, seq_len_host, x_scale=None, a_scale=None,
+                          stream=None):
+    """Project new tokens to per-head latents, quantise them and append.
+
+    x: [B * n_new, E] (f32 / bf16 / int8); A: [sum r_K + sum r_V, E] same dtype;
+    int8 inputs need x_scale fp32 [B * n_new] and a_scale fp16 [N_tot].
+    seq_len: device int32 [B] (advanced by n_new); seq_len_host: list of ints.
+    """
+    rows = x.shape[0]
+    if rows % k_cache.batch:
+        raise ValueError("x rows must be a multiple of the batch")
+    n_new = rows // k_cache.batch
+    E = x.shape[-1]
+    xdt = _dtype_code(x)
+    host = (C.c_int32 * k_cache.batch)(*[int(v) for v in seq_len_host])
+    need = lib.lk_latent_project_workspace_bytes(k_cache.desc(), v_cache.desc(), E, n_new, xdt)
+    ws = workspaces.get("project", need, x.device)
+    check(lib.lk_latent_project_append(
+        k_cache.desc(), v_cache.desc(), _ptr(x), xdt, _ptr(x_scale), _ptr(A), _dtype_code(A), _ptr(a_scale),
+        E, n_new, _ptr(seq_len), host, _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def latent_decode_attn(k_cache, v_cache, q, B_K, B_V, seq_len, max_seq_len, softmax_scale=None, out=None,
+                       out_dtype=None, n_split=0, stream=None):
+    """softmax(q K^T * scale) V over the latent caches, without forming K or V.
+
+    q: [B, n_heads, H]; B_K / B_V: per-head factors packed head after head,
+    [sum r, H]; seq_len: device int32 [B]; max_seq_len: host bound.
+    """
+    H = q.shape[-1]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(H)
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    need = lib.lk_latent_decode_workspace_bytes(k_cache.desc(), v_cache.desc(), int(max_seq_len), int(n_split))
+    ws = workspaces.get("decode", need, q.device)
+    check(lib.lk_latent_decode_attn(
+        k_cache.desc(), v_cache.desc(), _ptr(q), _dtype_code(q), _ptr(B_K), _ptr(B_V), _dtype_code(B_K), H,
+        _ptr(seq_len), int(max_seq_len), float(softmax_scale), _ptr(out), _dtype_code(out), int(n_split),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+class LowrankWeight:
+    """Device weights of one LASER hybrid linear (int8, fp16 scales)."""
+
+    def __init__(self, k_in, n_out, rank, dense_idx, lr_idx, W_D, s_D, U, s_U, V, s_V):
+        self.k_in, self.n_out, self.rank = k_in, n_out, rank
+        self.n_dense = 0 if dense_idx is None else int(dense_idx.numel())
+        self.tensors = (dense_idx, lr_idx, W_D, s_D, U, s_U, V, s_V)
+        self._desc = LowrankWeightDesc(k_in, n_out, rank, self.n_dense, *[
+            (t.data_ptr() if t is not None else None) for t in self.tensors])
+
+    def desc(self):
+        return C.byref(self._desc)
+
+
+def lowrank_linear(w, x_q, x_scale, residual=None, y=None, y_dtype=torch.bfloat16, t_q_out=None, t_scale_out=None,
+                   stream=None):
+    m = x_q.shape[0]
+    if y is None:
+        y = torch.empty((m, w.n_out), dtype=y_dtype, device=x_q.device)
+    need = lib.lk_lowrank_workspace_bytes(w.desc(), m)
+    ws = workspaces.get("lowrank", need, x_q.device)
+    check(lib.lk_lowrank_linear(w.desc(), _ptr(x_q), _ptr(x_scale), m, _ptr(residual), _ptr(y), _dtype_code(y),
+                                _ptr(t_q_out), _ptr(t_scale_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+def quantize_latent(v, kind="i8", group=32, stream=None):
+    """v: fp32 [m, r] -> (codes, scales) with the cache's quantisation rule."""
+    m, r = v.shape
+    if kind == "i8":
+        codes = torch.empty((m, r), dtype=torch.int8, device=v.device)
+        scales = torch.empty((m,), dtype=torch.float32, device=v.device)
+    else:
+        g = min(group, r)
+        codes = torch.empty((m, r // 2), dtype=torch.uint8, device=v.device)
+        scales = torch.empty((m, -(-r // g)), dtype=torch.float16, device=v.device)
+    check(lib.lk_quantize_latent(_ptr(v), m, r, LK_I8 if kind == "i8" else LK_I4, group, _ptr(codes),
+                                 _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def quantize_rows_i8(x, stream=None):
+    m, k = x.shape
+    q = torch.empty((m, k), dtype=torch.int8, device=x.device)
+    s = torch.empty((m,), dtype=torch.float32, device=x.device)
+    check(lib.lk_quantize_rows_i8(_ptr(x), _dtype_code(x), m, k, _ptr(q), _ptr(s), _stream(stream)))
+    return q, s
+
+
+def rmsnorm_quant_i8(x, eps=1e-5, stream=None):
+    m, k = x.shape
+    q = torch.empty((m, k), dtype=torch.int8, device=x.device)
+    s = torch.empty((m,), dtype=torch.float32, device=x.device)
+    check(lib.lk_rmsnorm_quant_i8(_ptr(x), _dtype_code(x), m, k, float(eps), _ptr(q), _ptr(s), _stream(stream)))
+    return q, s
+
+
+def swiglu_quant_i8(gate, up, stream=None):
+    m, n = gate.shape
+    q = torch.empty((m, n), dtype=torch.int8, device=gate.device)
+    s = torch.empty((m,), dtype=torch.float32, device=gate.device)
+    check(lib.lk_swiglu_quant_i8(_ptr(gate), _ptr(up), _dtype_code(gate), m, n, _ptr(q), _ptr(s),
+                                 _stream(stream)))
+    return q, s
+
+
+def device_status(reset=True):
+    """Synchronise and raise if a kernel reported an expired bounded wait."""
+    check(lib.lk_device_status(1 if reset else 0))

@@ -1,0 +1,594 @@
+// Latent decode attention, split-K over the sequence (sm_100a).
+//
+// Per (batch row b, head h, split s) one CTA of 128 threads:
+//   1. absorbs q into latent space: q~ = B_K^h q * softmax_scale * log2(e)
+//      (WSVD page §2C: the fused kernel works from the per-head latents;
+//      without positional rotation (q B_K^T) C^T equals q K^T);
+//   2. streams its slice of the latent cache (K codes, V codes and their
+//      scales) HBM -> shared memory with bulk copies on the TMA engine,
+//      4 stages deep, one mbarrier per stage;
+//   3. one token per thread per stage: score = sigma_K . (c_K . q~), a
+//      warp-uniform running max, p = 2^(score - max), and
+//      u += p * sigma_V * c_V in registers (r_V values);
+//   4. reduces (max, sum, u) over the CTA and writes it as a partial in
+//      latent space; the last CTA of the (b, h) to arrive (atomic ticket, no
+//      waiting) merges all partials and applies out = (u / sum) B_V^h.
+// K and V are never formed; the only per-token traffic is the latent codes
+// and their scales.
+#include "lk_common.cuh"
+#include "lk_internal.h"
+
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kStageT = 128;  // tokens per pipeline stage: one per thread
+constexpr int kStages = 4;
+constexpr int kMaxR = LK_MAX_RANK;
+
+struct DecodeParams {
+  const uint8_t* codes_k;
+  const uint8_t* codes_v;
+  const uint8_t* scales_k;
+  const uint8_t* scales_v;
+  const void* q;
+  const void* BK;
+  const void* BV;
+  const int32_t* seq_len;
+  void* out;
+  float* partials;    // [B * n_heads][n_split][part_stride]
+  int32_t* counters;  // [B * n_heads]
+  int batch, n_heads, head_dim, capacity;
+  int group_k, group_v;  // int4 requested group size (effective min(g, r))
+  int q_bf16, b_bf16, out_bf16;
+  int n_split, stages_per_split, part_stride, max_len;
+  float qscale;  // softmax_scale * log2(e)
+  // bytes of one pipeline stage region (max over heads), multiples of 128
+  int st_kc, st_vc, st_ks, st_vs;
+  uint8_t rk[LK_MAX_HEADS];
+  uint8_t rv[LK_MAX_HEADS];
+};
+
+struct HeadGeom {
+  int rk, rv;      // ranks
+  int rbk, rbv;    // code bytes per token
+  int ngk, ngv;    // scale groups per token (1 for int8)
+  int gk, gv;      // effective group size (int4)
+  int64_t kc_off;  // byte offset of this (b, h) K code plane
+  int64_t vc_off;
+  int64_t ks_off;  // element offset of this (b, h) K scale plane
+  int64_t vs_off;
+  int64_t bk_off;  // element offset of B_K^h
+  int64_t bv_off;
+};
+
+template <int KIND>
+LK_DEVICE int row_bytes(int r) { return KIND == 0 ? r : r / 2; }
+template <int KIND>
+LK_DEVICE int n_groups(int r, int g) { return KIND == 0 ? 1 : (r + g - 1) / g; }
+
+// Prefix sums over heads, computed by each warp with strided lanes + shuffles.
+template <int KIND>
+LK_DEVICE HeadGeom head_geometry(const DecodeParams& p, int b, int h) {
+  int lane = threadIdx.x & 31;
+  int pk = 0, pv = 0, tk = 0, tv = 0, pgk = 0, pgv = 0, tgk = 0, tgv = 0, prk = 0, prv = 0;
+  for (int i = lane; i < p.n_heads; i += 32) {
+    int rk = p.rk[i], rv = p.rv[i];
+    int bk = row_bytes<KIND>(rk), bv = row_bytes<KIND>(rv);
+    int gk = n_groups<KIND>(rk, min(p.group_k, rk)), gv = n_groups<KIND>(rv, min(p.group_v, rv));
+    tk += bk; tv += bv; tgk += gk; tgv += gv;
+    if (i < h) { pk += bk; pv += bv; pgk += gk; pgv += gv; prk += rk; prv += rv; }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    pk += __shfl_xor_sync(0xffffffffu, pk, o);
+    pv += __shfl_xor_sync(0xffffffffu, pv, o);
+    tk += __shfl_xor_sync(0xffffffffu, tk, o);
+    tv += __shfl_xor_sync(0xffffffffu, tv, o);
+    pgk += __shfl_xor_sync(0xffffffffu, pgk, o);
+    pgv += __shfl_xor_sync(0xffffffffu, pgv, o);
+    tgk += __shfl_xor_sync(0xffffffffu, tgk, o);
+    tgv += __shfl_xor_sync(0xffffffffu, tgv, o);
+    prk += __shfl_xor_sync(0xffffffffu, prk, o);
+    prv += __shfl_xor_sync(0xffffffffu, prv, o);
+  }
+  HeadGeom g;
+  g.rk = p.rk[h];
+  g.rv = p.rv[h];
+  g.rbk = row_bytes<KIND>(g.rk);
+  g.rbv = row_bytes<KIND>(g.rv);
+  g.gk = KIND == 0 ? g.rk : min(p.group_k, g.rk);
+  g.gv = KIND == 0 ? g.rv : min(p.group_v, g.rv);
+  g.ngk = n_groups<KIND>(g.rk, g.gk);
+  g.ngv = n_groups<KIND>(g.rv, g.gv);
+  const int64_t cap = p.capacity;
+  g.kc_off = ((int64_t)b * tk + pk) * cap;
+  g.vc_off = ((int64_t)b * tv + pv) * cap;
+  g.ks_off = ((int64_t)b * tgk + pgk) * cap;
+  g.vs_off = ((int64_t)b * tgv + pgv) * cap;
+  g.bk_off = (int64_t)prk * p.head_dim;
+  g.bv_off = (int64_t)prv * p.head_dim;
+  return g;
+}
+
+// Loads the code row chunk `c` (CS bytes) of local token `tl` from a staged
+// region laid out in 16-token blocks.
+template <int CS>
+struct Chunk;
+template <>
+struct Chunk<16> {
+  uint32_t w[4];
+  LK_DEVICE void load(const uint8_t* base, int rb, int tl, int c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(base + (tl >> 4) * 16 * rb + c * 256 + (tl & 15) * 16);
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  }
+};
+template <>
+struct Chunk<8> {
+  uint32_t w[2];
+  LK_DEVICE void load(const uint8_t* base, int rb, int tl, int c) {
+    const uint2 v = *reinterpret_cast<const uint2*>(base + (tl >> 4) * 16 * rb + c * 128 + (tl & 15) * 8);
+    w[0] = v.x; w[1] = v.y;
+  }
+};
+template <>
+struct Chunk<4> {
+  uint32_t w[1];
+  LK_DEVICE void load(const uint8_t* base, int rb, int tl, int c) {
+    w[0] = *reinterpret_cast<const uint32_t*>(base + (tl >> 4) * 16 * rb + c * 64 + (tl & 15) * 4);
+  }
+};
+
+// Dims covered by one 32-bit word of codes.
+template <int KIND>
+struct DimsPerWord { static constexpr int v = KIND == 0 ? 4 : 8; };
+
+// Expands word `wd` of codes into fp32 values (exact integers).
+template <int KIND>
+LK_DEVICE void expand_word(uint32_t wd, float* f) {
+  if (KIND == 0) {
+    const uint32_t x = wd ^ 0x80808080u;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) f[k] = lk_s8_from_xored(x, k);
+  } else {
+    const uint32_t x = wd ^ 0x88888888u;        // each nibble n -> c + 8
+    const uint32_t ev = x & 0x0F0F0F0Fu;         // dims 0, 2, 4, 6
+    const uint32_t od = (x >> 4) & 0x0F0F0F0Fu;  // dims 1, 3, 5, 7
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      f[2 * k] = __uint_as_float(__byte_perm(ev, 0x4B000000u, 0x7540u | k)) - 8388616.0f;
+      f[2 * k + 1] = __uint_as_float(__byte_perm(od, 0x4B000000u, 0x7540u | k)) - 8388616.0f;
+    }
+  }
+}
+
+LK_DEVICE float load_scale(const uint8_t* base, int i, int kind) {
+  return kind == 0 ? reinterpret_cast<const float*>(base)[i]
+                   : lk_f16_to_f32(reinterpret_cast<const uint16_t*>(base)[i]);
+}
+
+// Score of one token: sum over groups of sigma_g * (c . q~) restricted to the group.
+template <int KIND, int CS>
+LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom& g, int tl,
+                            const float* qt) {
+  constexpr int DPW = DimsPerWord<KIND>::v;
+  constexpr int WPC = CS / 4;                   // words per chunk
+  constexpr int MAXCH = (KIND == 0 ? kMaxR : kMaxR / 2) / CS;
+  const int nch = g.rbk / CS;
+  float s = 0.0f;
+  if (KIND == 0) {
+    float acc = 0.0f;
+#pragma unroll
+    for (int c = 0; c < MAXCH; ++c) {
+      if (c < nch) {
+        Chunk<CS> ch;
+        ch.load(kc, g.rbk, tl, c);
+#pragma unroll
+        for (int wi = 0; wi < WPC; ++wi) {
+          float f[4];
+          expand_word<0>(ch.w[wi], f);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) acc = fmaf(f[k], qt[(c * WPC + wi) * DPW + k], acc);
+        }
+      }
+    }
+    s = acc * reinterpret_cast<const float*>(ks)[tl];
+  } else {
+#pragma unroll
+    for (int c = 0; c < MAXCH; ++c) {
+      if (c < nch) {
+        Chunk<CS> ch;
+        ch.load(kc, g.rbk, tl, c);
+#pragma unroll
+        for (int wi = 0; wi < WPC; ++wi) {
+          float f[8];
+          expand_word<1>(ch.w[wi], f);
+          float acc = 0.0f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc = fmaf(f[k], qt[(c * WPC + wi) * DPW + k], acc);
+          const int dim0 = (c * WPC + wi) * DPW;
+          s = fmaf(acc, load_scale(ks, tl * g.ngk + dim0 / g.gk, 1), s);
+        }
+      }
+    }
+  }
+  return s;
+}
+
+// u += w * sigma_V * c_V for one token.
+template <int KIND, int CS>
+LK_DEVICE void accumulate_v(const uint8_t* vc, const uint8_t* vs, const HeadGeom& g, int tl,
+                            float p, float* u) {
+  constexpr int DPW = DimsPerWord<KIND>::v;
+  constexpr int WPC = CS / 4;
+  constexpr int MAXCH = (KIND == 0 ? kMaxR : kMaxR / 2) / CS;
+  const int nch = g.rbv / CS;
+  const float w0 = KIND == 0 ? p * reinterpret_cast<const float*>(vs)[tl] : 0.0f;
+#pragma unroll
+  for (int c = 0; c < MAXCH; ++c) {
+    if (c < nch) {
+      Chunk<CS> ch;
+      ch.load(vc, g.rbv, tl, c);
+#pragma unroll
+      for (int wi = 0; wi < WPC; ++wi) {
+        float f[DPW];
+        expand_word<KIND>(ch.w[wi], f);
+        const int dim0 = (c * WPC + wi) * DPW;
+        const float w = KIND == 0 ? w0 : p * load_scale(vs, tl * g.ngv + dim0 / g.gv, 1);
+#pragma unroll
+        for (int k = 0; k < DPW; ++k) u[dim0 + k] = fmaf(w, f[k], u[dim0 + k]);
+      }
+    }
+  }
+}
+
+struct SmemLayout {
+  int stage_bytes;
+  int off_kc, off_vc, off_ks, off_vs;  // within a stage
+  int off_qt;                          // q~ [kMaxR] floats
+  int off_red;                         // reduction scratch [4 warps][2 + kMaxR]
+  int off_bar;                         // mbarriers
+  int off_misc;
+  int total;
+};
+
+LK_DEVICE SmemLayout smem_layout(const DecodeParams& p) {
+  SmemLayout L;
+  L.off_kc = 0;
+  L.off_vc = p.st_kc;
+  L.off_ks = p.st_kc + p.st_vc;
+  L.off_vs = p.st_kc + p.st_vc + p.st_ks;
+  L.stage_bytes = p.st_kc + p.st_vc + p.st_ks + p.st_vs;
+  L.off_qt = kStages * L.stage_bytes;
+  L.off_red = L.off_qt + kMaxR * 4;
+  L.off_bar = L.off_red + 4 * (2 + kMaxR) * 4;
+  L.off_misc = L.off_bar + kStages * 8;
+  L.total = L.off_misc + 16;
+  return L;
+}
+
+template <int KIND, int CSK, int CSV>
+LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* smem, const SmemLayout& L,
+                           int b, int h, int split, int len, int first_stage, int n_my) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.off_bar);
+  float* qt_s = reinterpret_cast<float*>(smem + L.off_qt);
+  float* red = reinterpret_cast<float*>(smem + L.off_red);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.off_misc);
+  const int ssz = KIND == 0 ? 4 : 2;
+
+  auto issue = [&](int j) {  // stage j of this split -> buffer j % kStages
+    const int buf = j % kStages;
+    const int64_t t0 = (int64_t)(first_stage + j) * kStageT;
+    const int64_t end = min((int64_t)((len + 15) & ~15), (int64_t)p.capacity);
+    const int ntok = (int)min((int64_t)kStageT, end - t0);
+    uint8_t* st = smem + buf * L.stage_bytes;
+    const uint32_t bkc = ntok * g.rbk, bvc = ntok * g.rbv;
+    const uint32_t bks = ntok * g.ngk * ssz, bvs = ntok * g.ngv * ssz;
+    lk_mbar_arrive_expect_tx(&bars[buf], bkc + bvc + bks + bvs);
+    lk_bulk_g2s(st + L.off_kc, p.codes_k + g.kc_off + t0 * g.rbk, bkc, &bars[buf]);
+    lk_bulk_g2s(st + L.off_vc, p.codes_v + g.vc_off + t0 * g.rbv, bvc, &bars[buf]);
+    lk_bulk_g2s(st + L.off_ks, p.scales_k + (g.ks_off + t0 * g.ngk) * ssz, bks, &bars[buf]);
+    lk_bulk_g2s(st + L.off_vs, p.scales_v + (g.vs_off + t0 * g.ngv) * ssz, bvs, &bars[buf]);
+  };
+
+  if (tid == 0) {
+    for (int j = 0; j < min(kStages, n_my); ++j) issue(j);
+  }
+
+  // ---- absorb q: q~[i] = qscale * sum_d B_K[i][d] q[d]   (overlaps the first loads)
+  {
+    const int H = p.head_dim;
+    const int64_t qoff = ((int64_t)b * p.n_heads + h) * H;
+    for (int i = warp; i < g.rk; i += kThreads / 32) {
+      float acc = 0.0f;
+      for (int d = lane; d < H; d += 32) {
+        float qd, bkd;
+        if (p.q_bf16) qd = lk_bf16_to_f32(reinterpret_cast<const uint16_t*>(p.q)[qoff + d]);
+        else qd = reinterpret_cast<const float*>(p.q)[qoff + d];
+        const int64_t bi = g.bk_off + (int64_t)i * H + d;
+        if (p.b_bf16) bkd = lk_bf16_to_f32(reinterpret_cast<const uint16_t*>(p.BK)[bi]);
+        else bkd = reinterpret_cast<const float*>(p.BK)[bi];
+        acc = fmaf(qd, bkd, acc);
+      }
+      acc = lk_warp_sum(acc);
+      if (lane == 0) qt_s[i] = acc * p.qscale;
+    }
+  }
+  __syncthreads();
+  float qt[kMaxR];
+#pragma unroll
+  for (int i = 0; i < kMaxR; ++i) qt[i] = (i < g.rk) ? qt_s[i] : 0.0f;
+
+  float u[kMaxR];
+#pragma unroll
+  for (int i = 0; i < kMaxR; ++i) u[i] = 0.0f;
+  float m_run = -INFINITY, l_run = 0.0f;
+
+  bool aborted = false;
+  int stopped_at = 0;
+  for (int j = 0; j < n_my; ++j) {
+    const int buf = j % kStages;
+    const bool ok = lk_mbar_wait_bounded(&bars[buf], (uint32_t)((j / kStages) & 1), LK_WAIT_LIMIT_NS);
+    if (!ok) *abort_flag = 1;
+    const uint8_t* st = smem + buf * L.stage_bytes;
+    const int t = (first_stage + j) * kStageT + tid;
+    const bool valid = ok && t < len;
+    float s = -INFINITY;
+    if (valid) s = token_score<KIND, CSK>(st + L.off_kc, st + L.off_ks, g, tid, qt);
+    const float wmax = lk_warp_max(s);
+    if (wmax > m_run) {  // warp-uniform: rescale the running sums once per new max
+      const float alpha = exp2f(m_run - wmax);
+      l_run *= alpha;
+#pragma unroll
+      for (int i = 0; i < kMaxR; ++i) u[i] *= alpha;
+      m_run = wmax;
+    }
+    if (valid) {
+      const float pr = exp2f(s - m_run);
+      l_run += pr;
+      accumulate_v<KIND, CSV>(st + L.off_vc, st + L.off_vs, g, tid, pr, u);
+    }
+    __syncthreads();  // every thread is done with this buffer
+    if (*abort_flag) { aborted = true; stopped_at = j; break; }
+    if (tid == 0 && j + kStages < n_my) issue(j + kStages);
+  }
+  if (aborted) {
+    if (tid == 0) {
+      lk_dev_fail(LK_DEV_TIMEOUT_PIPE);
+      // drain copies still in flight into this CTA's shared memory: stages
+      // stopped_at .. stopped_at + kStages - 1 were issued and not all waited for
+      for (int j = stopped_at; j < min(n_my, stopped_at + kStages); ++j) {
+        if (!lk_mbar_wait_bounded(&bars[j % kStages], (uint32_t)((j / kStages) & 1), LK_WAIT_LIMIT_NS))
+          lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
+      }
+    }
+    m_run = -INFINITY;
+    l_run = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kMaxR; ++i) u[i] = 0.0f;
+  }
+
+  // ---- reduce (m, l, u) over the CTA
+  l_run = lk_warp_sum(l_run);
+#pragma unroll
+  for (int i = 0; i < kMaxR; ++i) {
+    if (i < g.rv) u[i] = lk_warp_sum(u[i]);
+  }
+  float* wred = red + warp * (2 + kMaxR);
+  if (lane == 0) {
+    wred[0] = m_run;
+    wred[1] = l_run;
+  }
+  // lane i keeps u[i] and u[i + 32]; write them out with static indices
+#pragma unroll
+  for (int i = 0; i < kMaxR; ++i) {
+    if (i < g.rv && lane == (i & 31)) wred[2 + i] = u[i];
+  }
+  __syncthreads();
+
+  const int nw = kThreads / 32;
+  float M = -INFINITY;
+  for (int w = 0; w < nw; ++w) M = fmaxf(M, red[w * (2 + kMaxR)]);
+  // tid j < rv merges u_j; tid == rv (or a spare thread) merges l
+  float* cta = red;  // reuse warp 0's slot after reading; stage through registers first
+  float mine = 0.0f;
+  if (M != -INFINITY) {
+    if (tid < g.rv) {
+      for (int w = 0; w < nw; ++w) {
+        const float mw = red[w * (2 + kMaxR)];
+        if (mw != -INFINITY) mine += red[w * (2 + kMaxR) + 2 + tid] * exp2f(mw - M);
+      }
+    } else if (tid == kMaxR) {
+      for (int w = 0; w < nw; ++w) {
+        const float mw = red[w * (2 + kMaxR)];
+        if (mw != -INFINITY) mine += red[w * (2 + kMaxR) + 1] * exp2f(mw - M);
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < g.rv) cta[2 + tid] = mine;
+  if (tid == kMaxR) cta[1] = mine;
+  if (tid == 0) cta[0] = M;
+  __syncthreads();
+
+  const int64_t bh = (int64_t)b * p.n_heads + h;
+  int* flag = reinterpret_cast<int*>(smem + L.off_misc) + 1;
+  if (p.n_split > 1) {
+    float* part = p.partials + (bh * p.n_split + split) * p.part_stride;
+    for (int i = tid; i < 2 + g.rv; i += kThreads) part[i] = cta[i];
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      const int ticket = atomicAdd(&p.counters[bh], 1);
+      *flag = (ticket == p.n_split - 1);
+    }
+    __syncthreads();
+    if (!*flag) return;
+    __threadfence();
+    // last arriver: merge every split's partial (all visible in L2)
+    float Mg = -INFINITY;
+    for (int s2 = 0; s2 < p.n_split; ++s2)
+      Mg = fmaxf(Mg, __ldcg(p.partials + (bh * p.n_split + s2) * p.part_stride));
+    float acc = 0.0f;
+    const int idx = (tid < g.rv) ? 2 + tid : (tid == kMaxR ? 1 : -1);
+    if (idx >= 0 && Mg != -INFINITY) {
+      for (int s2 = 0; s2 < p.n_split; ++s2) {
+        const float* ps = p.partials + (bh * p.n_split + s2) * p.part_stride;
+        const float ms = __ldcg(ps);
+        if (ms != -INFINITY) acc += __ldcg(ps + idx) * exp2f(ms - Mg);
+      }
+    }
+    __syncthreads();
+    if (idx >= 0) cta[idx] = acc;
+    if (tid == 0) {
+      cta[0] = Mg;
+      p.counters[bh] = 0;  // ready for the next call
+    }
+    __syncthreads();
+  }
+
+  // ---- out = (u / l) B_V^h
+  const float lsum = cta[1];
+  const float inv = (cta[0] == -INFINITY || lsum == 0.0f) ? 0.0f : 1.0f / lsum;
+  const int H = p.head_dim;
+  const int64_t ooff = bh * H;
+  for (int d = tid; d < H; d += kThreads) {
+    float o = 0.0f;
+    for (int j = 0; j < g.rv; ++j) {
+      const int64_t bi = g.bv_off + (int64_t)j * H + d;
+      const float bv = p.b_bf16 ? lk_bf16_to_f32(reinterpret_cast<const uint16_t*>(p.BV)[bi])
+                                : reinterpret_cast<const float*>(p.BV)[bi];
+      o = fmaf(cta[2 + j], bv, o);
+    }
+    o *= inv;
+    if (p.out_bf16) reinterpret_cast<uint16_t*>(p.out)[ooff + d] = lk_f32_to_bf16(o);
+    else reinterpret_cast<float*>(p.out)[ooff + d] = o;
+  }
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const __grid_constant__ DecodeParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const SmemLayout L = smem_layout(p);
+  const HeadGeom g = head_geometry<KIND>(p, b, h);
+  int len = p.seq_len[b];
+  len = max(0, min(len, p.max_len));
+
+  const int total_stages = (len + kStageT - 1) / kStageT;
+  const int first_stage = split * p.stages_per_split;
+  const int n_my = max(0, min(p.stages_per_split, total_stages - first_stage));
+
+  if (threadIdx.x == 0) {
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.off_bar);
+    for (int i = 0; i < kStages; ++i) lk_mbar_init(&bars[i], 1);
+    lk_fence_mbar_init();
+    *reinterpret_cast<int*>(smem + L.off_misc) = 0;
+  }
+  __syncthreads();
+
+  const int csk = lk_chunk_bytes(g.rbk), csv = lk_chunk_bytes(g.rbv);
+#define LK_BODY(A, B_) decode_body<KIND, A, B_>(p, g, smem, L, b, h, split, len, first_stage, n_my)
+  if (csk == 16) {
+    if (csv == 16) LK_BODY(16, 16); else if (csv == 8) LK_BODY(16, 8); else LK_BODY(16, 4);
+  } else if (csk == 8) {
+    if (csv == 16) LK_BODY(8, 16); else if (csv == 8) LK_BODY(8, 8); else LK_BODY(8, 4);
+  } else {
+    if (csv == 16) LK_BODY(4, 16); else if (csv == 8) LK_BODY(4, 8); else LK_BODY(4, 4);
+  }
+#undef LK_BODY
+}
+
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+}  // namespace
+
+LK_DEFINE_STATUS_ACCESSOR(lk_decode_status_word)
+
+namespace lk {
+
+int decode_pick_split(int units, int max_len, int num_sms) {
+  const int stages = (max_len + kStageT - 1) / kStageT;
+  if (stages <= 1) return 1;
+  const int target = num_sms * 3;  // about three resident CTAs per SM
+  int s = (target + units - 1) / units;
+  s = std::max(1, std::min(s, stages));
+  return s;
+}
+
+size_t decode_workspace_bytes(int batch, int n_heads, int rv_max, int n_split) {
+  const size_t counters = (size_t)round_up(batch * n_heads * 4, 256);
+  const size_t stride = (size_t)round_up(2 + rv_max, 4);
+  return counters + (size_t)batch * n_heads * n_split * stride * 4;
+}
+
+cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
+  DecodeParams p{};
+  p.codes_k = static_cast<const uint8_t*>(a.codes_k);
+  p.codes_v = static_cast<const uint8_t*>(a.codes_v);
+  p.scales_k = static_cast<const uint8_t*>(a.scales_k);
+  p.scales_v = static_cast<const uint8_t*>(a.scales_v);
+  p.q = a.q;
+  p.BK = a.BK;
+  p.BV = a.BV;
+  p.seq_len = a.seq_len;
+  p.out = a.out;
+  p.batch = a.batch;
+  p.n_heads = a.n_heads;
+  p.head_dim = a.head_dim;
+  p.capacity = a.capacity;
+  p.group_k = a.group_k;
+  p.group_v = a.group_v;
+  p.q_bf16 = a.q_bf16;
+  p.b_bf16 = a.b_bf16;
+  p.out_bf16 = a.out_bf16;
+  p.max_len = a.max_len;
+  p.qscale = a.softmax_scale * 1.4426950408889634f;
+  int rk_max = 0, rv_max = 0, rbk_max = 0, rbv_max = 0, ngk_max = 1, ngv_max = 1;
+  for (int h = 0; h < a.n_heads; ++h) {
+    p.rk[h] = (uint8_t)a.ranks_k[h];
+    p.rv[h] = (uint8_t)a.ranks_v[h];
+    rk_max = std::max(rk_max, a.ranks_k[h]);
+    rv_max = std::max(rv_max, a.ranks_v[h]);
+    if (a.kind == 1) {
+      const int gk = std::min(a.group_k, a.ranks_k[h]), gv = std::min(a.group_v, a.ranks_v[h]);
+      ngk_max = std::max(ngk_max, (a.ranks_k[h] + gk - 1) / gk);
+      ngv_max = std::max(ngv_max, (a.ranks_v[h] + gv - 1) / gv);
+    }
+  }
+  rbk_max = a.kind == 0 ? rk_max : rk_max / 2;
+  rbv_max = a.kind == 0 ? rv_max : rv_max / 2;
+  const int ssz = a.kind == 0 ? 4 : 2;
+  p.st_kc = round_up(kStageT * rbk_max, 128);
+  p.st_vc = round_up(kStageT * rbv_max, 128);
+  p.st_ks = round_up(kStageT * ngk_max * ssz, 128);
+  p.st_vs = round_up(kStageT * ngv_max * ssz, 128);
+  const int stages = std::max(1, (a.max_len + kStageT - 1) / kStageT);
+  int n_split = a.n_split;
+  if (n_split <= 0) n_split = decode_pick_split(a.batch * a.n_heads, a.max_len, a.num_sms);
+  n_split = std::max(1, std::min(n_split, stages));
+  p.stages_per_split = (stages + n_split - 1) / n_split;
+  n_split = (stages + p.stages_per_split - 1) / p.stages_per_split;
+  p.n_split = n_split;
+  p.part_stride = round_up(2 + rv_max, 4);
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  p.counters = reinterpret_cast<int32_t*>(ws);
+  p.partials = reinterpret_cast<float*>(ws + round_up(a.batch * a.n_heads * 4, 256));
+
+  const int stage_bytes = p.st_kc + p.st_vc + p.st_ks + p.st_vs;
+  const int smem = kStages * stage_bytes + kMaxR * 4 + 4 * (2 + kMaxR) * 4 + kStages * 8 + 16;
+  dim3 grid(n_split, a.n_heads, a.batch);
+  cudaError_t e;
+  if (a.kind == 0) {
+    e = cudaFuncSetAttribute(decode_attn_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    decode_attn_kernel<0><<<grid, kThreads, smem, stream>>>(p);
+  } else {
+    e = cudaFuncSetAttribute(decode_attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    decode_attn_kernel<1><<<grid, kThreads, smem, stream>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace lk

@@ -1,0 +1,110 @@
+// Internal launch interfaces between the C-ABI layer (lk_api.cu) and the
+// kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include <algorithm>
+
+#include "lk.h"
+
+namespace lk {
+
+// ---------------------------------------------------------------- decode
+struct DecodeLaunch {
+  const void* codes_k;
+  const void* codes_v;
+  const void* scales_k;
+  const void* scales_v;
+  const void* q;
+  const void* BK;
+  const void* BV;
+  const int32_t* seq_len;
+  void* out;
+  void* workspace;
+  const int32_t* ranks_k;  // host
+  const int32_t* ranks_v;  // host
+  int kind;                // 0 = int8, 1 = int4
+  int batch, n_heads, head_dim, capacity;
+  int group_k, group_v;
+  int q_bf16, b_bf16, out_bf16;
+  int max_len, n_split, num_sms;
+  float softmax_scale;
+};
+int decode_pick_split(int units, int max_len, int num_sms);
+size_t decode_workspace_bytes(int batch, int n_heads, int rv_max, int n_split);
+cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- projection
+enum XType { X_F32 = 0, X_BF16 = 1, X_I8 = 2 };
+
+// Heads of one cache as seen by the quantise-and-append epilogue.
+struct CacheView {
+  void* codes;
+  void* scales;
+  int kind;      // 0 = int8, 1 = int4
+  int group;
+  int n_heads;
+  int capacity;
+};
+
+struct ProjectLaunch {
+  CacheView k, v;
+  const int32_t* ranks_k;  // host
+  const int32_t* ranks_v;  // host
+  const void* x;
+  const float* x_scale;
+  const void* A;
+  const uint16_t* a_scale;
+  int xtype;
+  int batch, n_new, embed_dim, n_tot;
+  int32_t* seq_len;
+  void* workspace;
+  size_t workspace_bytes;
+  int num_sms;
+};
+size_t project_workspace_bytes(int rows, int n_tot, int embed_dim, int xtype, int num_sms);
+cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- low-rank linear
+struct LowrankLaunch {
+  int k_in, n_out, rank, n_dense, m;
+  const int32_t* dense_idx;
+  const int32_t* lr_idx;
+  const int8_t* W_D;
+  const uint16_t* s_D;
+  const int8_t* U;
+  const uint16_t* s_U;
+  const int8_t* V;
+  const uint16_t* s_V;
+  const int8_t* x_q;
+  const float* x_scale;
+  const uint16_t* residual;
+  void* y;
+  int y_bf16;
+  int8_t* t_q_out;
+  float* t_scale_out;
+  void* workspace;
+  int num_sms;
+};
+size_t lowrank_workspace_bytes(int k_in, int n_out, int rank, int n_dense, int m);
+cudaError_t launch_lowrank_linear(const LowrankLaunch& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- quantisers / elementwise
+cudaError_t launch_quantize_latent(const float* v, int m, int r, int kind, int group, void* codes,
+                                   void* scales, cudaStream_t stream);
+// mode 0: quantise x; 1: RMSNorm then quantise; 2: SwiGLU(x, x2) then quantise
+cudaError_t launch_rowquant(int mode, const void* x, const void* x2, int x_bf16, int m, int k,
+                            float eps, int8_t* x_q, float* x_scale, cudaStream_t stream);
+
+// ---------------------------------------------------------------- generic int8 GEMM
+// C[m][n] = sum_k A[m][k] * B[n][k]  (int32), A, B row-major with given row strides (bytes)
+cudaError_t launch_gemm_i8(const int8_t* A, int lda, const int8_t* B, int ldb, int32_t* C, int ldc,
+                           int M, int N, int K, cudaStream_t stream);
+
+}  // namespace lk
+
+// Per-translation-unit device status words (see lk_common.cuh).
+cudaError_t lk_decode_status_word(unsigned int* value, int reset);
