@@ -152,7 +152,9 @@ size_t lk_latent_project_workspace_bytes(const lk_latent_cache* k_cache,
  * computed split-K over t (flash-decoding) with per-split partials
  * (max, sum, u) merged in latent space.  K and V are never formed.
  *
- * q: [B, n_heads, head_dim], q_dtype LK_F32 or LK_BF16.
+ * q: [B, n_heads, head_dim], q_dtype LK_F32 or LK_BF16; head_dim a multiple
+ *   of 8 (<= LK_MAX_HEAD_DIM); q, B_K and B_V 16-byte aligned (they are
+ *   staged into shared memory with bulk copies).
  * B_K, B_V: per-head factors [r_h, head_dim] row-major, packed head after
  *   head (head h starts at element sum_{h'<h} r_h' * head_dim); b_dtype
  *   LK_F32 or LK_BF16.

@@ -211,8 +211,10 @@ lk_status lk_latent_decode_attn(const lk_latent_cache* k, const lk_latent_cache*
   if (q_dtype != LK_F32 && q_dtype != LK_BF16) return fail(LK_ERR_DTYPE, "q dtype must be LK_F32 or LK_BF16");
   if (b_dtype != LK_F32 && b_dtype != LK_BF16) return fail(LK_ERR_DTYPE, "B dtype must be LK_F32 or LK_BF16");
   if (out_dtype != LK_F32 && out_dtype != LK_BF16) return fail(LK_ERR_DTYPE, "out dtype must be LK_F32 or LK_BF16");
-  if (head_dim < 1 || head_dim > LK_MAX_HEAD_DIM)
-    return fail(LK_ERR_SHAPE, "head_dim %d outside [1, %d]", head_dim, LK_MAX_HEAD_DIM);
+  if (head_dim < 8 || head_dim > LK_MAX_HEAD_DIM || head_dim % 8 != 0)
+    return fail(LK_ERR_SHAPE, "head_dim %d must be a multiple of 8 in [8, %d]", head_dim, LK_MAX_HEAD_DIM);
+  if (!aligned(q, 16) || !aligned(B_K, 16) || !aligned(B_V, 16))
+    return fail(LK_ERR_ALIGN, "q, B_K and B_V must be 16-byte aligned");
   if (max_seq_len < 0 || max_seq_len > k->capacity)
     return fail(LK_ERR_SHAPE, "max_seq_len %d outside [0, capacity]", max_seq_len);
   if (n_split < 0) return fail(LK_ERR_SHAPE, "n_split %d < 0", n_split);

@@ -44,6 +44,8 @@ struct DecodeParams {
   float qscale;  // softmax_scale * log2(e)
   // bytes of one pipeline stage region (max over heads), multiples of 128
   int st_kc, st_vc, st_ks, st_vs;
+  int st_q, st_bk, st_bv;  // bytes of the staged q / B_K / B_V regions
+  int q_size, b_size;      // element sizes of q and of the factors
   uint8_t rk[LK_MAX_HEADS];
   uint8_t rv[LK_MAX_HEADS];
 };
@@ -244,12 +246,16 @@ LK_DEVICE void accumulate_v(const uint8_t* vc, const uint8_t* vs, const HeadGeom
 struct SmemLayout {
   int stage_bytes;
   int off_kc, off_vc, off_ks, off_vs;  // within a stage
+  int off_q, off_bk, off_bv;           // q^h, B_K^h, B_V^h staged once per CTA
   int off_qt;                          // q~ [kMaxR] floats
   int off_red;                         // reduction scratch [4 warps][2 + kMaxR]
-  int off_bar;                         // mbarriers
+  int off_mw;                          // merge weights and sums [2][kMaxSplit]
+  int off_bar;                         // kStages stage barriers + 1 factor barrier
   int off_misc;
   int total;
 };
+
+constexpr int kMaxSplit = 256;
 
 LK_DEVICE SmemLayout smem_layout(const DecodeParams& p) {
   SmemLayout L;
@@ -258,23 +264,35 @@ LK_DEVICE SmemLayout smem_layout(const DecodeParams& p) {
   L.off_ks = p.st_kc + p.st_vc;
   L.off_vs = p.st_kc + p.st_vc + p.st_ks;
   L.stage_bytes = p.st_kc + p.st_vc + p.st_ks + p.st_vs;
-  L.off_qt = kStages * L.stage_bytes;
+  L.off_q = kStages * L.stage_bytes;
+  L.off_bk = L.off_q + p.st_q;
+  L.off_bv = L.off_bk + p.st_bk;
+  L.off_qt = L.off_bv + p.st_bv;
   L.off_red = L.off_qt + kMaxR * 4;
-  L.off_bar = L.off_red + 4 * (2 + kMaxR) * 4;
-  L.off_misc = L.off_bar + kStages * 8;
+  L.off_mw = L.off_red + 4 * (2 + kMaxR) * 4;
+  L.off_bar = L.off_mw + 2 * kMaxSplit * 4;
+  L.off_misc = L.off_bar + (kStages + 1) * 8;
   L.total = L.off_misc + 16;
   return L;
+}
+
+LK_DEVICE float ld_f(const uint8_t* base, int i, int is_bf16) {
+  return is_bf16 ? lk_bf16_to_f32(reinterpret_cast<const uint16_t*>(base)[i])
+                 : reinterpret_cast<const float*>(base)[i];
 }
 
 template <int KIND, int CSK, int CSV>
 LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* smem, const SmemLayout& L,
                            int b, int h, int split, int len, int first_stage, int n_my) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int H = p.head_dim;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.off_bar);
+  uint64_t* fbar = bars + kStages;
   float* qt_s = reinterpret_cast<float*>(smem + L.off_qt);
   float* red = reinterpret_cast<float*>(smem + L.off_red);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.off_misc);
   const int ssz = KIND == 0 ? 4 : 2;
+  const int64_t bh = (int64_t)b * p.n_heads + h;
 
   auto issue = [&](int j) {  // stage j of this split -> buffer j % kStages
     const int buf = j % kStages;
@@ -292,29 +310,31 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
   };
 
   if (tid == 0) {
+    // factors first: q^h, B_K^h (needed before the first token) and B_V^h (epilogue)
+    const uint32_t qb = H * p.q_size, bkb = g.rk * H * p.b_size, bvb = g.rv * H * p.b_size;
+    lk_mbar_arrive_expect_tx(fbar, qb + bkb + bvb);
+    lk_bulk_g2s(smem + L.off_q, static_cast<const uint8_t*>(p.q) + bh * H * p.q_size, qb, fbar);
+    lk_bulk_g2s(smem + L.off_bk, static_cast<const uint8_t*>(p.BK) + g.bk_off * p.b_size, bkb, fbar);
+    lk_bulk_g2s(smem + L.off_bv, static_cast<const uint8_t*>(p.BV) + g.bv_off * p.b_size, bvb, fbar);
     for (int j = 0; j < min(kStages, n_my); ++j) issue(j);
   }
 
-  // ---- absorb q: q~[i] = qscale * sum_d B_K[i][d] q[d]   (overlaps the first loads)
-  {
-    const int H = p.head_dim;
-    const int64_t qoff = ((int64_t)b * p.n_heads + h) * H;
+  bool aborted = false;
+  int stopped_at = 0;
+  // ---- absorb q: q~[i] = qscale * sum_d B_K[i][d] q[d]
+  if (!lk_mbar_wait_bounded(fbar, 0, LK_WAIT_LIMIT_NS)) *abort_flag = 1;
+  if (!*abort_flag) {
+    const uint8_t* qs = smem + L.off_q;
+    const uint8_t* bks = smem + L.off_bk;
     for (int i = warp; i < g.rk; i += kThreads / 32) {
       float acc = 0.0f;
-      for (int d = lane; d < H; d += 32) {
-        float qd, bkd;
-        if (p.q_bf16) qd = lk_bf16_to_f32(reinterpret_cast<const uint16_t*>(p.q)[qoff + d]);
-        else qd = reinterpret_cast<const float*>(p.q)[qoff + d];
-        const int64_t bi = g.bk_off + (int64_t)i * H + d;
-        if (p.b_bf16) bkd = lk_bf16_to_f32(reinterpret_cast<const uint16_t*>(p.BK)[bi]);
-        else bkd = reinterpret_cast<const float*>(p.BK)[bi];
-        acc = fmaf(qd, bkd, acc);
-      }
+      for (int d = lane; d < H; d += 32) acc = fmaf(ld_f(qs, d, p.q_bf16), ld_f(bks, i * H + d, p.b_bf16), acc);
       acc = lk_warp_sum(acc);
       if (lane == 0) qt_s[i] = acc * p.qscale;
     }
   }
   __syncthreads();
+  if (*abort_flag) aborted = true;
   float qt[kMaxR];
 #pragma unroll
   for (int i = 0; i < kMaxR; ++i) qt[i] = (i < g.rk) ? qt_s[i] : 0.0f;
@@ -324,9 +344,7 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
   for (int i = 0; i < kMaxR; ++i) u[i] = 0.0f;
   float m_run = -INFINITY, l_run = 0.0f;
 
-  bool aborted = false;
-  int stopped_at = 0;
-  for (int j = 0; j < n_my; ++j) {
+  for (int j = 0; j < n_my && !aborted; ++j) {
     const int buf = j % kStages;
     const bool ok = lk_mbar_wait_bounded(&bars[buf], (uint32_t)((j / kStages) & 1), LK_WAIT_LIMIT_NS);
     if (!ok) *abort_flag = 1;
@@ -355,8 +373,8 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
   if (aborted) {
     if (tid == 0) {
       lk_dev_fail(LK_DEV_TIMEOUT_PIPE);
-      // drain copies still in flight into this CTA's shared memory: stages
-      // stopped_at .. stopped_at + kStages - 1 were issued and not all waited for
+      // drain copies still in flight into this CTA's shared memory
+      if (!lk_mbar_wait_bounded(fbar, 0, LK_WAIT_LIMIT_NS)) lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
       for (int j = stopped_at; j < min(n_my, stopped_at + kStages); ++j) {
         if (!lk_mbar_wait_bounded(&bars[j % kStages], (uint32_t)((j / kStages) & 1), LK_WAIT_LIMIT_NS))
           lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
@@ -379,7 +397,6 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
     wred[0] = m_run;
     wred[1] = l_run;
   }
-  // lane i keeps u[i] and u[i + 32]; write them out with static indices
 #pragma unroll
   for (int i = 0; i < kMaxR; ++i) {
     if (i < g.rv && lane == (i & 31)) wred[2 + i] = u[i];
@@ -389,29 +406,21 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
   const int nw = kThreads / 32;
   float M = -INFINITY;
   for (int w = 0; w < nw; ++w) M = fmaxf(M, red[w * (2 + kMaxR)]);
-  // tid j < rv merges u_j; tid == rv (or a spare thread) merges l
-  float* cta = red;  // reuse warp 0's slot after reading; stage through registers first
+  // thread j < rv merges u_j; thread kMaxR merges l
+  float* cta = red;
   float mine = 0.0f;
-  if (M != -INFINITY) {
-    if (tid < g.rv) {
-      for (int w = 0; w < nw; ++w) {
-        const float mw = red[w * (2 + kMaxR)];
-        if (mw != -INFINITY) mine += red[w * (2 + kMaxR) + 2 + tid] * exp2f(mw - M);
-      }
-    } else if (tid == kMaxR) {
-      for (int w = 0; w < nw; ++w) {
-        const float mw = red[w * (2 + kMaxR)];
-        if (mw != -INFINITY) mine += red[w * (2 + kMaxR) + 1] * exp2f(mw - M);
-      }
+  const int idx = (tid < g.rv) ? 2 + tid : (tid == kMaxR ? 1 : -1);
+  if (M != -INFINITY && idx >= 0) {
+    for (int w = 0; w < nw; ++w) {
+      const float mw = red[w * (2 + kMaxR)];
+      if (mw != -INFINITY) mine += red[w * (2 + kMaxR) + idx] * exp2f(mw - M);
     }
   }
   __syncthreads();
-  if (tid < g.rv) cta[2 + tid] = mine;
-  if (tid == kMaxR) cta[1] = mine;
+  if (idx >= 0) cta[idx] = mine;
   if (tid == 0) cta[0] = M;
   __syncthreads();
 
-  const int64_t bh = (int64_t)b * p.n_heads + h;
   int* flag = reinterpret_cast<int*>(smem + L.off_misc) + 1;
   if (p.n_split > 1) {
     float* part = p.partials + (bh * p.n_split + split) * p.part_stride;
@@ -425,18 +434,29 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
     __syncthreads();
     if (!*flag) return;
     __threadfence();
-    // last arriver: merge every split's partial (all visible in L2)
+    // last arriver: merge every split's partial (all visible in L2), all
+    // splits' loads in flight at once
+    float* mw = reinterpret_cast<float*>(smem + L.off_mw);
+    const float* P0 = p.partials + bh * p.n_split * p.part_stride;
+    for (int s2 = tid; s2 < p.n_split; s2 += kThreads) mw[s2] = __ldcg(P0 + (int64_t)s2 * p.part_stride);
+    __syncthreads();
     float Mg = -INFINITY;
-    for (int s2 = 0; s2 < p.n_split; ++s2)
-      Mg = fmaxf(Mg, __ldcg(p.partials + (bh * p.n_split + s2) * p.part_stride));
+    for (int s2 = 0; s2 < p.n_split; ++s2) Mg = fmaxf(Mg, mw[s2]);
+    __syncthreads();
+    for (int s2 = tid; s2 < p.n_split; s2 += kThreads)
+      mw[s2] = (mw[s2] == -INFINITY || Mg == -INFINITY) ? 0.0f : exp2f(mw[s2] - Mg);
+    __syncthreads();
     float acc = 0.0f;
-    const int idx = (tid < g.rv) ? 2 + tid : (tid == kMaxR ? 1 : -1);
-    if (idx >= 0 && Mg != -INFINITY) {
-      for (int s2 = 0; s2 < p.n_split; ++s2) {
-        const float* ps = p.partials + (bh * p.n_split + s2) * p.part_stride;
-        const float ms = __ldcg(ps);
-        if (ms != -INFINITY) acc += __ldcg(ps + idx) * exp2f(ms - Mg);
+    if (idx >= 0) {
+      int s2 = 0;
+      for (; s2 + 4 <= p.n_split; s2 += 4) {
+        float v0 = __ldcg(P0 + (int64_t)(s2 + 0) * p.part_stride + idx);
+        float v1 = __ldcg(P0 + (int64_t)(s2 + 1) * p.part_stride + idx);
+        float v2 = __ldcg(P0 + (int64_t)(s2 + 2) * p.part_stride + idx);
+        float v3 = __ldcg(P0 + (int64_t)(s2 + 3) * p.part_stride + idx);
+        acc += v0 * mw[s2] + v1 * mw[s2 + 1] + v2 * mw[s2 + 2] + v3 * mw[s2 + 3];
       }
+      for (; s2 < p.n_split; ++s2) acc += __ldcg(P0 + (int64_t)s2 * p.part_stride + idx) * mw[s2];
     }
     __syncthreads();
     if (idx >= 0) cta[idx] = acc;
@@ -447,19 +467,14 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
     __syncthreads();
   }
 
-  // ---- out = (u / l) B_V^h
+  // ---- out = (u / l) B_V^h, B_V^h from shared memory
   const float lsum = cta[1];
-  const float inv = (cta[0] == -INFINITY || lsum == 0.0f) ? 0.0f : 1.0f / lsum;
-  const int H = p.head_dim;
+  const float inv = (cta[0] == -INFINITY || lsum == 0.0f || aborted) ? 0.0f : 1.0f / lsum;
+  const uint8_t* bvs = smem + L.off_bv;
   const int64_t ooff = bh * H;
   for (int d = tid; d < H; d += kThreads) {
     float o = 0.0f;
-    for (int j = 0; j < g.rv; ++j) {
-      const int64_t bi = g.bv_off + (int64_t)j * H + d;
-      const float bv = p.b_bf16 ? lk_bf16_to_f32(reinterpret_cast<const uint16_t*>(p.BV)[bi])
-                                : reinterpret_cast<const float*>(p.BV)[bi];
-      o = fmaf(cta[2 + j], bv, o);
-    }
+    for (int j = 0; j < g.rv; ++j) o = fmaf(cta[2 + j], ld_f(bvs, j * H + d, p.b_bf16), o);
     o *= inv;
     if (p.out_bf16) reinterpret_cast<uint16_t*>(p.out)[ooff + d] = lk_f32_to_bf16(o);
     else reinterpret_cast<float*>(p.out)[ooff + d] = o;
@@ -481,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const __grid_c
 
   if (threadIdx.x == 0) {
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.off_bar);
-    for (int i = 0; i < kStages; ++i) lk_mbar_init(&bars[i], 1);
+    for (int i = 0; i < kStages + 1; ++i) lk_mbar_init(&bars[i], 1);
     lk_fence_mbar_init();
     *reinterpret_cast<int*>(smem + L.off_misc) = 0;
   }
@@ -566,7 +581,7 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   const int stages = std::max(1, (a.max_len + kStageT - 1) / kStageT);
   int n_split = a.n_split;
   if (n_split <= 0) n_split = decode_pick_split(a.batch * a.n_heads, a.max_len, a.num_sms);
-  n_split = std::max(1, std::min(n_split, stages));
+  n_split = std::max(1, std::min(std::min(n_split, stages), kMaxSplit));
   p.stages_per_split = (stages + n_split - 1) / n_split;
   n_split = (stages + p.stages_per_split - 1) / p.stages_per_split;
   p.n_split = n_split;
@@ -575,8 +590,14 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   p.counters = reinterpret_cast<int32_t*>(ws);
   p.partials = reinterpret_cast<float*>(ws + round_up(a.batch * a.n_heads * 4, 256));
 
+  p.q_size = a.q_bf16 ? 2 : 4;
+  p.b_size = a.b_bf16 ? 2 : 4;
+  p.st_q = round_up(a.head_dim * p.q_size, 128);
+  p.st_bk = round_up(rk_max * a.head_dim * p.b_size, 128);
+  p.st_bv = round_up(rv_max * a.head_dim * p.b_size, 128);
   const int stage_bytes = p.st_kc + p.st_vc + p.st_ks + p.st_vs;
-  const int smem = kStages * stage_bytes + kMaxR * 4 + 4 * (2 + kMaxR) * 4 + kStages * 8 + 16;
+  const int smem = kStages * stage_bytes + p.st_q + p.st_bk + p.st_bv + kMaxR * 4 + 4 * (2 + kMaxR) * 4 +
+                   2 * kMaxSplit * 4 + (kStages + 1) * 8 + 16;
   dim3 grid(n_split, a.n_heads, a.batch);
   cudaError_t e;
   if (a.kind == 0) {

@@ -6,8 +6,15 @@ Comparison rules used by the GPU parity tests:
     (projection, RMSNorm, SwiGLU): equal, except a difference of exactly one
     where the oracle's ratio v/s lies within `band` of a rounding tie (k + 1/2)
     or where the row's scale itself differs by a few ulps;
-  * attention outputs: max |err| <= tol * RMS(oracle output) with tol 1e-5
-    for fp32 paths and 1e-2 for bf16 outputs.
+  * float outputs: max |err| <= tol * RMS(oracle output) with tol 1e-5 for
+    fp32 outputs and 1e-2 for bf16 outputs; a bf16 output additionally may
+    carry its own storage rounding, at most half a bf16 ulp, i.e.
+    2^-8 * |value| (assert_close_bf16).
+  * float32 latents summed in a different order (length-E dot products):
+    scales agree to a relative 1e-4 and codes may differ by one only within
+    2e-3 (in code units) of a rounding tie.  For these inputs the fp32
+    rounding of a length-E sum is about sqrt(E) * 2^-24 * sum|x a| / |v|,
+    below 1e-4 relative for E <= 4096.
 """
 from __future__ import annotations
 
@@ -59,13 +66,31 @@ def assert_close_rms(got, want, tol, what=""):
     return err / scale if scale else err
 
 
+def assert_close_bf16(got, want, tol=1e-2, what="", ulps=0.5):
+    """|got - want| <= tol * RMS(want) + ulps * 2^-7 |want|.
+
+    2^-7 |v| bounds one bf16 ulp of v, so the default allows the output's own
+    rounding (half an ulp); chained stages that re-store bf16 values pass ulps=1."""
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    assert got.shape == want.shape, (got.shape, want.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    scale = rms(want)
+    err = np.abs(got - want)
+    allowed = tol * scale + ulps * 2.0 ** -7 * np.abs(want)
+    worst = int(np.argmax(err - allowed))
+    assert np.all(err <= allowed), (f"{what}: |err| {err.flat[worst]:.3e} > {allowed.flat[worst]:.3e} "
+                                    f"at value {want.flat[worst]:.3e} (RMS {scale:.3e})")
+    return float(np.max(err)) / scale if scale else float(np.max(err))
+
+
 def f32_ulp_diff(a, b):
     a = np.asarray(a, np.float32).view(np.int32).astype(np.int64)
     b = np.asarray(b, np.float32).view(np.int32).astype(np.int64)
     return np.abs(a - b)
 
 
-def check_codes_band(gpu_codes, gpu_scale, v32, kind="i8", group=32, band=1e-3, scale_ulps=4):
+def check_codes_band(gpu_codes, gpu_scale, v32, kind="i8", group=32, band=2e-3, scale_rel=1e-4):
     """Compare device codes (unpacked, [n, r]) and scales against the oracle
     quantisation of the oracle's own float32 values v32 [n, r].
 
@@ -75,8 +100,8 @@ def check_codes_band(gpu_codes, gpu_scale, v32, kind="i8", group=32, band=1e-3, 
         oc, os_ = O.quantize_i8(v32)
         s_or = os_.astype(np.float64)[:, None]
         s_gpu = np.asarray(gpu_scale, np.float32)
-        ulps = f32_ulp_diff(s_gpu, os_)
-        assert np.all(ulps <= scale_ulps), f"scale differs by {ulps.max()} ulp"
+        rel = np.abs(s_gpu.astype(np.float64) - os_) / np.maximum(os_.astype(np.float64), 1e-45)
+        assert np.all(rel <= scale_rel), f"scale differs by {rel.max():.2e} relative"
         s_gpu_b = np.broadcast_to(s_gpu.astype(np.float64)[:, None], v32.shape)
     else:
         oc, os_ = O.quantize_i4(v32, group)

@@ -76,6 +76,8 @@ def test_decode_validation(L):
     assert decode(L, k, cache(L, kind=L.LK_I4)) == L.LK_ERR_UNSUPPORTED
     assert decode(L, k, v, max_len=65) == L.LK_ERR_SHAPE                      # beyond capacity
     assert decode(L, k, v, H=0) == L.LK_ERR_SHAPE
+    assert decode(L, k, v, H=60) == L.LK_ERR_SHAPE                           # not a multiple of 8
+    assert decode(L, k, v, q=FAKE + 0x300008) == L.LK_ERR_ALIGN
     assert decode(L, k, v, H=300) == L.LK_ERR_SHAPE
     assert decode(L, k, v, q=0) == L.LK_ERR_INVALID_ARG
     assert decode(L, k, v, qdt=L.LK_I8) == L.LK_ERR_DTYPE
