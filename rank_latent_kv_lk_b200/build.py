@@ -1,6 +1,7 @@
 """Builds liblk.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-Usage: python -m rank_latent_kv_lk_b200.build [--force] [--verbose]
+Usage: python rank_latent_kv_lk_b200/build.py [--force] [--verbose] [--ptxas-info]
+(run as a script: importing the package would load the library it builds).
 
 Each .cu file compiles to an object under ``_build/`` (in parallel), then the
 objects link into ``rank_latent_kv_lk_b200/liblk.so``.  Objects are rebuilt

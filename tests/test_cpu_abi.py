@@ -16,8 +16,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def L():
-    from rank_latent_kv_lk_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     from rank_latent_kv_lk_b200 import _lib
     return _lib
 
