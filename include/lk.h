@@ -180,6 +180,37 @@ size_t lk_latent_decode_workspace_bytes(const lk_latent_cache* k_cache,
                                         int32_t n_split);
 
 /*
+ * Latent decode attention for callers that cannot allocate device memory
+ * (no counterpart in the paper).  Some callers cannot call cudaMalloc or
+ * hand out scratch buffers -- for example code running under an allocator
+ * that forbids new device allocations, or a host runtime that only passes
+ * tensors it already owns.  This variant takes the same arguments as
+ * lk_latent_decode_attn minus the workspace and keeps its split-K scratch
+ * (arrival counters + per-split partials) in a static device array of
+ * LK_DECODE_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that
+ * loads the library holds until the process exits.  It allocates nothing
+ * and calls no allocating routine; inputs and outputs are still the
+ * caller's.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - A request whose scratch would exceed LK_DECODE_NOALLOC_SCRATCH_BYTES is
+ *    rejected with LK_ERR_WORKSPACE (lk_last_error says how much it needs);
+ *    lower n_split or use lk_latent_decode_attn with a workspace.
+ *  - All calls share the one array: calls that overlap on the GPU (other
+ *    streams, other host threads) race on it.  Serialise them.
+ *  - The counters start at zero when the library loads; after each launch
+ *    the call clears them again on `stream`.
+ */
+#define LK_DECODE_NOALLOC_SCRATCH_BYTES (4u << 20)
+lk_status lk_latent_decode_attn_noalloc(const lk_latent_cache* k_cache, const lk_latent_cache* v_cache,
+                                        const void* q, lk_dtype q_dtype, const void* B_K,
+                                        const void* B_V, lk_dtype b_dtype, int32_t head_dim,
+                                        const int32_t* seq_len, int32_t max_seq_len,
+                                        float softmax_scale, void* out, lk_dtype out_dtype,
+                                        int32_t n_split, lk_stream_t stream);
+
+/*
  * LASER hybrid dense + low-rank linear, W8A8 (LASER technical summary §3:
  * selected input channels go through SVD factors, the rest stay dense; both
  * branches RTN-quantised).

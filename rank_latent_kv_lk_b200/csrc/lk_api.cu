@@ -80,6 +80,14 @@ size_t decode_ws_bytes(const lk_latent_cache* k, const lk_latent_cache* v, int m
 
 }  // namespace
 
+namespace lk {
+// Records an error for lk_last_error() from another translation unit.
+lk_status set_error(lk_status s, const char* msg) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
+  return s;
+}
+}  // namespace lk
+
 extern "C" {
 
 int32_t lk_version(void) { return 1; }

@@ -613,3 +613,88 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
 }
 
 }  // namespace lk
+
+// ---------------------------------------------------------------- allocation-free variant
+// Split-K scratch for lk_latent_decode_attn_noalloc: a file-scope device
+// array (zero at load), so callers that cannot allocate need no workspace.
+// Host code must not hand its name to a kernel (in host code it is only a
+// stand-in); the device address is looked up once per device below.
+#include <cstdio>
+#include <mutex>
+
+namespace lk {
+lk_status set_error(lk_status s, const char* msg);
+}
+
+static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[LK_DECODE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+}  // namespace
+
+extern "C" lk_status lk_latent_decode_attn_noalloc(const lk_latent_cache* k, const lk_latent_cache* v,
+                                                   const void* q, lk_dtype q_dtype, const void* B_K,
+                                                   const void* B_V, lk_dtype b_dtype, int32_t head_dim,
+                                                   const int32_t* seq_len, int32_t max_seq_len,
+                                                   float softmax_scale, void* out, lk_dtype out_dtype,
+                                                   int32_t n_split, lk_stream_t stream) {
+  char msg[256];
+  // enough of the arguments to size the scratch; lk_latent_decode_attn checks the rest
+  if (!k || !v || !k->ranks || !v->ranks) return lk::set_error(LK_ERR_INVALID_ARG, "null cache descriptor or ranks");
+  if (k->batch < 1 || k->n_heads < 1 || k->n_heads > LK_MAX_HEADS || v->n_heads != k->n_heads ||
+      v->batch != k->batch || max_seq_len < 0 || n_split < 0)
+    return lk::set_error(LK_ERR_SHAPE, "bad batch, heads, max_seq_len or n_split");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) {
+    snprintf(msg, sizeof(msg), "lk_latent_decode_attn_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+    return lk::set_error(LK_ERR_CUDA, msg);
+  }
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      // once per device, with that device current
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_decode_noalloc_scratch);
+      if (e != cudaSuccess || !p) {
+        snprintf(msg, sizeof(msg), "lk_latent_decode_attn_noalloc: cudaGetSymbolAddress: %s",
+                 cudaGetErrorString(e));
+        return lk::set_error(LK_ERR_CUDA, msg);
+      }
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  int rv_max = 0;
+  for (int h = 0; h < v->n_heads; ++h) rv_max = std::max(rv_max, (int)v->ranks[h]);
+  int num_sms = 0;
+  if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || num_sms <= 0)
+    num_sms = 148;
+  const int stages = std::max(1, (max_seq_len + kStageT - 1) / kStageT);
+  int n_eff = n_split > 0 ? std::min(n_split, stages) : lk::decode_pick_split(k->batch * k->n_heads, max_seq_len, num_sms);
+  n_eff = std::max(1, std::min(std::min(n_eff, stages), kMaxSplit));
+  const size_t need = lk::decode_workspace_bytes(k->batch, k->n_heads, rv_max, n_eff);
+  if (need > LK_DECODE_NOALLOC_SCRATCH_BYTES) {
+    snprintf(msg, sizeof(msg),
+             "lk_latent_decode_attn_noalloc: needs %zu bytes of scratch, the static array holds %u; "
+             "lower n_split or use lk_latent_decode_attn with a workspace",
+             need, (unsigned)LK_DECODE_NOALLOC_SCRATCH_BYTES);
+    return lk::set_error(LK_ERR_WORKSPACE, msg);
+  }
+  const lk_status st = lk_latent_decode_attn(k, v, q, q_dtype, B_K, B_V, b_dtype, head_dim, seq_len, max_seq_len,
+                                             softmax_scale, out, out_dtype, n_eff, scratch,
+                                             LK_DECODE_NOALLOC_SCRATCH_BYTES, stream);
+  if (st != LK_OK) return st;
+  // leave the arrival counters zero for the next call (the kernel already does;
+  // this also covers a call cut short)
+  const size_t counters = (size_t)((k->batch * k->n_heads * 4 + 255) / 256 * 256);
+  e = cudaMemsetAsync(scratch, 0, counters, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    snprintf(msg, sizeof(msg), "lk_latent_decode_attn_noalloc: clearing counters: %s", cudaGetErrorString(e));
+    return lk::set_error(LK_ERR_CUDA, msg);
+  }
+  return LK_OK;
+}
