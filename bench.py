@@ -150,7 +150,7 @@ class DecodeState:
         A, BK, BV = synth.factors(w, 0, self.rk, self.rv)
         self.A, self.BK, self.BV = A.to(device), BK.to(device), BV.to(device)
         self.ck = lk.LatentCache(w.batch, self.rk, w.capacity, w.kind, w.group, device)
-        self.cv = lk.LatentCache(w.batch, self.rv, w.capacity, w.kind, w.group, device)
+        self.cv = lk.LatentCache(w.batch, self.rv, w.capacity, w.kind, w.group, device, role="v")
         self.seq = torch.zeros(w.batch, dtype=torch.int32, device=device)
         x_ctx = synth.context_tokens(w, 0).to(device)
         lk.latent_project_append(self.ck, self.cv, x_ctx.reshape(-1, w.embed_dim), self.A, self.seq,

@@ -84,11 +84,17 @@ typedef enum {
  *
  * codes: for batch row b and head h, one contiguous plane of capacity * rb_h
  *   bytes at byte offset (b * sum_h rb_h + sum_{h' < h} rb_h') * capacity.
- *   Inside a plane, tokens are kept in blocks of 16; with chunk size
- *   cs = 16 if rb % 16 == 0, else 8 if rb % 8 == 0, else 4, byte k of token
- *   t's code row sits at
- *       (t / 16) * 16 * rb + (k / cs) * 16 * cs + (t % 16) * cs + (k % cs).
- *   (Thread-per-token readers then touch consecutive 16-byte words.)
+ *   Inside a plane, tokens are kept in blocks of 16 (16 * rb bytes each);
+ *   the order inside a block depends on the cache's role:
+ *   K caches (token-major chunks): with chunk size cs = 16 if rb % 16 == 0,
+ *     else 8 if rb % 8 == 0, else 4, byte k of token t's code row sits at
+ *       (t / 16) * 16 * rb + (k / cs) * 16 * cs + (t % 16) * cs + (k % cs)
+ *     (a reader with one thread per token touches consecutive words);
+ *   V caches (dimension-major): int8: the code of dim d of token t sits at
+ *       (t / 16) * 16 * rb + d * 16 + (t % 16);
+ *     int4: byte (t / 16) * 16 * rb + d * 8 + (t % 16) / 2 holds dim d of
+ *     tokens 2i (low nibble) and 2i + 1 (high nibble)
+ *     (one 32-bit word then holds 4 or 8 consecutive tokens of one dim).
  * scales: int8: fp32 [capacity] per (b, h) at element offset
  *   (b * n_heads + h) * capacity.  int4: fp16 [capacity][ng_h] per (b, h)
  *   at element offset (b * sum_h ng_h + sum_{h' < h} ng_h') * capacity.

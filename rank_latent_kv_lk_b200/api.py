@@ -57,10 +57,12 @@ workspaces = _WorkspacePool()
 class LatentCache:
     """Device latent cache of one layer for K or V (codes + scales planes)."""
 
-    def __init__(self, batch, ranks, capacity, kind="i8", group=32, device="cuda"):
+    def __init__(self, batch, ranks, capacity, kind="i8", group=32, device="cuda", role="k"):
+        """role: 'k' or 'v' -- the two caches of a layer lay codes out differently."""
         if kind not in ("i8", "i4"):
             raise ValueError("kind must be 'i8' or 'i4'")
-        self.geom = CacheGeometry(batch, ranks, capacity, kind, group)
+        self.role = role
+        self.geom = CacheGeometry(batch, ranks, capacity, kind, group, role)
         self.batch, self.ranks, self.capacity, self.kind, self.group = batch, list(ranks), capacity, kind, group
         self.codes = torch.zeros(self.geom.codes_bytes, dtype=torch.uint8, device=device)
         self.scales = torch.zeros(self.geom.scales_elems,

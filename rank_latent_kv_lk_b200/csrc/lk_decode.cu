@@ -1,29 +1,41 @@
 // Latent decode attention, split-K over the sequence (sm_100a).
 //
 // Per (batch row b, head h, split s) one CTA of 128 threads:
-//   1. absorbs q into latent space: q~ = B_K^h q * softmax_scale * log2(e)
+//   1. absorbs q into latent space, q~ = B_K^h q * softmax_scale * log2(e)
 //      (WSVD page §2C: the fused kernel works from the per-head latents;
-//      without positional rotation (q B_K^T) C^T equals q K^T);
+//      without positional rotation (q B_K^T) C^T equals q K^T), and writes
+//      q~ as a three-term int8 expansion q~ = a (t0 + t1/254 + t2/254^2)
+//      (error <= 6e-8 of max|q~|, i.e. float32 level);
 //   2. streams its slice of the latent cache (K codes, V codes and their
 //      scales) HBM -> shared memory with bulk copies on the TMA engine,
-//      4 stages deep, one mbarrier per stage;
-//   3. one token per thread per stage: score = sigma_K . (c_K . q~), a
-//      warp-uniform running max, p = 2^(score - max), and
-//      u += p * sigma_V * c_V in registers (r_V values);
-//   4. reduces (max, sum, u) over the CTA and writes it as a partial in
-//      latent space; the last CTA of the (b, h) to arrive (atomic ticket, no
-//      waiting) merges all partials and applies out = (u / sum) B_V^h.
-// K and V are never formed; the only per-token traffic is the latent codes
-// and their scales.
+//      kStages deep, one mbarrier per stage;
+//   3. per stage of 128 tokens:
+//      a. one token per thread: s_t = sigma_K (c_K . q~) with exact int32
+//         dp4a dot products against the expansion;
+//      b. a CTA-uniform running max, p_t = 2^(s_t - max), running sum;
+//      c. u += p_t sigma_V c_V: the stage's weights w_t = p_t sigma_V[t] are
+//         written as a three-term int8 expansion relative to the stage max
+//         (error <= 6e-8 of it), and each lane takes exact int32 dp4a sums
+//         over 4 (int8) or 8 (int4) tokens of one latent dim at a time from the
+//         dimension-major V layout; one float fold per stage;
+//   4. reduces (max, sum, u) over the CTA into a partial in latent space; the
+//      last CTA of the (b, h) to arrive (atomic ticket, no waiting) merges
+//      all partials and applies out = (u / sum) B_V^h.
+// K and V are never formed; the per-token traffic is the latent codes and
+// their scales.
 #include "lk_common.cuh"
 #include "lk_internal.h"
 
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kStageT = 128;  // tokens per pipeline stage: one per thread
-constexpr int kStages = 4;
+constexpr int kWarps = kThreads / 32;
+constexpr int kStageT = 128;  // tokens per pipeline stage: one per thread in the score phase
+constexpr int kStages = 3;
 constexpr int kMaxR = LK_MAX_RANK;
+constexpr int kMaxWords = kMaxR / 4;  // 32-bit words of q~ terms (int8 per dim)
+constexpr int kMaxGroups = 8;
+constexpr int kMaxSplit = 256;
 
 struct DecodeParams {
   const uint8_t* codes_k;
@@ -42,10 +54,10 @@ struct DecodeParams {
   int q_bf16, b_bf16, out_bf16;
   int n_split, stages_per_split, part_stride, max_len;
   float qscale;  // softmax_scale * log2(e)
-  // bytes of one pipeline stage region (max over heads), multiples of 128
+  // bytes of the shared-memory regions (max over heads), multiples of 128
   int st_kc, st_vc, st_ks, st_vs;
-  int st_q, st_bk, st_bv;  // bytes of the staged q / B_K / B_V regions
-  int q_size, b_size;      // element sizes of q and of the factors
+  int st_q, st_bk, st_bv;
+  int q_size, b_size;  // element sizes of q and of the factors
   uint8_t rk[LK_MAX_HEADS];
   uint8_t rv[LK_MAX_HEADS];
 };
@@ -112,8 +124,8 @@ LK_DEVICE HeadGeom head_geometry(const DecodeParams& p, int b, int h) {
   return g;
 }
 
-// Loads the code row chunk `c` (CS bytes) of local token `tl` from a staged
-// region laid out in 16-token blocks.
+// Loads the code chunk `c` (CS bytes) of local token `tl` from a staged
+// region laid out in 16-token blocks (chunk-major inside a block).
 template <int CS>
 struct Chunk;
 template <>
@@ -140,11 +152,18 @@ struct Chunk<4> {
   }
 };
 
-// Dims covered by one 32-bit word of codes.
-template <int KIND>
-struct DimsPerWord { static constexpr int v = KIND == 0 ? 4 : 8; };
+LK_DEVICE float load_scale(const uint8_t* base, int i, int kind) {
+  return kind == 0 ? reinterpret_cast<const float*>(base)[i]
+                   : lk_f16_to_f32(reinterpret_cast<const uint16_t*>(base)[i]);
+}
 
-// Expands word `wd` of codes into fp32 values (exact integers).
+LK_DEVICE float ld_f(const uint8_t* base, int i, int is_bf16) {
+  return is_bf16 ? lk_bf16_to_f32(reinterpret_cast<const uint16_t*>(base)[i])
+                 : reinterpret_cast<const float*>(base)[i];
+}
+
+// Expands code word `wd` into fp32 values: 4 signed bytes (int8) or 8 signed
+// nibbles (int4, low nibble = even dim).  Exact integers.
 template <int KIND>
 LK_DEVICE void expand_word(uint32_t wd, float* f) {
   if (KIND == 0) {
@@ -163,22 +182,30 @@ LK_DEVICE void expand_word(uint32_t wd, float* f) {
   }
 }
 
-LK_DEVICE float load_scale(const uint8_t* base, int i, int kind) {
-  return kind == 0 ? reinterpret_cast<const float*>(base)[i]
-                   : lk_f16_to_f32(reinterpret_cast<const uint16_t*>(base)[i]);
+// Signed int4 nibbles of a word as signed int8 bytes: `ev` gets the low
+// nibbles (elements 0, 2, 4, 6), `od` the high ones (1, 3, 5, 7).  Setting
+// the upper half of a byte whose bit 3 is set is one multiply: 0x08 * 0x1E =
+// 0xF0 stays inside its byte.
+LK_DEVICE void nibbles_to_s8(uint32_t x, int& ev, int& od) {
+  const uint32_t e = x & 0x0F0F0F0Fu, o = (x >> 4) & 0x0F0F0F0Fu;
+  ev = (int)(e | ((e & 0x08080808u) * 0x1Eu));
+  od = (int)(o | ((o & 0x08080808u) * 0x1Eu));
 }
 
-// Score of one token: sum over groups of sigma_g * (c . q~) restricted to the group.
+constexpr float kInv254 = 1.0f / 254.0f;
+constexpr float kInv254sq = 1.0f / (254.0f * 254.0f);
+
+// Score of one token in log2 units: sum over groups g of
+//   sigma_g * a * (D0 + D1/254 + D2/254^2),  D_i = c . t_i  (exact dp4a sums)
+// (int8 keys: one group and one scale per token).
 template <int KIND, int CS>
 LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom& g, int tl,
-                            const float* qt) {
-  constexpr int DPW = DimsPerWord<KIND>::v;
-  constexpr int WPC = CS / 4;                   // words per chunk
+                            const uint32_t (&qw)[3][kMaxWords], float qa) {
+  constexpr int WPC = CS / 4;  // words per chunk
   constexpr int MAXCH = (KIND == 0 ? kMaxR : kMaxR / 2) / CS;
   const int nch = g.rbk / CS;
-  float s = 0.0f;
   if (KIND == 0) {
-    float acc = 0.0f;
+    int d0 = 0, d1 = 0, d2 = 0;
 #pragma unroll
     for (int c = 0; c < MAXCH; ++c) {
       if (c < nch) {
@@ -186,15 +213,20 @@ LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom
         ch.load(kc, g.rbk, tl, c);
 #pragma unroll
         for (int wi = 0; wi < WPC; ++wi) {
-          float f[4];
-          expand_word<0>(ch.w[wi], f);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) acc = fmaf(f[k], qt[(c * WPC + wi) * DPW + k], acc);
+          const int w = c * WPC + wi;
+          d0 = __dp4a((int)ch.w[wi], (int)qw[0][w], d0);
+          d1 = __dp4a((int)ch.w[wi], (int)qw[1][w], d1);
+          d2 = __dp4a((int)ch.w[wi], (int)qw[2][w], d2);
         }
       }
     }
-    s = acc * reinterpret_cast<const float*>(ks)[tl];
+    const float x = fmaf((float)d2, kInv254sq, fmaf((float)d1, kInv254, (float)d0));
+    return reinterpret_cast<const float*>(ks)[tl] * (qa * x);
   } else {
+    float s = 0.0f;
+    int d0 = 0, d1 = 0, d2 = 0;
+    int cur_g = 0;
+    // code word w holds dims 8w .. 8w+7; groups are multiples of 8 dims
 #pragma unroll
     for (int c = 0; c < MAXCH; ++c) {
       if (c < nch) {
@@ -202,44 +234,24 @@ LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom
         ch.load(kc, g.rbk, tl, c);
 #pragma unroll
         for (int wi = 0; wi < WPC; ++wi) {
-          float f[8];
-          expand_word<1>(ch.w[wi], f);
-          float acc = 0.0f;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) acc = fmaf(f[k], qt[(c * WPC + wi) * DPW + k], acc);
-          const int dim0 = (c * WPC + wi) * DPW;
-          s = fmaf(acc, load_scale(ks, tl * g.ngk + dim0 / g.gk, 1), s);
+          const int w = c * WPC + wi;
+          const int gw = (8 * w) / g.gk;
+          if (gw != cur_g) {  // flush the finished group (uniform branch)
+            const float x = fmaf((float)d2, kInv254sq, fmaf((float)d1, kInv254, (float)d0));
+            s = fmaf(load_scale(ks, tl * g.ngk + cur_g, 1), qa * x, s);
+            d0 = d1 = d2 = 0;
+            cur_g = gw;
+          }
+          int ev, od;
+          nibbles_to_s8(ch.w[wi], ev, od);
+          d0 = __dp4a(od, (int)qw[0][2 * w + 1], __dp4a(ev, (int)qw[0][2 * w], d0));
+          d1 = __dp4a(od, (int)qw[1][2 * w + 1], __dp4a(ev, (int)qw[1][2 * w], d1));
+          d2 = __dp4a(od, (int)qw[2][2 * w + 1], __dp4a(ev, (int)qw[2][2 * w], d2));
         }
       }
     }
-  }
-  return s;
-}
-
-// u += w * sigma_V * c_V for one token.
-template <int KIND, int CS>
-LK_DEVICE void accumulate_v(const uint8_t* vc, const uint8_t* vs, const HeadGeom& g, int tl,
-                            float p, float* u) {
-  constexpr int DPW = DimsPerWord<KIND>::v;
-  constexpr int WPC = CS / 4;
-  constexpr int MAXCH = (KIND == 0 ? kMaxR : kMaxR / 2) / CS;
-  const int nch = g.rbv / CS;
-  const float w0 = KIND == 0 ? p * reinterpret_cast<const float*>(vs)[tl] : 0.0f;
-#pragma unroll
-  for (int c = 0; c < MAXCH; ++c) {
-    if (c < nch) {
-      Chunk<CS> ch;
-      ch.load(vc, g.rbv, tl, c);
-#pragma unroll
-      for (int wi = 0; wi < WPC; ++wi) {
-        float f[DPW];
-        expand_word<KIND>(ch.w[wi], f);
-        const int dim0 = (c * WPC + wi) * DPW;
-        const float w = KIND == 0 ? w0 : p * load_scale(vs, tl * g.ngv + dim0 / g.gv, 1);
-#pragma unroll
-        for (int k = 0; k < DPW; ++k) u[dim0 + k] = fmaf(w, f[k], u[dim0 + k]);
-      }
-    }
+    const float x = fmaf((float)d2, kInv254sq, fmaf((float)d1, kInv254, (float)d0));
+    return fmaf(load_scale(ks, tl * g.ngk + cur_g, 1), qa * x, s);
   }
 }
 
@@ -248,14 +260,21 @@ struct SmemLayout {
   int off_kc, off_vc, off_ks, off_vs;  // within a stage
   int off_q, off_bk, off_bv;           // q^h, B_K^h, B_V^h staged once per CTA
   int off_qt;                          // q~ [kMaxR] floats
-  int off_red;                         // reduction scratch [4 warps][2 + kMaxR]
-  int off_mw;                          // merge weights and sums [2][kMaxSplit]
+  int off_qterm;                       // q~ expansion bytes [3][kMaxR]
+  int off_smax;                        // per-warp stage max [kWarps]
+  int off_wmx;                         // per-warp, per-group weight max [kWarps][kMaxGroups]
+  int off_tw;                          // weight expansion bytes [kMaxGroups][3][kStageT]
+  int off_cta;                         // CTA partial [2 + kMaxR]
+  int off_lred;                        // [kWarps]
+  int off_mw;                          // merge weights [kMaxSplit]
   int off_bar;                         // kStages stage barriers + 1 factor barrier
   int off_misc;
   int total;
 };
 
-constexpr int kMaxSplit = 256;
+constexpr int kSmemFixed = kMaxR * 4 + 3 * kMaxR + kWarps * 4 + kWarps * kMaxGroups * 4 +
+                           kMaxGroups * 3 * kStageT + (2 + kMaxR) * 4 + kWarps * 4 + kMaxSplit * 4 +
+                           (kStages + 1) * 8 + 16;
 
 LK_DEVICE SmemLayout smem_layout(const DecodeParams& p) {
   SmemLayout L;
@@ -268,17 +287,22 @@ LK_DEVICE SmemLayout smem_layout(const DecodeParams& p) {
   L.off_bk = L.off_q + p.st_q;
   L.off_bv = L.off_bk + p.st_bk;
   L.off_qt = L.off_bv + p.st_bv;
-  L.off_red = L.off_qt + kMaxR * 4;
-  L.off_mw = L.off_red + 4 * (2 + kMaxR) * 4;
-  L.off_bar = L.off_mw + 2 * kMaxSplit * 4;
+  L.off_qterm = L.off_qt + kMaxR * 4;
+  L.off_smax = L.off_qterm + 3 * kMaxR;
+  L.off_wmx = L.off_smax + kWarps * 4;
+  L.off_tw = L.off_wmx + kWarps * kMaxGroups * 4;
+  L.off_cta = L.off_tw + kMaxGroups * 3 * kStageT;
+  L.off_lred = L.off_cta + (2 + kMaxR) * 4;
+  L.off_mw = L.off_lred + kWarps * 4;
+  L.off_bar = L.off_mw + kMaxSplit * 4;
   L.off_misc = L.off_bar + (kStages + 1) * 8;
   L.total = L.off_misc + 16;
   return L;
 }
 
-LK_DEVICE float ld_f(const uint8_t* base, int i, int is_bf16) {
-  return is_bf16 ? lk_bf16_to_f32(reinterpret_cast<const uint16_t*>(base)[i])
-                 : reinterpret_cast<const float*>(base)[i];
+inline int smem_bytes_for(const DecodeParams& p) {
+  const int stage = p.st_kc + p.st_vc + p.st_ks + p.st_vs;
+  return kStages * stage + p.st_q + p.st_bk + p.st_bv + kSmemFixed;
 }
 
 template <int KIND, int CSK, int CSV>
@@ -289,8 +313,15 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.off_bar);
   uint64_t* fbar = bars + kStages;
   float* qt_s = reinterpret_cast<float*>(smem + L.off_qt);
-  float* red = reinterpret_cast<float*>(smem + L.off_red);
+  int8_t* qterm = reinterpret_cast<int8_t*>(smem + L.off_qterm);
+  float* smax = reinterpret_cast<float*>(smem + L.off_smax);
+  float* wmx = reinterpret_cast<float*>(smem + L.off_wmx);
+  int8_t* tw = reinterpret_cast<int8_t*>(smem + L.off_tw);
+  float* cta = reinterpret_cast<float*>(smem + L.off_cta);
+  float* lred = reinterpret_cast<float*>(smem + L.off_lred);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.off_misc);
+  int* flag = reinterpret_cast<int*>(smem + L.off_misc) + 1;
+  float* qa_s = reinterpret_cast<float*>(smem + L.off_misc) + 2;
   const int ssz = KIND == 0 ? 4 : 2;
   const int64_t bh = (int64_t)b * p.n_heads + h;
 
@@ -310,7 +341,7 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
   };
 
   if (tid == 0) {
-    // factors first: q^h, B_K^h (needed before the first token) and B_V^h (epilogue)
+    // factors first: q^h and B_K^h (needed before the first token), B_V^h (epilogue)
     const uint32_t qb = H * p.q_size, bkb = g.rk * H * p.b_size, bvb = g.rv * H * p.b_size;
     lk_mbar_arrive_expect_tx(fbar, qb + bkb + bvb);
     lk_bulk_g2s(smem + L.off_q, static_cast<const uint8_t*>(p.q) + bh * H * p.q_size, qb, fbar);
@@ -326,7 +357,7 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
   if (!*abort_flag) {
     const uint8_t* qs = smem + L.off_q;
     const uint8_t* bks = smem + L.off_bk;
-    for (int i = warp; i < g.rk; i += kThreads / 32) {
+    for (int i = warp; i < g.rk; i += kWarps) {
       float acc = 0.0f;
       for (int d = lane; d < H; d += 32) acc = fmaf(ld_f(qs, d, p.q_bf16), ld_f(bks, i * H + d, p.b_bf16), acc);
       acc = lk_warp_sum(acc);
@@ -334,14 +365,49 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
     }
   }
   __syncthreads();
+  // ---- three-term int8 expansion of q~ (warp 0): q~ = a (t0 + t1/254 + t2/254^2)
+  if (warp == 0) {
+    const float v0 = lane < g.rk ? qt_s[lane] : 0.0f;
+    const float v1 = lane + 32 < g.rk ? qt_s[lane + 32] : 0.0f;
+    const float amax = lk_warp_max(fmaxf(fabsf(v0), fabsf(v1)));
+    const float a = amax / 127.0f;
+    const float inva = amax > 0.0f ? 127.0f / amax : 0.0f;
+    int tv[2][3];
+#pragma unroll
+    for (int q2 = 0; q2 < 2; ++q2) {
+      const float x = (q2 == 0 ? v0 : v1) * inva;
+      const float t0 = rintf(x);
+      const float x1 = (x - t0) * 254.0f;
+      const float t1 = rintf(x1);
+      const float x2 = (x1 - t1) * 254.0f;
+      const float t2 = fminf(fmaxf(rintf(x2), -127.0f), 127.0f);
+      tv[q2][0] = (int)t0; tv[q2][1] = (int)t1; tv[q2][2] = (int)t2;
+      const int d = lane + 32 * q2;
+      if (d < kMaxR) {
+        // int4 keys meet even dims and odd dims in separate words
+        const int pos = KIND == 0 ? d : ((d >> 3) << 3) + ((d & 1) ? 4 : 0) + ((d & 7) >> 1);
+        const bool live = d < g.rk;
+        qterm[0 * kMaxR + pos] = (int8_t)(live ? tv[q2][0] : 0);
+        qterm[1 * kMaxR + pos] = (int8_t)(live ? tv[q2][1] : 0);
+        qterm[2 * kMaxR + pos] = (int8_t)(live ? tv[q2][2] : 0);
+      }
+    }
+    if (lane == 0) *qa_s = a;
+  }
+  __syncthreads();
   if (*abort_flag) aborted = true;
-  float qt[kMaxR];
+  const float qa = *qa_s;
+  uint32_t qw[3][kMaxWords];
 #pragma unroll
-  for (int i = 0; i < kMaxR; ++i) qt[i] = (i < g.rk) ? qt_s[i] : 0.0f;
+  for (int i = 0; i < 3; ++i)
+#pragma unroll
+    for (int w = 0; w < kMaxWords; ++w) qw[i][w] = reinterpret_cast<const uint32_t*>(qterm + i * kMaxR)[w];
 
-  float u[kMaxR];
-#pragma unroll
-  for (int i = 0; i < kMaxR; ++i) u[i] = 0.0f;
+  // V phase lanes: latent dim d = 32 * pass + 8 * warp + (lane & 7); token
+  // quads (int8) or octets (int4) qg, qg + 4, ... with qg = lane >> 3
+  const int dl = lane & 7, qg = lane >> 3;
+  const int npass = (g.rv + 31) / 32;
+  float u[2] = {0.0f, 0.0f};
   float m_run = -INFINITY, l_run = 0.0f;
 
   for (int j = 0; j < n_my && !aborted; ++j) {
@@ -349,22 +415,99 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
     const bool ok = lk_mbar_wait_bounded(&bars[buf], (uint32_t)((j / kStages) & 1), LK_WAIT_LIMIT_NS);
     if (!ok) *abort_flag = 1;
     const uint8_t* st = smem + buf * L.stage_bytes;
-    const int t = (first_stage + j) * kStageT + tid;
-    const bool valid = ok && t < len;
+    const uint8_t* vs = st + L.off_vs;
+    const int tbase = (first_stage + j) * kStageT;
+    // a. score of this thread's token
+    const bool valid = ok && tbase + tid < len;
     float s = -INFINITY;
-    if (valid) s = token_score<KIND, CSK>(st + L.off_kc, st + L.off_ks, g, tid, qt);
-    const float wmax = lk_warp_max(s);
-    if (wmax > m_run) {  // warp-uniform: rescale the running sums once per new max
-      const float alpha = exp2f(m_run - wmax);
-      l_run *= alpha;
+    if (valid) s = token_score<KIND, CSK>(st + L.off_kc, st + L.off_ks, g, tid, qw, qa);
+    const float wm = lk_warp_max(s);
+    if (lane == 0) smax[warp] = wm;
+    __syncthreads();
+    // b. CTA-uniform running max; weights w_{t,g} = p_t sigma_V[t][g] and their
+    //    per-group stage max W_g
+    float m_new = m_run;
 #pragma unroll
-      for (int i = 0; i < kMaxR; ++i) u[i] *= alpha;
-      m_run = wmax;
+    for (int w = 0; w < kWarps; ++w) m_new = fmaxf(m_new, smax[w]);
+    const float alpha = (m_new == -INFINITY) ? 1.0f : exp2f(m_run - m_new);
+    const float pr = valid ? exp2f(s - m_new) : 0.0f;
+    l_run = fmaf(l_run, alpha, pr);
+    m_run = m_new;
+    for (int gi = 0; gi < g.ngv; ++gi) {
+      const float wgt = valid ? pr * load_scale(vs, tid * g.ngv + gi, KIND) : 0.0f;
+      const float gm = lk_warp_max(wgt);
+      if (lane == 0) wmx[warp * kMaxGroups + gi] = gm;
     }
-    if (valid) {
-      const float pr = exp2f(s - m_run);
-      l_run += pr;
-      accumulate_v<KIND, CSV>(st + L.off_vc, st + L.off_vs, g, tid, pr, u);
+    __syncthreads();
+    //    three-term int8 expansion of w * 127 / W_g (int4: even and odd tokens
+    //    of each octet in separate words)
+    const int pos = KIND == 0 ? tid : (tid & ~7) + ((tid & 1) ? 4 : 0) + ((tid & 7) >> 1);
+    for (int gi = 0; gi < g.ngv; ++gi) {
+      float W = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) W = fmaxf(W, wmx[w * kMaxGroups + gi]);
+      const float wgt = valid ? pr * load_scale(vs, tid * g.ngv + gi, KIND) : 0.0f;
+      const float x = W > 0.0f ? wgt * (127.0f / W) : 0.0f;
+      const float t0 = rintf(x);
+      const float x1 = (x - t0) * 254.0f;
+      const float t1 = rintf(x1);
+      const float t2 = fminf(fmaxf(rintf((x1 - t1) * 254.0f), -127.0f), 127.0f);
+      int8_t* tg = tw + gi * 3 * kStageT;
+      tg[pos] = (int8_t)(int)t0;
+      tg[kStageT + pos] = (int8_t)(int)t1;
+      tg[2 * kStageT + pos] = (int8_t)(int)t2;
+    }
+    __syncthreads();
+    // c. u_d = u_d * alpha + W_g/127 * sum_t (t0 + t1/254 + t2/254^2)_t c_{t,d}
+    const uint8_t* vc = st + L.off_vc;
+#pragma unroll
+    for (int ps = 0; ps < 2; ++ps) {
+      if (ps < npass) {
+        const int d = 32 * ps + 8 * warp + dl;
+        int a0 = 0, a1 = 0, a2 = 0;
+        const int gi = d < g.rv ? (KIND == 0 ? 0 : d / g.gv) : 0;
+        const int8_t* tg = tw + gi * 3 * kStageT;
+        if (d < g.rv) {
+          if (KIND == 0) {
+#pragma unroll
+            for (int i = 0; i < kStageT / 16; ++i) {  // 8 quads of 4 tokens per lane
+              const int quad = qg + 4 * i;
+              const int vw = *reinterpret_cast<const int*>(vc + (quad >> 2) * 16 * g.rbv + d * 16 + (quad & 3) * 4);
+              a0 = __dp4a(vw, reinterpret_cast<const int*>(tg)[quad], a0);
+              a1 = __dp4a(vw, reinterpret_cast<const int*>(tg + kStageT)[quad], a1);
+              a2 = __dp4a(vw, reinterpret_cast<const int*>(tg + 2 * kStageT)[quad], a2);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < kStageT / 32; ++i) {  // 4 octets of 8 tokens per lane
+              const int oct = qg + 4 * i;
+              const uint32_t vw =
+                  *reinterpret_cast<const uint32_t*>(vc + (oct >> 1) * 16 * g.rbv + d * 8 + (oct & 1) * 4);
+              int ev, od;
+              nibbles_to_s8(vw, ev, od);
+              const int* t0w = reinterpret_cast<const int*>(tg);
+              const int* t1w = reinterpret_cast<const int*>(tg + kStageT);
+              const int* t2w = reinterpret_cast<const int*>(tg + 2 * kStageT);
+              a0 = __dp4a(od, t0w[2 * oct + 1], __dp4a(ev, t0w[2 * oct], a0));
+              a1 = __dp4a(od, t1w[2 * oct + 1], __dp4a(ev, t1w[2 * oct], a1));
+              a2 = __dp4a(od, t2w[2 * oct + 1], __dp4a(ev, t2w[2 * oct], a2));
+            }
+          }
+        }
+        // the four lanes sharing dim d hold disjoint token sets
+#pragma unroll
+        for (int o = 8; o < 32; o <<= 1) {
+          a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+          a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+          a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+        }
+        float W = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) W = fmaxf(W, wmx[w * kMaxGroups + gi]);
+        const float contrib =
+            (W * (1.0f / 127.0f)) * fmaf((float)a2, kInv254sq, fmaf((float)a1, kInv254, (float)a0));
+        u[ps] = fmaf(u[ps], alpha, contrib);
+      }
     }
     __syncthreads();  // every thread is done with this buffer
     if (*abort_flag) { aborted = true; stopped_at = j; break; }
@@ -382,46 +525,29 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
     }
     m_run = -INFINITY;
     l_run = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kMaxR; ++i) u[i] = 0.0f;
+    u[0] = u[1] = 0.0f;
   }
 
-  // ---- reduce (m, l, u) over the CTA
-  l_run = lk_warp_sum(l_run);
+  // ---- CTA partial: m is CTA-uniform; each dim's u is held by one lane
+  const float lw = lk_warp_sum(l_run);
+  if (lane == 0) lred[warp] = lw;
+  if (qg == 0) {
 #pragma unroll
-  for (int i = 0; i < kMaxR; ++i) {
-    if (i < g.rv) u[i] = lk_warp_sum(u[i]);
-  }
-  float* wred = red + warp * (2 + kMaxR);
-  if (lane == 0) {
-    wred[0] = m_run;
-    wred[1] = l_run;
-  }
-#pragma unroll
-  for (int i = 0; i < kMaxR; ++i) {
-    if (i < g.rv && lane == (i & 31)) wred[2 + i] = u[i];
-  }
-  __syncthreads();
-
-  const int nw = kThreads / 32;
-  float M = -INFINITY;
-  for (int w = 0; w < nw; ++w) M = fmaxf(M, red[w * (2 + kMaxR)]);
-  // thread j < rv merges u_j; thread kMaxR merges l
-  float* cta = red;
-  float mine = 0.0f;
-  const int idx = (tid < g.rv) ? 2 + tid : (tid == kMaxR ? 1 : -1);
-  if (M != -INFINITY && idx >= 0) {
-    for (int w = 0; w < nw; ++w) {
-      const float mw = red[w * (2 + kMaxR)];
-      if (mw != -INFINITY) mine += red[w * (2 + kMaxR) + idx] * exp2f(mw - M);
+    for (int ps = 0; ps < 2; ++ps) {
+      const int d = 32 * ps + 8 * warp + dl;
+      if (ps < npass && d < g.rv) cta[2 + d] = u[ps];
     }
   }
   __syncthreads();
-  if (idx >= 0) cta[idx] = mine;
-  if (tid == 0) cta[0] = M;
+  if (tid == 0) {
+    float lsum = 0.0f;
+    for (int w = 0; w < kWarps; ++w) lsum += lred[w];
+    cta[0] = m_run;
+    cta[1] = lsum;
+  }
   __syncthreads();
 
-  int* flag = reinterpret_cast<int*>(smem + L.off_misc) + 1;
+  const int idx = (tid < g.rv) ? 2 + tid : (tid == kMaxR ? 1 : -1);
   if (p.n_split > 1) {
     float* part = p.partials + (bh * p.n_split + split) * p.part_stride;
     for (int i = tid; i < 2 + g.rv; i += kThreads) part[i] = cta[i];
@@ -450,10 +576,10 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
     if (idx >= 0) {
       int s2 = 0;
       for (; s2 + 4 <= p.n_split; s2 += 4) {
-        float v0 = __ldcg(P0 + (int64_t)(s2 + 0) * p.part_stride + idx);
-        float v1 = __ldcg(P0 + (int64_t)(s2 + 1) * p.part_stride + idx);
-        float v2 = __ldcg(P0 + (int64_t)(s2 + 2) * p.part_stride + idx);
-        float v3 = __ldcg(P0 + (int64_t)(s2 + 3) * p.part_stride + idx);
+        const float v0 = __ldcg(P0 + (int64_t)(s2 + 0) * p.part_stride + idx);
+        const float v1 = __ldcg(P0 + (int64_t)(s2 + 1) * p.part_stride + idx);
+        const float v2 = __ldcg(P0 + (int64_t)(s2 + 2) * p.part_stride + idx);
+        const float v3 = __ldcg(P0 + (int64_t)(s2 + 3) * p.part_stride + idx);
         acc += v0 * mw[s2] + v1 * mw[s2 + 1] + v2 * mw[s2 + 2] + v3 * mw[s2 + 3];
       }
       for (; s2 < p.n_split; ++s2) acc += __ldcg(P0 + (int64_t)s2 * p.part_stride + idx) * mw[s2];
@@ -482,7 +608,7 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
 }
 
 template <int KIND>
-__global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const SmemLayout L = smem_layout(p);
@@ -525,7 +651,7 @@ namespace lk {
 int decode_pick_split(int units, int max_len, int num_sms) {
   const int stages = (max_len + kStageT - 1) / kStageT;
   if (stages <= 1) return 1;
-  const int target = num_sms * 3;  // about three resident CTAs per SM
+  const int target = num_sms * 4;  // about four resident CTAs per SM
   int s = (target + units - 1) / units;
   s = std::max(1, std::min(s, stages));
   return s;
@@ -559,7 +685,7 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   p.out_bf16 = a.out_bf16;
   p.max_len = a.max_len;
   p.qscale = a.softmax_scale * 1.4426950408889634f;
-  int rk_max = 0, rv_max = 0, rbk_max = 0, rbv_max = 0, ngk_max = 1, ngv_max = 1;
+  int rk_max = 0, rv_max = 0, ngk_max = 1, ngv_max = 1;
   for (int h = 0; h < a.n_heads; ++h) {
     p.rk[h] = (uint8_t)a.ranks_k[h];
     p.rv[h] = (uint8_t)a.ranks_v[h];
@@ -571,13 +697,18 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
       ngv_max = std::max(ngv_max, (a.ranks_v[h] + gv - 1) / gv);
     }
   }
-  rbk_max = a.kind == 0 ? rk_max : rk_max / 2;
-  rbv_max = a.kind == 0 ? rv_max : rv_max / 2;
+  const int rbk_max = a.kind == 0 ? rk_max : rk_max / 2;
+  const int rbv_max = a.kind == 0 ? rv_max : rv_max / 2;
   const int ssz = a.kind == 0 ? 4 : 2;
   p.st_kc = round_up(kStageT * rbk_max, 128);
   p.st_vc = round_up(kStageT * rbv_max, 128);
   p.st_ks = round_up(kStageT * ngk_max * ssz, 128);
   p.st_vs = round_up(kStageT * ngv_max * ssz, 128);
+  p.q_size = a.q_bf16 ? 2 : 4;
+  p.b_size = a.b_bf16 ? 2 : 4;
+  p.st_q = round_up(a.head_dim * p.q_size, 128);
+  p.st_bk = round_up(rk_max * a.head_dim * p.b_size, 128);
+  p.st_bv = round_up(rv_max * a.head_dim * p.b_size, 128);
   const int stages = std::max(1, (a.max_len + kStageT - 1) / kStageT);
   int n_split = a.n_split;
   if (n_split <= 0) n_split = decode_pick_split(a.batch * a.n_heads, a.max_len, a.num_sms);
@@ -590,14 +721,7 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   p.counters = reinterpret_cast<int32_t*>(ws);
   p.partials = reinterpret_cast<float*>(ws + round_up(a.batch * a.n_heads * 4, 256));
 
-  p.q_size = a.q_bf16 ? 2 : 4;
-  p.b_size = a.b_bf16 ? 2 : 4;
-  p.st_q = round_up(a.head_dim * p.q_size, 128);
-  p.st_bk = round_up(rk_max * a.head_dim * p.b_size, 128);
-  p.st_bv = round_up(rv_max * a.head_dim * p.b_size, 128);
-  const int stage_bytes = p.st_kc + p.st_vc + p.st_ks + p.st_vs;
-  const int smem = kStages * stage_bytes + p.st_q + p.st_bk + p.st_bv + kMaxR * 4 + 4 * (2 + kMaxR) * 4 +
-                   2 * kMaxSplit * 4 + (kStages + 1) * 8 + 16;
+  const int smem = smem_bytes_for(p);
   dim3 grid(n_split, a.n_heads, a.batch);
   cudaError_t e;
   if (a.kind == 0) {

@@ -110,20 +110,41 @@ LK_DEVICE void append_head(const FinalizeParams& p, int lrow, int grow, int j) {
   const int tot_ng = is_k ? p.tot_ng_k : p.tot_ng_v;
   if (cv.kind == 0) {
     int8_t* plane = static_cast<int8_t*>(cv.codes) + ((int64_t)b * tot_rb + p.pref_rb[j]) * cap;
-    const int cs = lk_chunk_bytes(r);
-    if (lane < r) plane[lk_code_offset(pos, lane, r, cs)] = (int8_t)qr.c0;
-    if (lane + 32 < r) plane[lk_code_offset(pos, lane + 32, r, cs)] = (int8_t)qr.c1;
+    if (is_k) {  // token-major chunks
+      const int cs = lk_chunk_bytes(r);
+      if (lane < r) plane[lk_code_offset(pos, lane, r, cs)] = (int8_t)qr.c0;
+      if (lane + 32 < r) plane[lk_code_offset(pos, lane + 32, r, cs)] = (int8_t)qr.c1;
+    } else {     // dimension-major: dim d of token t at (t/16)*16*r + d*16 + t%16
+      const int64_t base = (pos >> 4) * 16 * r + (pos & 15);
+      if (lane < r) plane[base + lane * 16] = (int8_t)qr.c0;
+      if (lane + 32 < r) plane[base + (lane + 32) * 16] = (int8_t)qr.c1;
+    }
     if (lane == 0) static_cast<float*>(cv.scales)[((int64_t)b * cv.n_heads + hh) * cap + pos] = qr.s0;
   } else {
     const int rb = r / 2;
     uint8_t* plane = static_cast<uint8_t*>(cv.codes) + ((int64_t)b * tot_rb + p.pref_rb[j]) * cap;
-    const int cs = lk_chunk_bytes(rb);
-    const int n0 = __shfl_down_sync(0xffffffffu, qr.c0, 1);
-    const int n1 = __shfl_down_sync(0xffffffffu, qr.c1, 1);
-    if ((lane & 1) == 0) {
-      if (lane < r) plane[lk_code_offset(pos, lane / 2, rb, cs)] = (uint8_t)((qr.c0 & 0xF) | ((n0 & 0xF) << 4));
-      if (lane + 32 < r)
-        plane[lk_code_offset(pos, (lane + 32) / 2, rb, cs)] = (uint8_t)((qr.c1 & 0xF) | ((n1 & 0xF) << 4));
+    if (is_k) {  // token-major chunks, two dims per byte
+      const int cs = lk_chunk_bytes(rb);
+      const int n0 = __shfl_down_sync(0xffffffffu, qr.c0, 1);
+      const int n1 = __shfl_down_sync(0xffffffffu, qr.c1, 1);
+      if ((lane & 1) == 0) {
+        if (lane < r) plane[lk_code_offset(pos, lane / 2, rb, cs)] = (uint8_t)((qr.c0 & 0xF) | ((n0 & 0xF) << 4));
+        if (lane + 32 < r)
+          plane[lk_code_offset(pos, (lane + 32) / 2, rb, cs)] = (uint8_t)((qr.c1 & 0xF) | ((n1 & 0xF) << 4));
+      }
+    } else {     // dimension-major, two tokens per byte: write this token's nibble only
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        const int d = lane + 32 * q2;
+        if (d < r) {
+          const int64_t off = (pos >> 4) * 16 * rb + d * 8 + ((pos & 15) >> 1);
+          unsigned int* word = reinterpret_cast<unsigned int*>(plane + (off & ~(int64_t)3));
+          const unsigned int shift = (unsigned int)((off & 3) * 8 + (pos & 1) * 4);
+          const unsigned int code = (unsigned int)((q2 == 0 ? qr.c0 : qr.c1) & 0xF);
+          atomicAnd(word, ~(0xFu << shift));  // the neighbour token's nibble may be written concurrently
+          atomicOr(word, code << shift);
+        }
+      }
     }
     const int g = min(cv.group, r), ng = (r + g - 1) / g;
     uint16_t* sp = static_cast<uint16_t*>(cv.scales) + ((int64_t)b * tot_ng + p.pref_ng[j]) * cap + pos * ng;

@@ -52,7 +52,7 @@ class W8A8DecoderLayer:
         self.up = hybrid_weight(weights["up"], E, ffn_inter, device)
         self.down = hybrid_weight(weights["down"], ffn_inter, E, device)
         self.cache_k = LatentCache(batch, ranks_k, capacity, "i8", 32, device)
-        self.cache_v = LatentCache(batch, ranks_v, capacity, "i8", 32, device)
+        self.cache_v = LatentCache(batch, ranks_v, capacity, "i8", 32, device, role="v")
 
     def step(self, x, seq_len, lens, trace=None):
         """x: [B, E] bf16 (device); seq_len: device int32 [B]; lens: host list (advanced in place).

@@ -7,9 +7,12 @@ inspection.  It performs no quantisation or packing of values.
 Layout: for batch row b and head h the code plane holds capacity * rb_h bytes
 (rb_h = r_h for int8, r_h / 2 for int4) at byte offset
 (b * sum_h rb_h + sum_{h'<h} rb_h') * capacity; tokens are stored in blocks of
-16 and, inside a block, chunk-major with chunk size cs = 16, 8 or 4 bytes (the
-largest dividing rb).  Scales: fp32 [capacity] per (b, h) (int8) or fp16
-[capacity][ng_h] per (b, h) (int4), planes in the same (b, h) order.
+16.  Inside a block, K caches are chunk-major over each token's code row
+(chunk size cs = 16, 8 or 4 bytes, the largest dividing rb); V caches are
+dimension-major (int8: dim d of token t at d * 16 + t % 16; int4: dim d of
+tokens 2i, 2i + 1 share byte d * 8 + i, low nibble = even token).  Scales:
+fp32 [capacity] per (b, h) (int8) or fp16 [capacity][ng_h] per (b, h)
+(int4), planes in the same (b, h) order.
 """
 from __future__ import annotations
 
@@ -43,11 +46,55 @@ def tile_index(T, rb):
     return (t // 16) * 16 * rb + (k // cs) * 16 * cs + (t % 16) * cs + (k % cs)
 
 
+def _nibbles(rows):
+    """uint8 [T, nb] -> the 4-bit fields [T, 2 nb], low nibble first."""
+    out = np.empty(rows.shape[:-1] + (2 * rows.shape[-1],), np.uint8)
+    out[..., 0::2] = rows & 0xF
+    out[..., 1::2] = rows >> 4
+    return out
+
+
+def v_plane_from_rows(rows, rb, kind, capacity):
+    """Token rows of code bytes [T, rb] -> a dimension-major V plane [capacity * rb]."""
+    T = rows.shape[0]
+    Tp = (T + 15) // 16 * 16
+    plane = np.zeros(capacity * rb, np.uint8)
+    if kind == "i8":
+        full = np.zeros((Tp, rb), np.uint8)
+        full[:T] = rows
+        blocks = full.reshape(Tp // 16, 16, rb).transpose(0, 2, 1)   # [blk][dim][16 tokens]
+        plane[:Tp * rb] = blocks.reshape(-1)
+        return plane
+    nib = np.zeros((Tp, 2 * rb), np.uint8)
+    nib[:T] = _nibbles(rows)
+    blocks = nib.reshape(Tp // 16, 16, 2 * rb).transpose(0, 2, 1)     # [blk][dim][16 tokens]
+    packed = blocks[..., 0::2] | (blocks[..., 1::2] << 4)                # [blk][dim][8 bytes]
+    plane[:Tp * rb] = packed.reshape(-1)
+    return plane
+
+
+def rows_from_v_plane(plane, T, rb, kind):
+    """Inverse of v_plane_from_rows for the first T tokens."""
+    Tp = (T + 15) // 16 * 16
+    flat = np.asarray(plane[:Tp * rb], np.uint8)
+    if kind == "i8":
+        blocks = flat.reshape(Tp // 16, rb, 16).transpose(0, 2, 1)
+        return blocks.reshape(Tp, rb)[:T].copy()
+    blocks = flat.reshape(Tp // 16, 2 * rb, 8)                           # [blk][dim][8 bytes]
+    nib = np.empty((Tp // 16, 2 * rb, 16), np.uint8)
+    nib[..., 0::2] = blocks & 0xF
+    nib[..., 1::2] = blocks >> 4
+    tok = nib.transpose(0, 2, 1).reshape(Tp, 2 * rb)[:T]               # [token][dim]
+    return (tok[:, 0::2] | (tok[:, 1::2] << 4)).astype(np.uint8)
+
+
 class CacheGeometry:
     """Plane offsets of one cache (one layer, K or V)."""
 
-    def __init__(self, batch, ranks, capacity, kind, group=32):
+    def __init__(self, batch, ranks, capacity, kind, group=32, role="k"):
         assert capacity % 16 == 0
+        assert role in ("k", "v")
+        self.role = role
         self.batch = batch
         self.ranks = [int(r) for r in ranks]
         self.capacity = capacity
@@ -90,8 +137,11 @@ class CacheGeometry:
                 r = np.asarray(rows[b][h], np.uint8)
                 T = r.shape[0]
                 assert T <= self.capacity and r.shape[1] == self.rb[h]
-                off, _ = self.code_plane(b, h)
-                codes[off + tile_index(T, self.rb[h])] = r
+                off, n = self.code_plane(b, h)
+                if self.role == "k":
+                    codes[off + tile_index(T, self.rb[h])] = r
+                else:
+                    codes[off:off + n] = v_plane_from_rows(r, self.rb[h], self.kind, self.capacity)
                 soff, _ = self.scale_plane(b, h)
                 s = np.asarray(scales[b][h], self.scale_dtype).reshape(T, self.ng[h])
                 sc[soff:soff + T * self.ng[h]] = s.reshape(-1)
@@ -106,8 +156,11 @@ class CacheGeometry:
             rr, ss = [], []
             for h in range(len(self.ranks)):
                 T = int(lens[b])
-                off, _ = self.code_plane(b, h)
-                rr.append(codes[off + tile_index(T, self.rb[h])])
+                off, n = self.code_plane(b, h)
+                if self.role == "k":
+                    rr.append(codes[off + tile_index(T, self.rb[h])])
+                else:
+                    rr.append(rows_from_v_plane(codes[off:off + n], T, self.rb[h], self.kind))
                 soff, _ = self.scale_plane(b, h)
                 s = scales[soff:soff + T * self.ng[h]].reshape(T, self.ng[h])
                 ss.append(s[:, 0].copy() if self.kind == "i8" else s.copy())

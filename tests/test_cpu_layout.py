@@ -48,3 +48,29 @@ def test_plane_offsets_follow_the_header_formula():
     assert g.code_plane(0, 2) == ((16 + 32) * 32, 8 * 32)
     assert g.code_plane(1, 1) == ((56 + 16) * 32, 32 * 32)
     assert g.scale_plane(1, 2) == ((1 * 3 + 2) * 32, 32)
+
+
+@pytest.mark.parametrize("kind,ranks", [("i8", [8, 12, 32, 64]), ("i4", [8, 24, 64])])
+def test_v_role_dimension_major_roundtrip(kind, ranks):
+    rng = np.random.default_rng(1)
+    g = CacheGeometry(2, ranks, 48, kind, 16, role="v")
+    lens = [33, 48]
+    rb = [r if kind == "i8" else r // 2 for r in ranks]
+    rows = [[rng.integers(0, 256, (lens[b], n), dtype=np.uint8) for n in rb] for b in range(2)]
+    scales = [[rng.standard_normal((lens[b], ng)).astype(g.scale_dtype) for ng in g.ng] for b in range(2)]
+    c, s = g.pack(rows, scales)
+    r2, _ = g.unpack(c, s, lens)
+    for b in range(2):
+        for h in range(len(ranks)):
+            assert np.array_equal(r2[b][h], rows[b][h])
+    # the header's placement: int8 dim d of token t at (t/16)*16*rb + d*16 + t%16;
+    # int4 byte (t/16)*16*rb + d*8 + (t%16)/2, low nibble = even token
+    off, _ = g.code_plane(1, 1)
+    t, d = 37, 5
+    if kind == "i8":
+        assert c[off + (t // 16) * 16 * rb[1] + d * 16 + t % 16] == rows[1][1][t, d]
+    else:
+        byte = c[off + (t // 16) * 16 * rb[1] + d * 8 + (t % 16) // 2]
+        nib = (byte >> 4) if t % 2 else (byte & 0xF)
+        src = rows[1][1][t, d // 2]
+        assert nib == ((src >> 4) if d % 2 else (src & 0xF))

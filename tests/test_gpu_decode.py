@@ -40,7 +40,7 @@ def make_case(B, ranks_k, ranks_v, H, lens, kind="i8", group=32, capacity=None, 
         lat_v.append([mk(r) for r in ranks_v])
     ok, ov, (rk_rows, rk_sc), (rv_rows, rv_sc) = build_caches(lat_k, lat_v, ranks_k, ranks_v, kind, group)
     ck = lk.LatentCache(B, ranks_k, capacity, kind, group)
-    cv = lk.LatentCache(B, ranks_v, capacity, kind, group)
+    cv = lk.LatentCache(B, ranks_v, capacity, kind, group, role="v")
     ck.load(rk_rows, rk_sc)
     cv.load(rv_rows, rv_sc)
     g = torch.Generator().manual_seed(seed + 1)

@@ -26,7 +26,7 @@ class Harness:
         lk = _lk()
         self.B, self.rk, self.rv, self.kind, self.group = B, ranks_k, ranks_v, kind, group
         self.ck = lk.LatentCache(B, ranks_k, capacity, kind, group)
-        self.cv = lk.LatentCache(B, ranks_v, capacity, kind, group)
+        self.cv = lk.LatentCache(B, ranks_v, capacity, kind, group, role="v")
         self.seq = torch.zeros(B, dtype=torch.int32, device="cuda")
         self.lens = [0] * B
         self.v_oracle = [[] for _ in range(B)]  # per row: list of float32 [n, N_tot]

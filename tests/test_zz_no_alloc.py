@@ -35,7 +35,7 @@ def _case(seed):
     _, _, (rk_rows, rk_sc), (rv_rows, rv_sc) = build_caches(lat_k, lat_v, ranks_k, ranks_v, "i8", 32)
     cap = 2064
     ck = lk.LatentCache(B, ranks_k, cap, "i8", 32)
-    cv = lk.LatentCache(B, ranks_v, cap, "i8", 32)
+    cv = lk.LatentCache(B, ranks_v, cap, "i8", 32, role="v")
     ck.load(rk_rows, rk_sc)
     cv.load(rv_rows, rv_sc)
     g = torch.Generator().manual_seed(seed)
