@@ -1,6 +1,6 @@
 // Latent decode attention, split-K over the sequence (sm_100a).
 //
-// Per (batch row b, head h, split s) one CTA of 128 threads:
+// Per (batch row b, head h, split s) one CTA of 256 threads:
 //   1. absorbs q into latent space, q~ = B_K^h q * softmax_scale * log2(e)
 //      (WSVD page §2C: the fused kernel works from the per-head latents;
 //      without positional rotation (q B_K^T) C^T equals q K^T), and writes
@@ -8,16 +8,18 @@
 //      (error <= 6e-8 of max|q~|, i.e. float32 level);
 //   2. streams its slice of the latent cache (K codes, V codes and their
 //      scales) HBM -> shared memory with bulk copies on the TMA engine,
-//      kStages deep, one mbarrier per stage;
-//   3. per stage of 128 tokens:
+//      2 or 3 stages deep, one mbarrier per stage;
+//   3. per stage of 256 tokens (three block barriers):
 //      a. one token per thread: s_t = sigma_K (c_K . q~) with exact int32
 //         dp4a dot products against the expansion;
 //      b. a CTA-uniform running max, p_t = 2^(s_t - max), running sum;
 //      c. u += p_t sigma_V c_V: the stage's weights w_t = p_t sigma_V[t] are
-//         written as a three-term int8 expansion relative to the stage max
-//         (error <= 6e-8 of it), and each lane takes exact int32 dp4a sums
-//         over 4 (int8) or 8 (int4) tokens of one latent dim at a time from the
-//         dimension-major V layout; one float fold per stage;
+//         written as a three-term int8 expansion relative to
+//         W = max_t p_t * max_t sigma_V[t] >= every w_t (both maxima come out
+//         of the score reduction; error <= 6e-8 W per weight), and each
+//         lane takes exact int32 dp4a sums over 4 (int8) or 8 (int4) tokens
+//         of one latent dim at a time from the dimension-major V layout; one
+//         float fold per stage;
 //   4. reduces (max, sum, u) over the CTA into a partial in latent space; the
 //      last CTA of the (b, h) to arrive (atomic ticket, no waiting) merges
 //      all partials and applies out = (u / sum) B_V^h.
@@ -28,10 +30,10 @@
 
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kStageT = 128;  // tokens per pipeline stage: one per thread in the score phase
-constexpr int kStages = 3;
+constexpr int kStageT = 256;   // tokens per pipeline stage: one per thread in the score phase
+constexpr int kMaxStages = 3;  // pipeline depth chosen at launch (2 or 3)
 constexpr int kMaxR = LK_MAX_RANK;
 constexpr int kMaxWords = kMaxR / 4;  // 32-bit words of q~ terms (int8 per dim)
 constexpr int kMaxGroups = 8;
@@ -56,7 +58,8 @@ struct DecodeParams {
   float qscale;  // softmax_scale * log2(e)
   // bytes of the shared-memory regions (max over heads), multiples of 128
   int st_kc, st_vc, st_ks, st_vs;
-  int st_q, st_bk, st_bv;
+  int st_bv, st_tw;
+  int nstages;
   int q_size, b_size;  // element sizes of q and of the factors
   uint8_t rk[LK_MAX_HEADS];
   uint8_t rv[LK_MAX_HEADS];
@@ -258,23 +261,21 @@ LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom
 struct SmemLayout {
   int stage_bytes;
   int off_kc, off_vc, off_ks, off_vs;  // within a stage
-  int off_q, off_bk, off_bv;           // q^h, B_K^h, B_V^h staged once per CTA
+  int off_bv;                          // B_V^h staged once per CTA
   int off_qt;                          // q~ [kMaxR] floats
   int off_qterm;                       // q~ expansion bytes [3][kMaxR]
-  int off_smax;                        // per-warp stage max [kWarps]
-  int off_wmx;                         // per-warp, per-group weight max [kWarps][kMaxGroups]
-  int off_tw;                          // weight expansion bytes [kMaxGroups][3][kStageT]
+  int off_red;                         // per-warp stage maxima [kWarps][1 + kMaxGroups]
+  int off_tw;                          // weight expansion bytes [ngv][3][kStageT]
   int off_cta;                         // CTA partial [2 + kMaxR]
   int off_lred;                        // [kWarps]
   int off_mw;                          // merge weights [kMaxSplit]
-  int off_bar;                         // kStages stage barriers + 1 factor barrier
+  int off_bar;                         // kMaxStages stage barriers + 1 factor barrier
   int off_misc;
   int total;
 };
 
-constexpr int kSmemFixed = kMaxR * 4 + 3 * kMaxR + kWarps * 4 + kWarps * kMaxGroups * 4 +
-                           kMaxGroups * 3 * kStageT + (2 + kMaxR) * 4 + kWarps * 4 + kMaxSplit * 4 +
-                           (kStages + 1) * 8 + 16;
+constexpr int kSmemFixed = kMaxR * 4 + 3 * kMaxR + kWarps * (1 + kMaxGroups) * 4 + (2 + kMaxR) * 4 +
+                           kWarps * 4 + kMaxSplit * 4 + (kMaxStages + 1) * 8 + 16;
 
 LK_DEVICE SmemLayout smem_layout(const DecodeParams& p) {
   SmemLayout L;
@@ -283,26 +284,23 @@ LK_DEVICE SmemLayout smem_layout(const DecodeParams& p) {
   L.off_ks = p.st_kc + p.st_vc;
   L.off_vs = p.st_kc + p.st_vc + p.st_ks;
   L.stage_bytes = p.st_kc + p.st_vc + p.st_ks + p.st_vs;
-  L.off_q = kStages * L.stage_bytes;
-  L.off_bk = L.off_q + p.st_q;
-  L.off_bv = L.off_bk + p.st_bk;
-  L.off_qt = L.off_bv + p.st_bv;
+  L.off_bv = p.nstages * L.stage_bytes;
+  L.off_tw = L.off_bv + p.st_bv;
+  L.off_qt = L.off_tw + p.st_tw;
   L.off_qterm = L.off_qt + kMaxR * 4;
-  L.off_smax = L.off_qterm + 3 * kMaxR;
-  L.off_wmx = L.off_smax + kWarps * 4;
-  L.off_tw = L.off_wmx + kWarps * kMaxGroups * 4;
-  L.off_cta = L.off_tw + kMaxGroups * 3 * kStageT;
+  L.off_red = L.off_qterm + 3 * kMaxR;
+  L.off_cta = L.off_red + kWarps * (1 + kMaxGroups) * 4;
   L.off_lred = L.off_cta + (2 + kMaxR) * 4;
   L.off_mw = L.off_lred + kWarps * 4;
   L.off_bar = L.off_mw + kMaxSplit * 4;
-  L.off_misc = L.off_bar + (kStages + 1) * 8;
+  L.off_misc = L.off_bar + (kMaxStages + 1) * 8;
   L.total = L.off_misc + 16;
   return L;
 }
 
 inline int smem_bytes_for(const DecodeParams& p) {
   const int stage = p.st_kc + p.st_vc + p.st_ks + p.st_vs;
-  return kStages * stage + p.st_q + p.st_bk + p.st_bv + kSmemFixed;
+  return p.nstages * stage + p.st_bv + p.st_tw + kSmemFixed;
 }
 
 template <int KIND, int CSK, int CSV>
@@ -310,12 +308,12 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
                            int b, int h, int split, int len, int first_stage, int n_my) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int H = p.head_dim;
+  const int NS = p.nstages;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.off_bar);
-  uint64_t* fbar = bars + kStages;
+  uint64_t* fbar = bars + kMaxStages;
   float* qt_s = reinterpret_cast<float*>(smem + L.off_qt);
   int8_t* qterm = reinterpret_cast<int8_t*>(smem + L.off_qterm);
-  float* smax = reinterpret_cast<float*>(smem + L.off_smax);
-  float* wmx = reinterpret_cast<float*>(smem + L.off_wmx);
+  float* red = reinterpret_cast<float*>(smem + L.off_red);
   int8_t* tw = reinterpret_cast<int8_t*>(smem + L.off_tw);
   float* cta = reinterpret_cast<float*>(smem + L.off_cta);
   float* lred = reinterpret_cast<float*>(smem + L.off_lred);
@@ -324,9 +322,10 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
   float* qa_s = reinterpret_cast<float*>(smem + L.off_misc) + 2;
   const int ssz = KIND == 0 ? 4 : 2;
   const int64_t bh = (int64_t)b * p.n_heads + h;
+  constexpr int RW = 1 + kMaxGroups;  // per-warp reduction row: score max, then sigma_V max per group
 
-  auto issue = [&](int j) {  // stage j of this split -> buffer j % kStages
-    const int buf = j % kStages;
+  auto issue = [&](int j) {  // stage j of this split -> buffer j % NS
+    const int buf = j % NS;
     const int64_t t0 = (int64_t)(first_stage + j) * kStageT;
     const int64_t end = min((int64_t)((len + 15) & ~15), (int64_t)p.capacity);
     const int ntok = (int)min((int64_t)kStageT, end - t0);
@@ -341,27 +340,39 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
   };
 
   if (tid == 0) {
-    // factors first: q^h and B_K^h (needed before the first token), B_V^h (epilogue)
-    const uint32_t qb = H * p.q_size, bkb = g.rk * H * p.b_size, bvb = g.rv * H * p.b_size;
-    lk_mbar_arrive_expect_tx(fbar, qb + bkb + bvb);
-    lk_bulk_g2s(smem + L.off_q, static_cast<const uint8_t*>(p.q) + bh * H * p.q_size, qb, fbar);
-    lk_bulk_g2s(smem + L.off_bk, static_cast<const uint8_t*>(p.BK) + g.bk_off * p.b_size, bkb, fbar);
+    // B_V^h for the epilogue, then the first stages of latent codes
+    const uint32_t bvb = g.rv * H * p.b_size;
+    lk_mbar_arrive_expect_tx(fbar, bvb);
     lk_bulk_g2s(smem + L.off_bv, static_cast<const uint8_t*>(p.BV) + g.bv_off * p.b_size, bvb, fbar);
-    for (int j = 0; j < min(kStages, n_my); ++j) issue(j);
+    for (int j = 0; j < min(NS, n_my); ++j) issue(j);
   }
 
-  bool aborted = false;
-  int stopped_at = 0;
-  // ---- absorb q: q~[i] = qscale * sum_d B_K[i][d] q[d]
-  if (!lk_mbar_wait_bounded(fbar, 0, LK_WAIT_LIMIT_NS)) *abort_flag = 1;
-  if (!*abort_flag) {
-    const uint8_t* qs = smem + L.off_q;
-    const uint8_t* bks = smem + L.off_bk;
-    for (int i = warp; i < g.rk; i += kWarps) {
+  // ---- absorb q: q~[i] = qscale * sum_d B_K[i][d] q[d], B_K^h and q read from
+  //      global memory with every load of a thread in flight at once
+  {
+    int rp2 = 4;
+    while (rp2 < g.rk) rp2 <<= 1;
+    const int tpr = min(32, kThreads / rp2);  // threads per row (a power of two)
+    const int rows_per_pass = kThreads / tpr;
+    const int part = tid % tpr;
+    const int64_t qoff = bh * H;
+    const int npass = (g.rk + rows_per_pass - 1) / rows_per_pass;  // uniform across the CTA
+    for (int ps = 0; ps < npass; ++ps) {
+      const int i = tid / tpr + ps * rows_per_pass;
       float acc = 0.0f;
-      for (int d = lane; d < H; d += 32) acc = fmaf(ld_f(qs, d, p.q_bf16), ld_f(bks, i * H + d, p.b_bf16), acc);
-      acc = lk_warp_sum(acc);
-      if (lane == 0) qt_s[i] = acc * p.qscale;
+      if (i < g.rk) {
+#pragma unroll 8
+        for (int d = part; d < H; d += tpr) {
+          const float qd = p.q_bf16 ? lk_bf16_to_f32(reinterpret_cast<const uint16_t*>(p.q)[qoff + d])
+                                    : reinterpret_cast<const float*>(p.q)[qoff + d];
+          const int64_t bi = g.bk_off + (int64_t)i * H + d;
+          const float bk = p.b_bf16 ? lk_bf16_to_f32(reinterpret_cast<const uint16_t*>(p.BK)[bi])
+                                    : reinterpret_cast<const float*>(p.BK)[bi];
+          acc = fmaf(qd, bk, acc);
+        }
+      }
+      for (int o = 1; o < tpr; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (part == 0 && i < g.rk) qt_s[i] = acc * p.qscale;
     }
   }
   __syncthreads();
@@ -372,30 +383,24 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
     const float amax = lk_warp_max(fmaxf(fabsf(v0), fabsf(v1)));
     const float a = amax / 127.0f;
     const float inva = amax > 0.0f ? 127.0f / amax : 0.0f;
-    int tv[2][3];
 #pragma unroll
     for (int q2 = 0; q2 < 2; ++q2) {
       const float x = (q2 == 0 ? v0 : v1) * inva;
       const float t0 = rintf(x);
       const float x1 = (x - t0) * 254.0f;
       const float t1 = rintf(x1);
-      const float x2 = (x1 - t1) * 254.0f;
-      const float t2 = fminf(fmaxf(rintf(x2), -127.0f), 127.0f);
-      tv[q2][0] = (int)t0; tv[q2][1] = (int)t1; tv[q2][2] = (int)t2;
+      const float t2 = fminf(fmaxf(rintf((x1 - t1) * 254.0f), -127.0f), 127.0f);
       const int d = lane + 32 * q2;
-      if (d < kMaxR) {
-        // int4 keys meet even dims and odd dims in separate words
-        const int pos = KIND == 0 ? d : ((d >> 3) << 3) + ((d & 1) ? 4 : 0) + ((d & 7) >> 1);
-        const bool live = d < g.rk;
-        qterm[0 * kMaxR + pos] = (int8_t)(live ? tv[q2][0] : 0);
-        qterm[1 * kMaxR + pos] = (int8_t)(live ? tv[q2][1] : 0);
-        qterm[2 * kMaxR + pos] = (int8_t)(live ? tv[q2][2] : 0);
-      }
+      // int4 keys meet even dims and odd dims in separate words
+      const int pos = KIND == 0 ? d : ((d >> 3) << 3) + ((d & 1) ? 4 : 0) + ((d & 7) >> 1);
+      const bool live = d < g.rk;
+      qterm[0 * kMaxR + pos] = (int8_t)(live ? (int)t0 : 0);
+      qterm[1 * kMaxR + pos] = (int8_t)(live ? (int)t1 : 0);
+      qterm[2 * kMaxR + pos] = (int8_t)(live ? (int)t2 : 0);
     }
     if (lane == 0) *qa_s = a;
   }
   __syncthreads();
-  if (*abort_flag) aborted = true;
   const float qa = *qa_s;
   uint32_t qw[3][kMaxWords];
 #pragma unroll
@@ -403,51 +408,56 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
 #pragma unroll
     for (int w = 0; w < kMaxWords; ++w) qw[i][w] = reinterpret_cast<const uint32_t*>(qterm + i * kMaxR)[w];
 
-  // V phase lanes: latent dim d = 32 * pass + 8 * warp + (lane & 7); token
-  // quads (int8) or octets (int4) qg, qg + 4, ... with qg = lane >> 3
+  // V phase lanes: latent dim d = 8 * warp + (lane & 7); token quads (int8)
+  // or octets (int4) qg, qg + 4, ... with qg = lane >> 3
   const int dl = lane & 7, qg = lane >> 3;
-  const int npass = (g.rv + 31) / 32;
-  float u[2] = {0.0f, 0.0f};
+  const int dv = 8 * warp + dl;
+  const int gv_of_d = dv < g.rv ? (KIND == 0 ? 0 : dv / g.gv) : 0;
+  float u = 0.0f;
   float m_run = -INFINITY, l_run = 0.0f;
+  bool aborted = false;
+  int stopped_at = 0;
 
-  for (int j = 0; j < n_my && !aborted; ++j) {
-    const int buf = j % kStages;
-    const bool ok = lk_mbar_wait_bounded(&bars[buf], (uint32_t)((j / kStages) & 1), LK_WAIT_LIMIT_NS);
+  for (int j = 0; j < n_my; ++j) {
+    const int buf = j % NS;
+    const bool ok = lk_mbar_wait_bounded(&bars[buf], (uint32_t)((j / NS) & 1), LK_WAIT_LIMIT_NS);
     if (!ok) *abort_flag = 1;
     const uint8_t* st = smem + buf * L.stage_bytes;
     const uint8_t* vs = st + L.off_vs;
     const int tbase = (first_stage + j) * kStageT;
-    // a. score of this thread's token
+    // a. score of this thread's token; stage maxima of the score and of sigma_V
     const bool valid = ok && tbase + tid < len;
     float s = -INFINITY;
     if (valid) s = token_score<KIND, CSK>(st + L.off_kc, st + L.off_ks, g, tid, qw, qa);
-    const float wm = lk_warp_max(s);
-    if (lane == 0) smax[warp] = wm;
-    __syncthreads();
-    // b. CTA-uniform running max; weights w_{t,g} = p_t sigma_V[t][g] and their
-    //    per-group stage max W_g
-    float m_new = m_run;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) m_new = fmaxf(m_new, smax[w]);
-    const float alpha = (m_new == -INFINITY) ? 1.0f : exp2f(m_run - m_new);
-    const float pr = valid ? exp2f(s - m_new) : 0.0f;
-    l_run = fmaf(l_run, alpha, pr);
-    m_run = m_new;
-    for (int gi = 0; gi < g.ngv; ++gi) {
-      const float wgt = valid ? pr * load_scale(vs, tid * g.ngv + gi, KIND) : 0.0f;
-      const float gm = lk_warp_max(wgt);
-      if (lane == 0) wmx[warp * kMaxGroups + gi] = gm;
+    {
+      const float wm = lk_warp_max(s);
+      if (lane == 0) red[warp * RW] = wm;
+      for (int gi = 0; gi < g.ngv; ++gi) {
+        const float sm = lk_warp_max(valid ? load_scale(vs, tid * g.ngv + gi, KIND) : 0.0f);
+        if (lane == 0) red[warp * RW + 1 + gi] = sm;
+      }
     }
     __syncthreads();
-    //    three-term int8 expansion of w * 127 / W_g (int4: even and odd tokens
-    //    of each octet in separate words)
+    // b. CTA-uniform running max, p_t, and the weights' three-term expansion
+    //    x = p_t sigma_V[t][g] * 127 / W_g (int4: even and odd tokens of each
+    //    octet in separate words)
+    float smx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) smx = fmaxf(smx, red[w * RW]);
+    const float m_new = fmaxf(m_run, smx);
+    const float alpha = (m_new == -INFINITY) ? 1.0f : exp2f(m_run - m_new);
+    const float pr = valid ? exp2f(s - m_new) : 0.0f;
+    const float pmax = (smx == -INFINITY) ? 0.0f : exp2f(smx - m_new);  // largest p of the stage
+    l_run = fmaf(l_run, alpha, pr);
+    m_run = m_new;
     const int pos = KIND == 0 ? tid : (tid & ~7) + ((tid & 1) ? 4 : 0) + ((tid & 7) >> 1);
     for (int gi = 0; gi < g.ngv; ++gi) {
       float W = 0.0f;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) W = fmaxf(W, wmx[w * kMaxGroups + gi]);
-      const float wgt = valid ? pr * load_scale(vs, tid * g.ngv + gi, KIND) : 0.0f;
-      const float x = W > 0.0f ? wgt * (127.0f / W) : 0.0f;
+      for (int w = 0; w < kWarps; ++w) W = fmaxf(W, red[w * RW + 1 + gi]);
+      W *= pmax;
+      const float x = (valid && W > 0.0f) ? fminf(pr * load_scale(vs, tid * g.ngv + gi, KIND) * (127.0f / W), 127.0f)
+                                          : 0.0f;
       const float t0 = rintf(x);
       const float x1 = (x - t0) * 254.0f;
       const float t1 = rintf(x1);
@@ -459,85 +469,79 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
     }
     __syncthreads();
     // c. u_d = u_d * alpha + W_g/127 * sum_t (t0 + t1/254 + t2/254^2)_t c_{t,d}
-    const uint8_t* vc = st + L.off_vc;
+    {
+      const uint8_t* vc = st + L.off_vc;
+      const int8_t* tg = tw + gv_of_d * 3 * kStageT;
+      const int* t0w = reinterpret_cast<const int*>(tg);
+      const int* t1w = reinterpret_cast<const int*>(tg + kStageT);
+      const int* t2w = reinterpret_cast<const int*>(tg + 2 * kStageT);
+      int a0 = 0, a1 = 0, a2 = 0;
+      if (dv < g.rv) {
+        if (KIND == 0) {
 #pragma unroll
-    for (int ps = 0; ps < 2; ++ps) {
-      if (ps < npass) {
-        const int d = 32 * ps + 8 * warp + dl;
-        int a0 = 0, a1 = 0, a2 = 0;
-        const int gi = d < g.rv ? (KIND == 0 ? 0 : d / g.gv) : 0;
-        const int8_t* tg = tw + gi * 3 * kStageT;
-        if (d < g.rv) {
-          if (KIND == 0) {
+          for (int i = 0; i < kStageT / 16; ++i) {  // 16 quads of 4 tokens per lane
+            const int quad = qg + 4 * i;
+            const int vw = *reinterpret_cast<const int*>(vc + (quad >> 2) * 16 * g.rbv + dv * 16 + (quad & 3) * 4);
+            a0 = __dp4a(vw, t0w[quad], a0);
+            a1 = __dp4a(vw, t1w[quad], a1);
+            a2 = __dp4a(vw, t2w[quad], a2);
+          }
+        } else {
 #pragma unroll
-            for (int i = 0; i < kStageT / 16; ++i) {  // 8 quads of 4 tokens per lane
-              const int quad = qg + 4 * i;
-              const int vw = *reinterpret_cast<const int*>(vc + (quad >> 2) * 16 * g.rbv + d * 16 + (quad & 3) * 4);
-              a0 = __dp4a(vw, reinterpret_cast<const int*>(tg)[quad], a0);
-              a1 = __dp4a(vw, reinterpret_cast<const int*>(tg + kStageT)[quad], a1);
-              a2 = __dp4a(vw, reinterpret_cast<const int*>(tg + 2 * kStageT)[quad], a2);
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < kStageT / 32; ++i) {  // 4 octets of 8 tokens per lane
-              const int oct = qg + 4 * i;
-              const uint32_t vw =
-                  *reinterpret_cast<const uint32_t*>(vc + (oct >> 1) * 16 * g.rbv + d * 8 + (oct & 1) * 4);
-              int ev, od;
-              nibbles_to_s8(vw, ev, od);
-              const int* t0w = reinterpret_cast<const int*>(tg);
-              const int* t1w = reinterpret_cast<const int*>(tg + kStageT);
-              const int* t2w = reinterpret_cast<const int*>(tg + 2 * kStageT);
-              a0 = __dp4a(od, t0w[2 * oct + 1], __dp4a(ev, t0w[2 * oct], a0));
-              a1 = __dp4a(od, t1w[2 * oct + 1], __dp4a(ev, t1w[2 * oct], a1));
-              a2 = __dp4a(od, t2w[2 * oct + 1], __dp4a(ev, t2w[2 * oct], a2));
-            }
+          for (int i = 0; i < kStageT / 32; ++i) {  // 8 octets of 8 tokens per lane
+            const int oct = qg + 4 * i;
+            const uint32_t vw =
+                *reinterpret_cast<const uint32_t*>(vc + (oct >> 1) * 16 * g.rbv + dv * 8 + (oct & 1) * 4);
+            int ev, od;
+            nibbles_to_s8(vw, ev, od);
+            a0 = __dp4a(od, t0w[2 * oct + 1], __dp4a(ev, t0w[2 * oct], a0));
+            a1 = __dp4a(od, t1w[2 * oct + 1], __dp4a(ev, t1w[2 * oct], a1));
+            a2 = __dp4a(od, t2w[2 * oct + 1], __dp4a(ev, t2w[2 * oct], a2));
           }
         }
-        // the four lanes sharing dim d hold disjoint token sets
-#pragma unroll
-        for (int o = 8; o < 32; o <<= 1) {
-          a0 += __shfl_xor_sync(0xffffffffu, a0, o);
-          a1 += __shfl_xor_sync(0xffffffffu, a1, o);
-          a2 += __shfl_xor_sync(0xffffffffu, a2, o);
-        }
-        float W = 0.0f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) W = fmaxf(W, wmx[w * kMaxGroups + gi]);
-        const float contrib =
-            (W * (1.0f / 127.0f)) * fmaf((float)a2, kInv254sq, fmaf((float)a1, kInv254, (float)a0));
-        u[ps] = fmaf(u[ps], alpha, contrib);
       }
+      // the four lanes sharing dim d hold disjoint token sets
+#pragma unroll
+      for (int o = 8; o < 32; o <<= 1) {
+        a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+        a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+        a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+      }
+      float W = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) W = fmaxf(W, red[w * RW + 1 + gv_of_d]);
+      W *= pmax;
+      const float contrib =
+          (W * (1.0f / 127.0f)) * fmaf((float)a2, kInv254sq, fmaf((float)a1, kInv254, (float)a0));
+      u = fmaf(u, alpha, contrib);
     }
-    __syncthreads();  // every thread is done with this buffer
+    __syncthreads();  // every thread is done with this buffer and with red / tw
     if (*abort_flag) { aborted = true; stopped_at = j; break; }
-    if (tid == 0 && j + kStages < n_my) issue(j + kStages);
+    if (tid == 0 && j + NS < n_my) issue(j + NS);
   }
   if (aborted) {
     if (tid == 0) {
       lk_dev_fail(LK_DEV_TIMEOUT_PIPE);
       // drain copies still in flight into this CTA's shared memory
-      if (!lk_mbar_wait_bounded(fbar, 0, LK_WAIT_LIMIT_NS)) lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
-      for (int j = stopped_at; j < min(n_my, stopped_at + kStages); ++j) {
-        if (!lk_mbar_wait_bounded(&bars[j % kStages], (uint32_t)((j / kStages) & 1), LK_WAIT_LIMIT_NS))
+      for (int j = stopped_at; j < min(n_my, stopped_at + NS); ++j) {
+        if (!lk_mbar_wait_bounded(&bars[j % NS], (uint32_t)((j / NS) & 1), LK_WAIT_LIMIT_NS))
           lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
       }
     }
     m_run = -INFINITY;
     l_run = 0.0f;
-    u[0] = u[1] = 0.0f;
+    u = 0.0f;
+  }
+  // B_V^h must have landed before the epilogue (and before the CTA may exit)
+  if (!lk_mbar_wait_bounded(fbar, 0, LK_WAIT_LIMIT_NS)) {
+    if (tid == 0) lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
+    aborted = true;
   }
 
   // ---- CTA partial: m is CTA-uniform; each dim's u is held by one lane
   const float lw = lk_warp_sum(l_run);
   if (lane == 0) lred[warp] = lw;
-  if (qg == 0) {
-#pragma unroll
-    for (int ps = 0; ps < 2; ++ps) {
-      const int d = 32 * ps + 8 * warp + dl;
-      if (ps < npass && d < g.rv) cta[2 + d] = u[ps];
-    }
-  }
+  if (qg == 0 && dv < g.rv) cta[2 + dv] = u;
   __syncthreads();
   if (tid == 0) {
     float lsum = 0.0f;
@@ -608,7 +612,7 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
 }
 
 template <int KIND>
-__global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const SmemLayout L = smem_layout(p);
@@ -622,7 +626,7 @@ __global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_cons
 
   if (threadIdx.x == 0) {
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.off_bar);
-    for (int i = 0; i < kStages + 1; ++i) lk_mbar_init(&bars[i], 1);
+    for (int i = 0; i < kMaxStages + 1; ++i) lk_mbar_init(&bars[i], 1);
     lk_fence_mbar_init();
     *reinterpret_cast<int*>(smem + L.off_misc) = 0;
   }
@@ -651,7 +655,7 @@ namespace lk {
 int decode_pick_split(int units, int max_len, int num_sms) {
   const int stages = (max_len + kStageT - 1) / kStageT;
   if (stages <= 1) return 1;
-  const int target = num_sms * 4;  // about four resident CTAs per SM
+  const int target = num_sms * 2;  // about two resident CTAs per SM
   int s = (target + units - 1) / units;
   s = std::max(1, std::min(s, stages));
   return s;
@@ -706,9 +710,11 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   p.st_vs = round_up(kStageT * ngv_max * ssz, 128);
   p.q_size = a.q_bf16 ? 2 : 4;
   p.b_size = a.b_bf16 ? 2 : 4;
-  p.st_q = round_up(a.head_dim * p.q_size, 128);
-  p.st_bk = round_up(rk_max * a.head_dim * p.b_size, 128);
   p.st_bv = round_up(rv_max * a.head_dim * p.b_size, 128);
+  p.st_tw = round_up(ngv_max * 3 * kStageT, 128);
+  // three stages when two CTAs still fit on an SM, else two
+  p.nstages = kMaxStages;
+  if (smem_bytes_for(p) > 113 * 1024) p.nstages = 2;
   const int stages = std::max(1, (a.max_len + kStageT - 1) / kStageT);
   int n_split = a.n_split;
   if (n_split <= 0) n_split = decode_pick_split(a.batch * a.n_heads, a.max_len, a.num_sms);
