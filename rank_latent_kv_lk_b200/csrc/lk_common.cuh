@@ -143,6 +143,10 @@ LK_DEVICE void lk_mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
+LK_DEVICE void lk_mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(lk_smem_addr(bar)) : "memory");
+}
+
 LK_DEVICE bool lk_mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(

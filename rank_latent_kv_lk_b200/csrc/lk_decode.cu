@@ -30,10 +30,12 @@
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+constexpr int kCW = 8;                          // consumer warps
+constexpr int kConsumerThreads = kCW * 32;
+constexpr int kWTerms = 4;                      // int8 terms of the weight expansion
+constexpr int kThreads = kConsumerThreads + 32;  // + one producer warp
 constexpr int kStageT = 256;   // tokens per pipeline stage: one per thread in the score phase
-constexpr int kMaxStages = 3;  // pipeline depth chosen at launch (2 or 3)
+constexpr int kMaxStages = 8;  // pipeline depth chosen at launch (2 .. 8)
 constexpr int kMaxR = LK_MAX_RANK;
 constexpr int kMaxWords = kMaxR / 4;  // 32-bit words of q~ terms (int8 per dim)
 constexpr int kMaxGroups = 8;
@@ -262,20 +264,19 @@ struct SmemLayout {
   int stage_bytes;
   int off_kc, off_vc, off_ks, off_vs;  // within a stage
   int off_bv;                          // B_V^h staged once per CTA
+  int off_tw;                          // per consumer warp: weight expansion bytes [ngv][3][32]
   int off_qt;                          // q~ [kMaxR] floats
   int off_qterm;                       // q~ expansion bytes [3][kMaxR]
-  int off_red;                         // per-warp stage maxima [kWarps][1 + kMaxGroups]
-  int off_tw;                          // weight expansion bytes [ngv][3][kStageT]
+  int off_wst;                         // per consumer warp: (m, l, u[kMaxR])
   int off_cta;                         // CTA partial [2 + kMaxR]
-  int off_lred;                        // [kWarps]
   int off_mw;                          // merge weights [kMaxSplit]
-  int off_bar;                         // kMaxStages stage barriers + 1 factor barrier
+  int off_bar;                         // full[kMaxStages], empty[kMaxStages], factor barrier
   int off_misc;
   int total;
 };
 
-constexpr int kSmemFixed = kMaxR * 4 + 3 * kMaxR + kWarps * (1 + kMaxGroups) * 4 + (2 + kMaxR) * 4 +
-                           kWarps * 4 + kMaxSplit * 4 + (kMaxStages + 1) * 8 + 16;
+constexpr int kSmemFixed = kMaxR * 4 + 3 * kMaxR + kCW * (2 + kMaxR) * 4 + (2 + kMaxR) * 4 + kMaxSplit * 4 +
+                           (2 * kMaxStages + 1) * 8 + 16;
 
 LK_DEVICE SmemLayout smem_layout(const DecodeParams& p) {
   SmemLayout L;
@@ -288,12 +289,11 @@ LK_DEVICE SmemLayout smem_layout(const DecodeParams& p) {
   L.off_tw = L.off_bv + p.st_bv;
   L.off_qt = L.off_tw + p.st_tw;
   L.off_qterm = L.off_qt + kMaxR * 4;
-  L.off_red = L.off_qterm + 3 * kMaxR;
-  L.off_cta = L.off_red + kWarps * (1 + kMaxGroups) * 4;
-  L.off_lred = L.off_cta + (2 + kMaxR) * 4;
-  L.off_mw = L.off_lred + kWarps * 4;
+  L.off_wst = L.off_qterm + 3 * kMaxR;
+  L.off_cta = L.off_wst + kCW * (2 + kMaxR) * 4;
+  L.off_mw = L.off_cta + (2 + kMaxR) * 4;
   L.off_bar = L.off_mw + kMaxSplit * 4;
-  L.off_misc = L.off_bar + (kMaxStages + 1) * 8;
+  L.off_misc = L.off_bar + (2 * kMaxStages + 1) * 8;
   L.total = L.off_misc + 16;
   return L;
 }
@@ -309,54 +309,29 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int H = p.head_dim;
   const int NS = p.nstages;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.off_bar);
-  uint64_t* fbar = bars + kMaxStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.off_bar);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* fbar = full + 2 * kMaxStages;
   float* qt_s = reinterpret_cast<float*>(smem + L.off_qt);
   int8_t* qterm = reinterpret_cast<int8_t*>(smem + L.off_qterm);
-  float* red = reinterpret_cast<float*>(smem + L.off_red);
-  int8_t* tw = reinterpret_cast<int8_t*>(smem + L.off_tw);
+  float* wst = reinterpret_cast<float*>(smem + L.off_wst);
   float* cta = reinterpret_cast<float*>(smem + L.off_cta);
-  float* lred = reinterpret_cast<float*>(smem + L.off_lred);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.off_misc);
   int* flag = reinterpret_cast<int*>(smem + L.off_misc) + 1;
   float* qa_s = reinterpret_cast<float*>(smem + L.off_misc) + 2;
   const int ssz = KIND == 0 ? 4 : 2;
   const int64_t bh = (int64_t)b * p.n_heads + h;
-  constexpr int RW = 1 + kMaxGroups;  // per-warp reduction row: score max, then sigma_V max per group
 
-  auto issue = [&](int j) {  // stage j of this split -> buffer j % NS
-    const int buf = j % NS;
-    const int64_t t0 = (int64_t)(first_stage + j) * kStageT;
-    const int64_t end = min((int64_t)((len + 15) & ~15), (int64_t)p.capacity);
-    const int ntok = (int)min((int64_t)kStageT, end - t0);
-    uint8_t* st = smem + buf * L.stage_bytes;
-    const uint32_t bkc = ntok * g.rbk, bvc = ntok * g.rbv;
-    const uint32_t bks = ntok * g.ngk * ssz, bvs = ntok * g.ngv * ssz;
-    lk_mbar_arrive_expect_tx(&bars[buf], bkc + bvc + bks + bvs);
-    lk_bulk_g2s(st + L.off_kc, p.codes_k + g.kc_off + t0 * g.rbk, bkc, &bars[buf]);
-    lk_bulk_g2s(st + L.off_vc, p.codes_v + g.vc_off + t0 * g.rbv, bvc, &bars[buf]);
-    lk_bulk_g2s(st + L.off_ks, p.scales_k + (g.ks_off + t0 * g.ngk) * ssz, bks, &bars[buf]);
-    lk_bulk_g2s(st + L.off_vs, p.scales_v + (g.vs_off + t0 * g.ngv) * ssz, bvs, &bars[buf]);
-  };
-
-  if (tid == 0) {
-    // B_V^h for the epilogue, then the first stages of latent codes
-    const uint32_t bvb = g.rv * H * p.b_size;
-    lk_mbar_arrive_expect_tx(fbar, bvb);
-    lk_bulk_g2s(smem + L.off_bv, static_cast<const uint8_t*>(p.BV) + g.bv_off * p.b_size, bvb, fbar);
-    for (int j = 0; j < min(NS, n_my); ++j) issue(j);
-  }
-
-  // ---- absorb q: q~[i] = qscale * sum_d B_K[i][d] q[d], B_K^h and q read from
+  // ---- absorb q (consumer threads): q~[i] = qscale * sum_d B_K[i][d] q[d], from
   //      global memory with every load of a thread in flight at once
-  {
+  if (warp < kCW) {
     int rp2 = 4;
     while (rp2 < g.rk) rp2 <<= 1;
-    const int tpr = min(32, kThreads / rp2);  // threads per row (a power of two)
-    const int rows_per_pass = kThreads / tpr;
+    const int tpr = min(32, kConsumerThreads / rp2);  // threads per row (a power of two)
+    const int rows_per_pass = kConsumerThreads / tpr;
     const int part = tid % tpr;
     const int64_t qoff = bh * H;
-    const int npass = (g.rk + rows_per_pass - 1) / rows_per_pass;  // uniform across the CTA
+    const int npass = (g.rk + rows_per_pass - 1) / rows_per_pass;
     for (int ps = 0; ps < npass; ++ps) {
       const int i = tid / tpr + ps * rows_per_pass;
       float acc = 0.0f;
@@ -401,153 +376,196 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
     if (lane == 0) *qa_s = a;
   }
   __syncthreads();
-  const float qa = *qa_s;
-  uint32_t qw[3][kMaxWords];
-#pragma unroll
-  for (int i = 0; i < 3; ++i)
-#pragma unroll
-    for (int w = 0; w < kMaxWords; ++w) qw[i][w] = reinterpret_cast<const uint32_t*>(qterm + i * kMaxR)[w];
 
-  // V phase lanes: latent dim d = 8 * warp + (lane & 7); token quads (int8)
-  // or octets (int4) qg, qg + 4, ... with qg = lane >> 3
-  const int dl = lane & 7, qg = lane >> 3;
-  const int dv = 8 * warp + dl;
-  const int gv_of_d = dv < g.rv ? (KIND == 0 ? 0 : dv / g.gv) : 0;
-  float u = 0.0f;
-  float m_run = -INFINITY, l_run = 0.0f;
-  bool aborted = false;
-  int stopped_at = 0;
-
-  for (int j = 0; j < n_my; ++j) {
-    const int buf = j % NS;
-    const bool ok = lk_mbar_wait_bounded(&bars[buf], (uint32_t)((j / NS) & 1), LK_WAIT_LIMIT_NS);
-    if (!ok) *abort_flag = 1;
-    const uint8_t* st = smem + buf * L.stage_bytes;
-    const uint8_t* vs = st + L.off_vs;
-    const int tbase = (first_stage + j) * kStageT;
-    // a. score of this thread's token; stage maxima of the score and of sigma_V
-    const bool valid = ok && tbase + tid < len;
-    float s = -INFINITY;
-    if (valid) s = token_score<KIND, CSK>(st + L.off_kc, st + L.off_ks, g, tid, qw, qa);
-    {
-      const float wm = lk_warp_max(s);
-      if (lane == 0) red[warp * RW] = wm;
-      for (int gi = 0; gi < g.ngv; ++gi) {
-        const float sm = lk_warp_max(valid ? load_scale(vs, tid * g.ngv + gi, KIND) : 0.0f);
-        if (lane == 0) red[warp * RW + 1 + gi] = sm;
+  if (warp == kCW) {
+    // ================= producer warp: bulk copies, gated by the empty barriers
+    if (lane == 0) {
+      auto issue = [&](int j) {  // stage j of this split -> buffer j % NS
+        const int buf = j % NS;
+        const int64_t t0 = (int64_t)(first_stage + j) * kStageT;
+        const int64_t end = min((int64_t)((len + 15) & ~15), (int64_t)p.capacity);
+        const int ntok = (int)min((int64_t)kStageT, end - t0);
+        uint8_t* st = smem + buf * L.stage_bytes;
+        const uint32_t bkc = ntok * g.rbk, bvc = ntok * g.rbv;
+        const uint32_t bks = ntok * g.ngk * ssz, bvs = ntok * g.ngv * ssz;
+        lk_mbar_arrive_expect_tx(&full[buf], bkc + bvc + bks + bvs);
+        lk_bulk_g2s(st + L.off_kc, p.codes_k + g.kc_off + t0 * g.rbk, bkc, &full[buf]);
+        lk_bulk_g2s(st + L.off_vc, p.codes_v + g.vc_off + t0 * g.rbv, bvc, &full[buf]);
+        lk_bulk_g2s(st + L.off_ks, p.scales_k + (g.ks_off + t0 * g.ngk) * ssz, bks, &full[buf]);
+        lk_bulk_g2s(st + L.off_vs, p.scales_v + (g.vs_off + t0 * g.ngv) * ssz, bvs, &full[buf]);
+      };
+      const uint32_t bvb = g.rv * H * p.b_size;
+      lk_mbar_arrive_expect_tx(fbar, bvb);
+      lk_bulk_g2s(smem + L.off_bv, static_cast<const uint8_t*>(p.BV) + g.bv_off * p.b_size, bvb, fbar);
+      int issued = 0;
+      for (int j = 0; j < n_my; ++j) {
+        if (*abort_flag) break;
+        if (j >= NS) {  // the consumers released this buffer's previous stage
+          if (!lk_mbar_wait_bounded(&empty[j % NS], (uint32_t)(((j / NS) - 1) & 1), LK_WAIT_LIMIT_NS)) {
+            *abort_flag = 1;
+            break;
+          }
+        }
+        issue(j);
+        issued = j + 1;
+      }
+      // before the CTA may finish, every copy this CTA started has landed
+      for (int j = max(0, issued - NS); j < issued; ++j) {
+        if (!lk_mbar_wait_bounded(&full[j % NS], (uint32_t)((j / NS) & 1), LK_WAIT_LIMIT_NS)) {
+          lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
+          *abort_flag = 1;
+        }
+      }
+      if (!lk_mbar_wait_bounded(fbar, 0, LK_WAIT_LIMIT_NS)) {
+        lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
+        *abort_flag = 1;
       }
     }
-    __syncthreads();
-    // b. CTA-uniform running max, p_t, and the weights' three-term expansion
-    //    x = p_t sigma_V[t][g] * 127 / W_g (int4: even and odd tokens of each
-    //    octet in separate words)
-    float smx = -INFINITY;
+  } else {
+    // ================= consumer warp: tokens 32 * warp .. 32 * warp + 31 of every stage
+    const float qa = *qa_s;
+    uint32_t qw[3][kMaxWords];
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) smx = fmaxf(smx, red[w * RW]);
-    const float m_new = fmaxf(m_run, smx);
-    const float alpha = (m_new == -INFINITY) ? 1.0f : exp2f(m_run - m_new);
-    const float pr = valid ? exp2f(s - m_new) : 0.0f;
-    const float pmax = (smx == -INFINITY) ? 0.0f : exp2f(smx - m_new);  // largest p of the stage
-    l_run = fmaf(l_run, alpha, pr);
-    m_run = m_new;
-    const int pos = KIND == 0 ? tid : (tid & ~7) + ((tid & 1) ? 4 : 0) + ((tid & 7) >> 1);
-    for (int gi = 0; gi < g.ngv; ++gi) {
-      float W = 0.0f;
+    for (int i = 0; i < 3; ++i)
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) W = fmaxf(W, red[w * RW + 1 + gi]);
-      W *= pmax;
-      const float x = (valid && W > 0.0f) ? fminf(pr * load_scale(vs, tid * g.ngv + gi, KIND) * (127.0f / W), 127.0f)
-                                          : 0.0f;
-      const float t0 = rintf(x);
-      const float x1 = (x - t0) * 254.0f;
-      const float t1 = rintf(x1);
-      const float t2 = fminf(fmaxf(rintf((x1 - t1) * 254.0f), -127.0f), 127.0f);
-      int8_t* tg = tw + gi * 3 * kStageT;
-      tg[pos] = (int8_t)(int)t0;
-      tg[kStageT + pos] = (int8_t)(int)t1;
-      tg[2 * kStageT + pos] = (int8_t)(int)t2;
-    }
-    __syncthreads();
-    // c. u_d = u_d * alpha + W_g/127 * sum_t (t0 + t1/254 + t2/254^2)_t c_{t,d}
-    {
+      for (int w = 0; w < kMaxWords; ++w) qw[i][w] = reinterpret_cast<const uint32_t*>(qterm + i * kMaxR)[w];
+    // weight-expansion bytes of this warp: [group][term][32 tokens]
+    int8_t* tw = reinterpret_cast<int8_t*>(smem + L.off_tw) + warp * (p.st_tw / kCW);
+    const int tl = 32 * warp + lane;  // this lane's token within a stage
+    // int4 values: even and odd tokens of an octet live in separate words
+    const int tpos = KIND == 0 ? lane : (lane & ~7) + ((lane & 1) ? 4 : 0) + ((lane & 7) >> 1);
+    // V: this lane owns latent dims lane and lane + 32; exact int32 sums of
+    // (expanded weight term) x code, folded into float only when the running
+    // max or the reference scale changes
+    int A[2][kWTerms];
+    float u[2] = {0.0f, 0.0f};
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+      for (int i = 0; i < kWTerms; ++i) A[k][i] = 0;
+    float m_run = -INFINITY, l_run = 0.0f;
+    float wref = 0.0f;  // every weight of the open accumulation is <= wref
+    auto fold = [&](float alpha) {
+      const float sc = wref * (1.0f / 127.0f);
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        float x = (float)A[k][kWTerms - 1];
+#pragma unroll
+        for (int i = kWTerms - 2; i >= 0; --i) x = fmaf(x, kInv254, (float)A[k][i]);
+        u[k] = (u[k] + sc * x) * alpha;
+#pragma unroll
+        for (int i = 0; i < kWTerms; ++i) A[k][i] = 0;
+      }
+    };
+
+    for (int j = 0; j < n_my; ++j) {
+      const int buf = j % NS;
+      if (!lk_mbar_wait_bounded(&full[buf], (uint32_t)((j / NS) & 1), LK_WAIT_LIMIT_NS)) *abort_flag = 1;
+      if (*abort_flag) break;
+      const uint8_t* st = smem + buf * L.stage_bytes;
+      const uint8_t* vs = st + L.off_vs;
+      const bool valid = (first_stage + j) * kStageT + tl < len;
+      // a. score; a new running max (warp vote) folds the open sums
+      float s = -INFINITY;
+      if (valid) s = token_score<KIND, CSK>(st + L.off_kc, st + L.off_ks, g, tl, qw, qa);
+      if (__any_sync(0xffffffffu, s > m_run)) {
+        const float m_new = fmaxf(m_run, lk_warp_max(s));
+        const float alpha = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - m_new);
+        fold(alpha);
+        l_run *= alpha;
+        m_run = m_new;
+      }
+      const float pr = valid ? exp2f(s - m_run) : 0.0f;
+      l_run += pr;
+      // b. reference scale: a larger V scale (warp vote) folds, then raises wref
+      float smax_t = 0.0f;
+      for (int gi = 0; gi < g.ngv; ++gi) smax_t = fmaxf(smax_t, valid ? load_scale(vs, tl * g.ngv + gi, KIND) : 0.0f);
+      if (__any_sync(0xffffffffu, smax_t > wref)) {
+        fold(1.0f);
+        wref = fmaxf(wref, lk_warp_max(smax_t));
+      }
+      //    weights w = p sigma_V as a four-term int8 expansion of w * 127 / wref
+      const float inv = wref > 0.0f ? 127.0f / wref : 0.0f;
+      for (int gi = 0; gi < g.ngv; ++gi) {
+        const float sg = valid ? load_scale(vs, tl * g.ngv + gi, KIND) : 0.0f;
+        float x = fminf(pr * sg * inv, 127.0f);
+        int8_t* tg = tw + gi * (kWTerms * 32);
+#pragma unroll
+        for (int i = 0; i < kWTerms; ++i) {
+          const float t = fminf(fmaxf(rintf(x), -127.0f), 127.0f);
+          tg[32 * i + tpos] = (int8_t)(int)t;
+          x = (x - t) * 254.0f;
+        }
+      }
+      __syncwarp();
+      // c. A[d][i] += sum over the warp's 32 tokens of term_i(t) * c_{t,d}
       const uint8_t* vc = st + L.off_vc;
-      const int8_t* tg = tw + gv_of_d * 3 * kStageT;
-      const int* t0w = reinterpret_cast<const int*>(tg);
-      const int* t1w = reinterpret_cast<const int*>(tg + kStageT);
-      const int* t2w = reinterpret_cast<const int*>(tg + 2 * kStageT);
-      int a0 = 0, a1 = 0, a2 = 0;
-      if (dv < g.rv) {
-        if (KIND == 0) {
 #pragma unroll
-          for (int i = 0; i < kStageT / 16; ++i) {  // 16 quads of 4 tokens per lane
-            const int quad = qg + 4 * i;
-            const int vw = *reinterpret_cast<const int*>(vc + (quad >> 2) * 16 * g.rbv + dv * 16 + (quad & 3) * 4);
-            a0 = __dp4a(vw, t0w[quad], a0);
-            a1 = __dp4a(vw, t1w[quad], a1);
-            a2 = __dp4a(vw, t2w[quad], a2);
-          }
-        } else {
+      for (int k = 0; k < 2; ++k) {
+        const int d = lane + 32 * k;
+        if (d < g.rv) {
+          const int gi = KIND == 0 ? 0 : d / g.gv;
+          const uint32_t* T = reinterpret_cast<const uint32_t*>(tw + gi * (kWTerms * 32));
 #pragma unroll
-          for (int i = 0; i < kStageT / 32; ++i) {  // 8 octets of 8 tokens per lane
-            const int oct = qg + 4 * i;
-            const uint32_t vw =
-                *reinterpret_cast<const uint32_t*>(vc + (oct >> 1) * 16 * g.rbv + dv * 8 + (oct & 1) * 4);
-            int ev, od;
-            nibbles_to_s8(vw, ev, od);
-            a0 = __dp4a(od, t0w[2 * oct + 1], __dp4a(ev, t0w[2 * oct], a0));
-            a1 = __dp4a(od, t1w[2 * oct + 1], __dp4a(ev, t1w[2 * oct], a1));
-            a2 = __dp4a(od, t2w[2 * oct + 1], __dp4a(ev, t2w[2 * oct], a2));
+          for (int blk = 0; blk < 2; ++blk) {  // the warp's two 16-token blocks
+            const int b16 = 2 * warp + blk;
+            if (KIND == 0) {
+              const uint4 v = *reinterpret_cast<const uint4*>(vc + b16 * 16 * g.rbv + d * 16);
+              const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int qd = 0; qd < 4; ++qd)
+#pragma unroll
+                for (int i = 0; i < kWTerms; ++i) A[k][i] = __dp4a((int)vw[qd], (int)T[8 * i + 4 * blk + qd], A[k][i]);
+            } else {
+              const uint2 v = *reinterpret_cast<const uint2*>(vc + b16 * 16 * g.rbv + d * 8);
+              const uint32_t vw[2] = {v.x, v.y};
+#pragma unroll
+              for (int oc = 0; oc < 2; ++oc) {
+                int ev, od;
+                nibbles_to_s8(vw[oc], ev, od);
+                const int o = 2 * blk + oc;  // octet of the warp's tokens
+#pragma unroll
+                for (int i = 0; i < kWTerms; ++i)
+                  A[k][i] = __dp4a(od, (int)T[8 * i + 2 * o + 1], __dp4a(ev, (int)T[8 * i + 2 * o], A[k][i]));
+              }
+            }
           }
         }
       }
-      // the four lanes sharing dim d hold disjoint token sets
-#pragma unroll
-      for (int o = 8; o < 32; o <<= 1) {
-        a0 += __shfl_xor_sync(0xffffffffu, a0, o);
-        a1 += __shfl_xor_sync(0xffffffffu, a1, o);
-        a2 += __shfl_xor_sync(0xffffffffu, a2, o);
-      }
-      float W = 0.0f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) W = fmaxf(W, red[w * RW + 1 + gv_of_d]);
-      W *= pmax;
-      const float contrib =
-          (W * (1.0f / 127.0f)) * fmaf((float)a2, kInv254sq, fmaf((float)a1, kInv254, (float)a0));
-      u = fmaf(u, alpha, contrib);
+      __syncwarp();  // this warp is done with the stage buffer and its weight bytes
+      if (lane == 0) lk_mbar_arrive(&empty[buf]);
     }
-    __syncthreads();  // every thread is done with this buffer and with red / tw
-    if (*abort_flag) { aborted = true; stopped_at = j; break; }
-    if (tid == 0 && j + NS < n_my) issue(j + NS);
-  }
-  if (aborted) {
-    if (tid == 0) {
-      lk_dev_fail(LK_DEV_TIMEOUT_PIPE);
-      // drain copies still in flight into this CTA's shared memory
-      for (int j = stopped_at; j < min(n_my, stopped_at + NS); ++j) {
-        if (!lk_mbar_wait_bounded(&bars[j % NS], (uint32_t)((j / NS) & 1), LK_WAIT_LIMIT_NS))
-          lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
-      }
+    fold(1.0f);
+    // per-warp state (m, l, u)
+    const float lw = lk_warp_sum(l_run);
+    float* ws = wst + warp * (2 + kMaxR);
+    if (lane == 0) {
+      ws[0] = m_run;
+      ws[1] = lw;
     }
-    m_run = -INFINITY;
-    l_run = 0.0f;
-    u = 0.0f;
+    if (lane < g.rv) ws[2 + lane] = u[0];
+    if (lane + 32 < g.rv) ws[2 + lane + 32] = u[1];
   }
-  // B_V^h must have landed before the epilogue (and before the CTA may exit)
-  if (!lk_mbar_wait_bounded(fbar, 0, LK_WAIT_LIMIT_NS)) {
-    if (tid == 0) lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
-    aborted = true;
-  }
-
-  // ---- CTA partial: m is CTA-uniform; each dim's u is held by one lane
-  const float lw = lk_warp_sum(l_run);
-  if (lane == 0) lred[warp] = lw;
-  if (qg == 0 && dv < g.rv) cta[2 + dv] = u;
   __syncthreads();
-  if (tid == 0) {
-    float lsum = 0.0f;
-    for (int w = 0; w < kWarps; ++w) lsum += lred[w];
-    cta[0] = m_run;
-    cta[1] = lsum;
+  const bool aborted = *abort_flag != 0;
+  if (aborted && tid == 0) lk_dev_fail(LK_DEV_TIMEOUT_PIPE);
+
+  // ---- merge the consumer warps' states into the CTA partial
+  {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kCW; ++w) M = fmaxf(M, wst[w * (2 + kMaxR)]);
+    const int idx = (tid < g.rv) ? 2 + tid : (tid == kMaxR ? 1 : -1);
+    float acc = 0.0f;
+    if (idx >= 0 && M != -INFINITY && !aborted) {
+#pragma unroll
+      for (int w = 0; w < kCW; ++w) {
+        const float mw = wst[w * (2 + kMaxR)];
+        if (mw != -INFINITY) acc += wst[w * (2 + kMaxR) + idx] * exp2f(mw - M);
+      }
+    }
+    if (idx >= 0) cta[idx] = acc;
+    if (tid == 0) cta[0] = aborted ? -INFINITY : M;
   }
   __syncthreads();
 
@@ -626,7 +644,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const __grid_c
 
   if (threadIdx.x == 0) {
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.off_bar);
-    for (int i = 0; i < kMaxStages + 1; ++i) lk_mbar_init(&bars[i], 1);
+    for (int i = 0; i < kMaxStages; ++i) lk_mbar_init(&bars[i], 1);                       // full
+    for (int i = kMaxStages; i < 2 * kMaxStages; ++i) lk_mbar_init(&bars[i], kCW);       // empty
+    lk_mbar_init(&bars[2 * kMaxStages], 1);                                              // factor
     lk_fence_mbar_init();
     *reinterpret_cast<int*>(smem + L.off_misc) = 0;
   }
@@ -655,7 +675,10 @@ namespace lk {
 int decode_pick_split(int units, int max_len, int num_sms) {
   const int stages = (max_len + kStageT - 1) / kStageT;
   if (stages <= 1) return 1;
-  const int target = num_sms * 2;  // about two resident CTAs per SM
+  // splitting only pays while the (batch, head) units leave SMs idle: with
+  // two resident CTAs per SM, aim for about one full wave
+  if (units >= num_sms) return 1;
+  const int target = num_sms * 2;
   int s = (target + units - 1) / units;
   s = std::max(1, std::min(s, stages));
   return s;
@@ -711,10 +734,15 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   p.q_size = a.q_bf16 ? 2 : 4;
   p.b_size = a.b_bf16 ? 2 : 4;
   p.st_bv = round_up(rv_max * a.head_dim * p.b_size, 128);
-  p.st_tw = round_up(ngv_max * 3 * kStageT, 128);
-  // three stages when two CTAs still fit on an SM, else two
-  p.nstages = kMaxStages;
-  if (smem_bytes_for(p) > 113 * 1024) p.nstages = 2;
+  p.st_tw = kCW * round_up(ngv_max * kWTerms * 32, 16);
+  // as many stages as fit while two CTAs share an SM (about 64 KB of copies
+  // in flight per SM keeps HBM busy), between 2 and kMaxStages
+  {
+    p.nstages = 0;
+    const int stage = p.st_kc + p.st_vc + p.st_ks + p.st_vs;
+    const int room = 110 * 1024 - (smem_bytes_for(p));  // smem_bytes_for counts 0 stages here
+    p.nstages = std::max(2, std::min(kMaxStages, room / std::max(stage, 1)));
+  }
   const int stages = std::max(1, (a.max_len + kStageT - 1) / kStageT);
   int n_split = a.n_split;
   if (n_split <= 0) n_split = decode_pick_split(a.batch * a.n_heads, a.max_len, a.num_sms);
