@@ -9,14 +9,16 @@
 //      the int8 dequantisation scales when the inputs are int8, quantise the
 //      r_h values (absmax, RNE) and write codes + scale at position
 //      seq_len[b] + t in the token-tiled cache layout.
-// Decode (<= 32 rows) runs both phases in ONE launch: a split-E GEMV with
-// every weight chunk loaded up front, then per-head arrival tickets (no
-// waiting) so the CTA that completes a head appends it, and the CTA that
-// completes the last head advances seq_len.  Prefill runs the tiled GEMM per
+// Decode (<= 32 rows) runs both phases in ONE launch: a cluster of CTAs per
+// head splits E, and the cluster's rank 0 sums the partials over distributed
+// shared memory and appends; the last head to finish advances seq_len.  Prefill runs the tiled GEMM per
 // row chunk, then an epilogue launch.
 #include "lk_common.cuh"
 #include "lk_internal.h"
 #include "lk_quant.cuh"
+
+#include <cooperative_groups.h>
+namespace cg = cooperative_groups;
 
 namespace lk {
 cudaError_t launch_gemm_f(const void* A, int lda, const void* B, int ldb, float* C, int ldc, int M,
@@ -28,7 +30,6 @@ namespace {
 constexpr int kGemvThreads = 256;
 constexpr int kColsPerWarp = 4;
 constexpr int kColsPerCta = kColsPerWarp * (kGemvThreads / 32);  // 32
-constexpr int kMT = 8;  // rows per pass
 constexpr int kGemvMaxRows = 32;
 
 template <int XT> struct XTraits;
@@ -72,14 +73,12 @@ struct FinalizeParams {
   int16_t pref_ng[2 * LK_MAX_HEADS];   // prefix of scale groups within its cache
 };
 
+LK_DEVICE void append_values(const FinalizeParams& p, int grow, int j, float v0, float v1);
+
 // Sums the partials of head j for local row lrow, quantises them and writes
 // the codes and scale of token seq_len[b] + t into the cache (one warp).
 LK_DEVICE void append_head(const FinalizeParams& p, int lrow, int grow, int j) {
   const int lane = threadIdx.x & 31;
-  const int b = grow / p.n_new, t = grow % p.n_new;
-  const bool is_k = j < p.k.n_heads;
-  const lk::CacheView& cv = is_k ? p.k : p.v;
-  const int hh = is_k ? j : j - p.k.n_heads;
   const int r = p.rank[j];
   const int col0 = p.col[j];
   float vals[2];
@@ -89,18 +88,48 @@ LK_DEVICE void append_head(const FinalizeParams& p, int lrow, int grow, int j) {
     float val = 0.0f;
     if (d < r) {
       const int n = col0 + d;
+      // all slices' partials in flight at once, then summed in slice order
+      const uint32_t* src = p.ws + (int64_t)lrow * p.n_tot + n;
+      const int64_t stride = (int64_t)p.ws_rows * p.n_tot;
       if (p.int_inputs) {
         int acc = 0;
-        for (int s = 0; s < p.n_ksplit; ++s) acc += (int)__ldcg(p.ws + ((int64_t)s * p.ws_rows + lrow) * p.n_tot + n);
+        int s = 0;
+        for (; s + 8 <= p.n_ksplit; s += 8) {
+          uint32_t v[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[k] = __ldcg(src + (s + k) * stride);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc += (int)v[k];
+        }
+        for (; s < p.n_ksplit; ++s) acc += (int)__ldcg(src + s * stride);
         val = __fmul_rn(__fmul_rn((float)acc, p.x_scale[grow]), lk_f16_to_f32(p.a_scale[n]));
       } else {
-        for (int s = 0; s < p.n_ksplit; ++s)
-          val += __uint_as_float(__ldcg(p.ws + ((int64_t)s * p.ws_rows + lrow) * p.n_tot + n));
+        int s = 0;
+        for (; s + 8 <= p.n_ksplit; s += 8) {
+          uint32_t v[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[k] = __ldcg(src + (s + k) * stride);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) val += __uint_as_float(v[k]);
+        }
+        for (; s < p.n_ksplit; ++s) val += __uint_as_float(__ldcg(src + s * stride));
       }
     }
     vals[q] = val;
   }
-  const LkQRow qr = lk_quantize_row_warp(vals[0], vals[1], r, cv.kind, cv.group);
+  append_values(p, grow, j, vals[0], vals[1]);
+}
+
+// Quantises one head's latent row (lane l holds dims l and l + 32) and writes
+// the codes and scale of token seq_len[b] + t into the cache (one warp).
+LK_DEVICE void append_values(const FinalizeParams& p, int grow, int j, float v0, float v1) {
+  const int lane = threadIdx.x & 31;
+  const int b = grow / p.n_new, t = grow % p.n_new;
+  const bool is_k = j < p.k.n_heads;
+  const lk::CacheView& cv = is_k ? p.k : p.v;
+  const int hh = is_k ? j : j - p.k.n_heads;
+  const int r = p.rank[j];
+  const LkQRow qr = lk_quantize_row_warp(v0, v1, r, cv.kind, cv.group);
   const int64_t pos = (int64_t)p.seq_len[b] + t;
   const int cap = cv.capacity;
   // the host checked the capacity against its copy of seq_len; never write past
@@ -174,152 +203,159 @@ __global__ void __launch_bounds__(128) proj_finalize_kernel(const __grid_constan
   if (threadIdx.x == 0) *p.counter = 0;
 }
 
-// ---------------------------------------------------------------- decode: one fused launch
-constexpr int kDecU = 2;  // 16-byte chunks per lane per column in one E-slice
+// ---------------------------------------------------------------- decode: one cluster per head
+// A thread-block cluster of kClusterE CTAs owns one head: CTA q reduces the
+// q-th slice of E for every latent column of the head and every row; the
+// cluster's rank 0 sums the kClusterE partials over distributed shared memory,
+// quantises and appends.  No partials leave the SMs and nobody waits on a
+// global counter; the last head to finish advances seq_len (atomic ticket).
+constexpr int kClusterE = 4;
+constexpr int kProjNC = 2;  // latent columns a warp works on at once
+constexpr int kProjU = 4;   // 16-byte chunks per lane per column in flight
 
-struct DecodeProjParams {
+struct ClusterProjParams {
   FinalizeParams f;
   const void* x;
   const void* A;
   int M, E, slice;
-  int32_t* head_cnt;            // [n_heads_tot] arrival counters
-  int32_t* done_cnt;            // heads appended so far
-  int16_t expect[2 * LK_MAX_HEADS];  // arrivals that complete head j
+  int32_t* done_cnt;
 };
 
-// Split-E GEMV over 32 latent columns per CTA (4 per warp) with every weight
-// chunk of the slice loaded up front, then per-head tickets: the CTA whose
-// arrival completes a head quantises and appends it; the CTA completing the
-// last head advances seq_len.
-template <int XT>
-__global__ void __launch_bounds__(kGemvThreads) proj_decode_kernel(const __grid_constant__ DecodeProjParams p) {
+template <int XT, int MT>
+__global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid_constant__ ClusterProjParams p) {
   using T = typename XTraits<XT>::T;
   constexpr int VE = XTraits<XT>::VE;
   constexpr bool INT = XT == lk::X_I8;
-  extern __shared__ __align__(16) uint8_t xs_raw[];  // [M][slice] of T
-  __shared__ int ready[2 * LK_MAX_HEADS];
-  __shared__ int n_ready;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
   const FinalizeParams& f = p.f;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int j = blockIdx.y;
+  const int r = f.rank[j], col0 = f.col[j];
+  const int M = p.M;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int e0 = rank * p.slice;
+  const int elen = max(0, min(p.slice, p.E - e0));
+  const int chunks = elen / VE;
+  uint32_t* part = reinterpret_cast<uint32_t*>(smem_raw);                    // [kMaxR][M]
+  T* xs = reinterpret_cast<T*>(smem_raw + (size_t)LK_MAX_RANK * M * 4);      // [M][slice]
   const T* x = static_cast<const T*>(p.x);
   const T* A = static_cast<const T*>(p.A);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int ks = blockIdx.y;
-  const int e0 = ks * p.slice;
-  const int elen = min(p.slice, p.E - e0);
-  const int chunks = elen / VE;
-  const int n0 = blockIdx.x * kColsPerCta;
-  const int nbase = n0 + warp * kColsPerWarp;
-  const int N = f.n_tot, M = p.M;
-  T* xs = reinterpret_cast<T*>(xs_raw);
 
-  // all weight loads of this lane in flight before any use
-  uint4 wv[kColsPerWarp][kDecU];
-#pragma unroll
-  for (int j = 0; j < kColsPerWarp; ++j)
-#pragma unroll
-    for (int u = 0; u < kDecU; ++u) {
-      const int cc = lane + 32 * u, n = nbase + j;
-      wv[j][u] = (cc < chunks && n < N)
-                     ? __ldg(reinterpret_cast<const uint4*>(A + (int64_t)n * p.E + e0 + cc * VE))
-                     : make_uint4(0, 0, 0, 0);
-    }
   for (int c = threadIdx.x; c < M * chunks; c += kGemvThreads) {
     const int mm = c / chunks, cc = c % chunks;
     *reinterpret_cast<uint4*>(xs + mm * p.slice + cc * VE) =
         *reinterpret_cast<const uint4*>(x + (int64_t)mm * p.E + e0 + cc * VE);
   }
-  if (threadIdx.x == 0) n_ready = 0;
   __syncthreads();
 
-  for (int m0 = 0; m0 < M; m0 += kMT) {
-    const int mt = min(kMT, M - m0);
-    float facc[kColsPerWarp][kMT];
-    int iacc[kColsPerWarp][kMT];
+  for (int cb = warp * kProjNC; cb < r; cb += (kGemvThreads / 32) * kProjNC) {
+    for (int m0 = 0; m0 < M; m0 += MT) {
+      const int mt = min(MT, M - m0);
+      float facc[kProjNC][MT];
+      int iacc[kProjNC][MT];
 #pragma unroll
-    for (int j = 0; j < kColsPerWarp; ++j)
+      for (int jj = 0; jj < kProjNC; ++jj)
 #pragma unroll
-      for (int i = 0; i < kMT; ++i) { facc[j][i] = 0.0f; iacc[j][i] = 0; }
+        for (int i = 0; i < MT; ++i) { facc[jj][i] = 0.0f; iacc[jj][i] = 0; }
+      for (int u0 = 0; u0 < chunks; u0 += 32 * kProjU) {
+        uint4 wv[kProjNC][kProjU];
 #pragma unroll
-    for (int u = 0; u < kDecU; ++u) {
-      const int cc = lane + 32 * u;
-      if (cc < chunks) {
+        for (int jj = 0; jj < kProjNC; ++jj)
 #pragma unroll
-        for (int i = 0; i < kMT; ++i) {
-          if (i < mt) {
-            const uint4 xv4 = *reinterpret_cast<const uint4*>(xs + (m0 + i) * p.slice + cc * VE);
-            if (INT) {
+          for (int u = 0; u < kProjU; ++u) {
+            const int cc = u0 + lane + 32 * u, cl = cb + jj;
+            wv[jj][u] = (cc < chunks && cl < r)
+                            ? __ldg(reinterpret_cast<const uint4*>(A + (int64_t)(col0 + cl) * p.E + e0 + cc * VE))
+                            : make_uint4(0, 0, 0, 0);
+          }
 #pragma unroll
-              for (int j = 0; j < kColsPerWarp; ++j) {
-                int a = iacc[j][i];
-                a = __dp4a((int)xv4.x, (int)wv[j][u].x, a);
-                a = __dp4a((int)xv4.y, (int)wv[j][u].y, a);
-                a = __dp4a((int)xv4.z, (int)wv[j][u].z, a);
-                a = __dp4a((int)xv4.w, (int)wv[j][u].w, a);
-                iacc[j][i] = a;
-              }
-            } else {
-              float xf[VE];
-              expand16<XT>(xv4, xf);
+        for (int u = 0; u < kProjU; ++u) {
+          const int cc = u0 + lane + 32 * u;
+          if (cc < chunks) {
 #pragma unroll
-              for (int j = 0; j < kColsPerWarp; ++j) {
-                float wf[VE];
-                expand16<XT>(wv[j][u], wf);
-                float a = facc[j][i];
+            for (int i = 0; i < MT; ++i) {
+              if (i < mt) {
+                const uint4 xv4 = *reinterpret_cast<const uint4*>(xs + (m0 + i) * p.slice + cc * VE);
+                if (INT) {
 #pragma unroll
-                for (int k = 0; k < VE; ++k) a = fmaf(xf[k], wf[k], a);
-                facc[j][i] = a;
+                  for (int jj = 0; jj < kProjNC; ++jj) {
+                    int a = iacc[jj][i];
+                    a = __dp4a((int)xv4.x, (int)wv[jj][u].x, a);
+                    a = __dp4a((int)xv4.y, (int)wv[jj][u].y, a);
+                    a = __dp4a((int)xv4.z, (int)wv[jj][u].z, a);
+                    a = __dp4a((int)xv4.w, (int)wv[jj][u].w, a);
+                    iacc[jj][i] = a;
+                  }
+                } else {
+                  float xf[VE];
+                  expand16<XT>(xv4, xf);
+#pragma unroll
+                  for (int jj = 0; jj < kProjNC; ++jj) {
+                    float wf[VE];
+                    expand16<XT>(wv[jj][u], wf);
+                    float a = facc[jj][i];
+#pragma unroll
+                    for (int k = 0; k < VE; ++k) a = fmaf(xf[k], wf[k], a);
+                    facc[jj][i] = a;
+                  }
+                }
               }
             }
           }
         }
       }
-    }
 #pragma unroll
-    for (int j = 0; j < kColsPerWarp; ++j) {
+      for (int jj = 0; jj < kProjNC; ++jj) {
 #pragma unroll
-      for (int i = 0; i < kMT; ++i) {
-        uint32_t val;
-        if (INT) {
-          int a = iacc[j][i];
+        for (int i = 0; i < MT; ++i) {
+          uint32_t val;
+          if (INT) {
+            int a = iacc[jj][i];
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-          val = (uint32_t)a;
-        } else {
-          val = __float_as_uint(lk_warp_sum(facc[j][i]));
+            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+            val = (uint32_t)a;
+          } else {
+            val = __float_as_uint(lk_warp_sum(facc[jj][i]));
+          }
+          if (lane == 0 && i < mt && cb + jj < r) part[(cb + jj) * M + m0 + i] = val;
         }
-        const int n = nbase + j;
-        if (lane == j * kMT + i && i < mt && n < N) f.ws[((int64_t)ks * M + m0 + i) * N + n] = val;
       }
     }
   }
+  cluster.sync();  // every CTA's partials are visible to the cluster
 
-  // arrivals: this CTA's 32 columns of slice ks are written
-  __threadfence();
-  __syncthreads();
-  const int n_heads_tot = f.k.n_heads + f.v.n_heads;
-  if (threadIdx.x == 0) {
-    int nr = 0;
-    for (int j = 0; j < n_heads_tot; ++j) {
-      const int c0 = f.col[j], c1 = f.col[j] + f.rank[j];
-      if (c0 < n0 + kColsPerCta && c1 > n0) {
-        if (atomicAdd(&p.head_cnt[j], 1) + 1 == p.expect[j]) ready[nr++] = j;
+  if (rank == 0) {
+    for (int m = warp; m < M; m += kGemvThreads / 32) {
+      float vals[2];
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        const int d = lane + 32 * q2;
+        float val = 0.0f;
+        if (d < r) {
+          const int n = col0 + d;
+          if (INT) {
+            int acc = 0;
+#pragma unroll
+            for (int q = 0; q < kClusterE; ++q) acc += (int)cluster.map_shared_rank(part, q)[d * M + m];
+            val = __fmul_rn(__fmul_rn((float)acc, f.x_scale[m]), lk_f16_to_f32(f.a_scale[n]));
+          } else {
+#pragma unroll
+            for (int q = 0; q < kClusterE; ++q) val += __uint_as_float(cluster.map_shared_rank(part, q)[d * M + m]);
+          }
+        }
+        vals[q2] = val;
       }
+      append_values(f, m, j, vals[0], vals[1]);
     }
-    n_ready = nr;
   }
-  __syncthreads();
-  const int nr = n_ready;
-  if (nr == 0) return;
-  __threadfence();
-  for (int it = warp; it < nr * M; it += kGemvThreads / 32) {
-    const int j = ready[it / M], m = it % M;
-    append_head(f, m, m, j);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < nr; ++i) p.head_cnt[ready[i]] = 0;
+  cluster.sync();  // the other CTAs keep their partials until rank 0 has read them
+
+  if (rank == 0 && threadIdx.x == 0) {
     __threadfence();
-    if (atomicAdd(p.done_cnt, nr) + nr == n_heads_tot) {
+    const int n_heads_tot = f.k.n_heads + f.v.n_heads;
+    if (atomicAdd(p.done_cnt, 1) == n_heads_tot - 1) {  // every head appended: advance the rows
+      __threadfence();
       for (int b = 0; b < f.batch; ++b) f.seq_len[b] += f.n_new;
       *p.done_cnt = 0;
     }
@@ -328,10 +364,10 @@ __global__ void __launch_bounds__(kGemvThreads) proj_decode_kernel(const __grid_
 
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-// E-slice per CTA for the decode kernel: kDecU chunks of 16 bytes per lane.
-int decode_slice(int xtype) {
+// E-slice of each cluster CTA for the decode kernel (16-byte multiple).
+int cluster_slice(int E, int xtype) {
   const int ve = xtype == lk::X_F32 ? 4 : (xtype == lk::X_BF16 ? 8 : 16);
-  return 32 * ve * kDecU;
+  return round_up((E + kClusterE - 1) / kClusterE, ve);
 }
 
 int x_ve(int xtype) { return xtype == lk::X_F32 ? 4 : (xtype == lk::X_BF16 ? 8 : 16); }
@@ -350,9 +386,7 @@ size_t project_workspace_bytes(int rows, int n_tot, int embed_dim, int xtype, in
   (void)num_sms;
   size_t body;
   if (rows <= kGemvMaxRows) {
-    const int slice = decode_slice(xtype);
-    const int nks = (embed_dim + slice - 1) / slice;
-    body = (size_t)nks * rows * n_tot * 4;
+    body = 0;  // partials stay in the cluster's shared memory
   } else {
     body = (size_t)std::min(rows, kPrefillRowChunk) * n_tot * 4;
   }
@@ -398,10 +432,8 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
   cudaError_t e;
 
   if (rows <= kGemvMaxRows) {
-    DecodeProjParams d{};
-    const int slice = decode_slice(a.xtype);
-    const int nks = (a.embed_dim + slice - 1) / slice;
-    f.n_ksplit = nks;
+    ClusterProjParams d{};
+    f.n_ksplit = 1;
     f.ws_rows = rows;
     f.row0 = 0;
     f.rows = rows;
@@ -411,28 +443,42 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
     d.A = a.A;
     d.M = rows;
     d.E = a.embed_dim;
-    d.slice = slice;
+    d.slice = cluster_slice(a.embed_dim, a.xtype);
     d.done_cnt = static_cast<int32_t*>(a.workspace);
-    d.head_cnt = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(a.workspace) + 256);
-    for (int j = 0; j < heads_tot; ++j) {
-      const int c0 = f.col[j], c1 = f.col[j] + f.rank[j] - 1;
-      d.expect[j] = (int16_t)((c1 / kColsPerCta - c0 / kColsPerCta + 1) * nks);
-    }
-    const size_t smem = (size_t)rows * slice * x_size(a.xtype);
-    dim3 grid((a.n_tot + kColsPerCta - 1) / kColsPerCta, nks);
-    if (a.xtype == X_F32) {
-      e = cudaFuncSetAttribute(proj_decode_kernel<X_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      proj_decode_kernel<X_F32><<<grid, kGemvThreads, smem, stream>>>(d);
-    } else if (a.xtype == X_BF16) {
-      e = cudaFuncSetAttribute(proj_decode_kernel<X_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      proj_decode_kernel<X_BF16><<<grid, kGemvThreads, smem, stream>>>(d);
-    } else {
-      e = cudaFuncSetAttribute(proj_decode_kernel<X_I8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      proj_decode_kernel<X_I8><<<grid, kGemvThreads, smem, stream>>>(d);
-    }
+    const size_t smem = (size_t)LK_MAX_RANK * rows * 4 + (size_t)rows * d.slice * x_size(a.xtype);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kClusterE, heads_tot, 1);
+    cfg.blockDim = dim3(kGemvThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kClusterE;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int mt = rows <= 1 ? 1 : (rows <= 2 ? 2 : (rows <= 4 ? 4 : 8));
+#define LK_PROJ_LAUNCH(XTV, MTV)                                                                         \
+  do {                                                                                                \
+    e = cudaFuncSetAttribute(proj_cluster_kernel<XTV, MTV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             (int)smem);                                                             \
+    if (e != cudaSuccess) return e;                                                                   \
+    e = cudaLaunchKernelEx(&cfg, proj_cluster_kernel<XTV, MTV>, d);                                  \
+  } while (0)
+#define LK_PROJ_MT(XTV)                          \
+  do {                                           \
+    if (mt == 1) LK_PROJ_LAUNCH(XTV, 1);         \
+    else if (mt == 2) LK_PROJ_LAUNCH(XTV, 2);    \
+    else if (mt == 4) LK_PROJ_LAUNCH(XTV, 4);    \
+    else LK_PROJ_LAUNCH(XTV, 8);                 \
+  } while (0)
+    if (a.xtype == X_F32) LK_PROJ_MT(X_F32);
+    else if (a.xtype == X_BF16) LK_PROJ_MT(X_BF16);
+    else LK_PROJ_MT(X_I8);
+#undef LK_PROJ_MT
+#undef LK_PROJ_LAUNCH
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
 
