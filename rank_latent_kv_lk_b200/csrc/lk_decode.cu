@@ -28,6 +28,9 @@
 #include "lk_common.cuh"
 #include "lk_internal.h"
 
+#include <cooperative_groups.h>
+namespace cg = cooperative_groups;
+
 namespace {
 
 constexpr int kCW = 8;                          // consumer warps
@@ -60,9 +63,10 @@ struct DecodeParams {
   float qscale;  // softmax_scale * log2(e)
   // bytes of the shared-memory regions (max over heads), multiples of 128
   int st_kc, st_vc, st_ks, st_vs;
-  int st_bv, st_tw;
+  int st_q, st_bk, st_bv, st_tw;
   int nstages;
   int q_size, b_size;  // element sizes of q and of the factors
+  int cluster_merge;   // the n_split CTAs of a head form one thread-block cluster
   uint8_t rk[LK_MAX_HEADS];
   uint8_t rv[LK_MAX_HEADS];
 };
@@ -263,7 +267,7 @@ LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom
 struct SmemLayout {
   int stage_bytes;
   int off_kc, off_vc, off_ks, off_vs;  // within a stage
-  int off_bv;                          // B_V^h staged once per CTA
+  int off_q, off_bk, off_bv;           // q^h, B_K^h, B_V^h staged once per CTA
   int off_tw;                          // per consumer warp: weight expansion bytes [ngv][3][32]
   int off_qt;                          // q~ [kMaxR] floats
   int off_qterm;                       // q~ expansion bytes [3][kMaxR]
@@ -285,7 +289,9 @@ LK_DEVICE SmemLayout smem_layout(const DecodeParams& p) {
   L.off_ks = p.st_kc + p.st_vc;
   L.off_vs = p.st_kc + p.st_vc + p.st_ks;
   L.stage_bytes = p.st_kc + p.st_vc + p.st_ks + p.st_vs;
-  L.off_bv = p.nstages * L.stage_bytes;
+  L.off_q = p.nstages * L.stage_bytes;
+  L.off_bk = L.off_q + p.st_q;
+  L.off_bv = L.off_bk + p.st_bk;
   L.off_tw = L.off_bv + p.st_bv;
   L.off_qt = L.off_tw + p.st_tw;
   L.off_qterm = L.off_qt + kMaxR * 4;
@@ -300,7 +306,7 @@ LK_DEVICE SmemLayout smem_layout(const DecodeParams& p) {
 
 inline int smem_bytes_for(const DecodeParams& p) {
   const int stage = p.st_kc + p.st_vc + p.st_ks + p.st_vs;
-  return p.nstages * stage + p.st_bv + p.st_tw + kSmemFixed;
+  return p.nstages * stage + p.st_q + p.st_bk + p.st_bv + p.st_tw + kSmemFixed;
 }
 
 template <int KIND, int CSK, int CSV>
@@ -322,32 +328,44 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
   const int ssz = KIND == 0 ? 4 : 2;
   const int64_t bh = (int64_t)b * p.n_heads + h;
 
-  // ---- absorb q (consumer threads): q~[i] = qscale * sum_d B_K[i][d] q[d], from
-  //      global memory with every load of a thread in flight at once
+  auto issue = [&](int j) {  // stage j of this split -> buffer j % NS
+    const int buf = j % NS;
+    const int64_t t0 = (int64_t)(first_stage + j) * kStageT;
+    const int64_t end = min((int64_t)((len + 15) & ~15), (int64_t)p.capacity);
+    const int ntok = (int)min((int64_t)kStageT, end - t0);
+    uint8_t* st = smem + buf * L.stage_bytes;
+    const uint32_t bkc = ntok * g.rbk, bvc = ntok * g.rbv;
+    const uint32_t bks = ntok * g.ngk * ssz, bvs = ntok * g.ngv * ssz;
+    lk_mbar_arrive_expect_tx(&full[buf], bkc + bvc + bks + bvs);
+    lk_bulk_g2s(st + L.off_kc, p.codes_k + g.kc_off + t0 * g.rbk, bkc, &full[buf]);
+    lk_bulk_g2s(st + L.off_vc, p.codes_v + g.vc_off + t0 * g.rbv, bvc, &full[buf]);
+    lk_bulk_g2s(st + L.off_ks, p.scales_k + (g.ks_off + t0 * g.ngk) * ssz, bks, &full[buf]);
+    lk_bulk_g2s(st + L.off_vs, p.scales_v + (g.vs_off + t0 * g.ngv) * ssz, bvs, &full[buf]);
+  };
+  // the producer starts the copies at once: B_V^h, then the first stages (the
+  // buffers are free), so they stream in while q is absorbed
+  if (tid == kConsumerThreads) {
+    const uint32_t qb = H * p.q_size, bkb = g.rk * H * p.b_size, bvb = g.rv * H * p.b_size;
+    lk_mbar_arrive_expect_tx(fbar, qb + bkb + bvb);
+    lk_bulk_g2s(smem + L.off_q, static_cast<const uint8_t*>(p.q) + bh * H * p.q_size, qb, fbar);
+    lk_bulk_g2s(smem + L.off_bk, static_cast<const uint8_t*>(p.BK) + g.bk_off * p.b_size, bkb, fbar);
+    lk_bulk_g2s(smem + L.off_bv, static_cast<const uint8_t*>(p.BV) + g.bv_off * p.b_size, bvb, fbar);
+    for (int j = 0; j < min(NS, n_my); ++j) issue(j);
+  }
+
+  // ---- absorb q (consumer warps): q~[i] = qscale * sum_d B_K[i][d] q[d] from the
+  //      staged copies of q^h and B_K^h
   if (warp < kCW) {
-    int rp2 = 4;
-    while (rp2 < g.rk) rp2 <<= 1;
-    const int tpr = min(32, kConsumerThreads / rp2);  // threads per row (a power of two)
-    const int rows_per_pass = kConsumerThreads / tpr;
-    const int part = tid % tpr;
-    const int64_t qoff = bh * H;
-    const int npass = (g.rk + rows_per_pass - 1) / rows_per_pass;
-    for (int ps = 0; ps < npass; ++ps) {
-      const int i = tid / tpr + ps * rows_per_pass;
-      float acc = 0.0f;
-      if (i < g.rk) {
-#pragma unroll 8
-        for (int d = part; d < H; d += tpr) {
-          const float qd = p.q_bf16 ? lk_bf16_to_f32(reinterpret_cast<const uint16_t*>(p.q)[qoff + d])
-                                    : reinterpret_cast<const float*>(p.q)[qoff + d];
-          const int64_t bi = g.bk_off + (int64_t)i * H + d;
-          const float bk = p.b_bf16 ? lk_bf16_to_f32(reinterpret_cast<const uint16_t*>(p.BK)[bi])
-                                    : reinterpret_cast<const float*>(p.BK)[bi];
-          acc = fmaf(qd, bk, acc);
-        }
+    if (!lk_mbar_wait_bounded(fbar, 0, LK_WAIT_LIMIT_NS)) *abort_flag = 1;
+    const uint8_t* qs = smem + L.off_q;
+    const uint8_t* bks = smem + L.off_bk;
+    if (!*abort_flag) {
+      for (int i = warp; i < g.rk; i += kCW) {
+        float acc = 0.0f;
+        for (int d = lane; d < H; d += 32) acc = fmaf(ld_f(qs, d, p.q_bf16), ld_f(bks, i * H + d, p.b_bf16), acc);
+        acc = lk_warp_sum(acc);
+        if (lane == 0) qt_s[i] = acc * p.qscale;
       }
-      for (int o = 1; o < tpr; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (part == 0 && i < g.rk) qt_s[i] = acc * p.qscale;
     }
   }
   __syncthreads();
@@ -380,25 +398,8 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
   if (warp == kCW) {
     // ================= producer warp: bulk copies, gated by the empty barriers
     if (lane == 0) {
-      auto issue = [&](int j) {  // stage j of this split -> buffer j % NS
-        const int buf = j % NS;
-        const int64_t t0 = (int64_t)(first_stage + j) * kStageT;
-        const int64_t end = min((int64_t)((len + 15) & ~15), (int64_t)p.capacity);
-        const int ntok = (int)min((int64_t)kStageT, end - t0);
-        uint8_t* st = smem + buf * L.stage_bytes;
-        const uint32_t bkc = ntok * g.rbk, bvc = ntok * g.rbv;
-        const uint32_t bks = ntok * g.ngk * ssz, bvs = ntok * g.ngv * ssz;
-        lk_mbar_arrive_expect_tx(&full[buf], bkc + bvc + bks + bvs);
-        lk_bulk_g2s(st + L.off_kc, p.codes_k + g.kc_off + t0 * g.rbk, bkc, &full[buf]);
-        lk_bulk_g2s(st + L.off_vc, p.codes_v + g.vc_off + t0 * g.rbv, bvc, &full[buf]);
-        lk_bulk_g2s(st + L.off_ks, p.scales_k + (g.ks_off + t0 * g.ngk) * ssz, bks, &full[buf]);
-        lk_bulk_g2s(st + L.off_vs, p.scales_v + (g.vs_off + t0 * g.ngv) * ssz, bvs, &full[buf]);
-      };
-      const uint32_t bvb = g.rv * H * p.b_size;
-      lk_mbar_arrive_expect_tx(fbar, bvb);
-      lk_bulk_g2s(smem + L.off_bv, static_cast<const uint8_t*>(p.BV) + g.bv_off * p.b_size, bvb, fbar);
-      int issued = 0;
-      for (int j = 0; j < n_my; ++j) {
+      int issued = min(NS, n_my);
+      for (int j = issued; j < n_my; ++j) {
         if (*abort_flag) break;
         if (j >= NS) {  // the consumers released this buffer's previous stage
           if (!lk_mbar_wait_bounded(&empty[j % NS], (uint32_t)(((j / NS) - 1) & 1), LK_WAIT_LIMIT_NS)) {
@@ -570,7 +571,30 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
   __syncthreads();
 
   const int idx = (tid < g.rv) ? 2 + tid : (tid == kMaxR ? 1 : -1);
-  if (p.n_split > 1) {
+  if (p.cluster_merge) {
+    // the head's splits form one cluster: rank 0 merges the partials straight
+    // from the other CTAs' shared memory
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const unsigned nrank = cluster.num_blocks();
+    const bool lead = cluster.block_rank() == 0;
+    float acc = 0.0f, Mg = -INFINITY;
+    if (lead) {
+      for (unsigned q = 0; q < nrank; ++q) Mg = fmaxf(Mg, cluster.map_shared_rank(cta, q)[0]);
+      if (idx >= 0 && Mg != -INFINITY) {
+        for (unsigned q = 0; q < nrank; ++q) {
+          const float* pq = cluster.map_shared_rank(cta, q);
+          const float mq = pq[0];
+          if (mq != -INFINITY) acc += pq[idx] * exp2f(mq - Mg);
+        }
+      }
+    }
+    cluster.sync();  // every rank's partial has been read
+    if (!lead) return;
+    if (idx >= 0) cta[idx] = acc;
+    if (tid == 0) cta[0] = Mg;
+    __syncthreads();
+  } else if (p.n_split > 1) {
     float* part = p.partials + (bh * p.n_split + split) * p.part_stride;
     for (int i = tid; i < 2 + g.rv; i += kThreads) part[i] = cta[i];
     __threadfence();
@@ -680,7 +704,7 @@ int decode_pick_split(int units, int max_len, int num_sms) {
   if (units >= num_sms) return 1;
   const int target = num_sms * 2;
   int s = (target + units - 1) / units;
-  s = std::max(1, std::min(s, stages));
+  s = std::max(1, std::min(std::min(s, stages), 8));  // <= 8: the splits merge inside one cluster
   return s;
 }
 
@@ -733,6 +757,8 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   p.st_vs = round_up(kStageT * ngv_max * ssz, 128);
   p.q_size = a.q_bf16 ? 2 : 4;
   p.b_size = a.b_bf16 ? 2 : 4;
+  p.st_q = round_up(a.head_dim * p.q_size, 128);
+  p.st_bk = round_up(rk_max * a.head_dim * p.b_size, 128);
   p.st_bv = round_up(rv_max * a.head_dim * p.b_size, 128);
   p.st_tw = kCW * round_up(ngv_max * kWTerms * 32, 16);
   // as many stages as fit while two CTAs share an SM (about 64 KB of copies
@@ -755,18 +781,32 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   p.counters = reinterpret_cast<int32_t*>(ws);
   p.partials = reinterpret_cast<float*>(ws + round_up(a.batch * a.n_heads * 4, 256));
 
+  // up to eight splits of a head merge inside a cluster (portable cluster size)
+  p.cluster_merge = (n_split > 1 && n_split <= 8) ? 1 : 0;
   const int smem = smem_bytes_for(p);
-  dim3 grid(n_split, a.n_heads, a.batch);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_split, a.n_heads, a.batch);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.cluster_merge ? n_split : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   cudaError_t e;
   if (a.kind == 0) {
     e = cudaFuncSetAttribute(decode_attn_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    decode_attn_kernel<0><<<grid, kThreads, smem, stream>>>(p);
+    e = cudaLaunchKernelEx(&cfg, decode_attn_kernel<0>, p);
   } else {
     e = cudaFuncSetAttribute(decode_attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    decode_attn_kernel<1><<<grid, kThreads, smem, stream>>>(p);
+    e = cudaLaunchKernelEx(&cfg, decode_attn_kernel<1>, p);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

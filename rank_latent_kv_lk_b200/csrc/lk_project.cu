@@ -237,17 +237,9 @@ __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid
   const int e0 = rank * p.slice;
   const int elen = max(0, min(p.slice, p.E - e0));
   const int chunks = elen / VE;
-  uint32_t* part = reinterpret_cast<uint32_t*>(smem_raw);                    // [kMaxR][M]
-  T* xs = reinterpret_cast<T*>(smem_raw + (size_t)LK_MAX_RANK * M * 4);      // [M][slice]
-  const T* x = static_cast<const T*>(p.x);
+  uint32_t* part = reinterpret_cast<uint32_t*>(smem_raw);  // [kMaxR][M]
+  const T* x = static_cast<const T*>(p.x);  // read through L1: every warp of the CTA uses the same slice
   const T* A = static_cast<const T*>(p.A);
-
-  for (int c = threadIdx.x; c < M * chunks; c += kGemvThreads) {
-    const int mm = c / chunks, cc = c % chunks;
-    *reinterpret_cast<uint4*>(xs + mm * p.slice + cc * VE) =
-        *reinterpret_cast<const uint4*>(x + (int64_t)mm * p.E + e0 + cc * VE);
-  }
-  __syncthreads();
 
   for (int cb = warp * kProjNC; cb < r; cb += (kGemvThreads / 32) * kProjNC) {
     for (int m0 = 0; m0 < M; m0 += MT) {
@@ -276,7 +268,7 @@ __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid
 #pragma unroll
             for (int i = 0; i < MT; ++i) {
               if (i < mt) {
-                const uint4 xv4 = *reinterpret_cast<const uint4*>(xs + (m0 + i) * p.slice + cc * VE);
+                const uint4 xv4 = __ldg(reinterpret_cast<const uint4*>(x + (int64_t)(m0 + i) * p.E + e0 + cc * VE));
                 if (INT) {
 #pragma unroll
                   for (int jj = 0; jj < kProjNC; ++jj) {
@@ -445,7 +437,7 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
     d.E = a.embed_dim;
     d.slice = cluster_slice(a.embed_dim, a.xtype);
     d.done_cnt = static_cast<int32_t*>(a.workspace);
-    const size_t smem = (size_t)LK_MAX_RANK * rows * 4 + (size_t)rows * d.slice * x_size(a.xtype);
+    const size_t smem = (size_t)LK_MAX_RANK * rows * 4;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kClusterE, heads_tot, 1);
     cfg.blockDim = dim3(kGemvThreads, 1, 1);
