@@ -155,8 +155,10 @@ size_t lk_latent_project_workspace_bytes(const lk_latent_cache* k_cache,
  *   s_t = softmax_scale * sigma_K[t] . (c_K[t] . q~)   (per group for int4)
  *   p = softmax(s);  u = sum_t p_t * sigma_V[t] * c_V[t]   (r_V values)
  *   out^h = u B_V^h                                  ([H])
- * computed split-K over t (flash-decoding) with per-split partials
- * (max, sum, u) merged in latent space.  K and V are never formed.
+ * computed split-K over t (flash-decoding): the (b, h, 224-token stage)
+ * items are dealt out in equal ranges to a fixed grid of CTAs; a (b, h) cut
+ * by a range boundary leaves partials (max, sum, u) that are merged in latent
+ * space by the last piece to finish.  K and V are never formed.
  *
  * q: [B, n_heads, head_dim], q_dtype LK_F32 or LK_BF16; head_dim a multiple
  *   of 8 (<= LK_MAX_HEAD_DIM); q, B_K and B_V 16-byte aligned (they are
@@ -168,11 +170,16 @@ size_t lk_latent_project_workspace_bytes(const lk_latent_cache* k_cache,
  *   bound on those values (<= capacity); positions past it are not read.
  *   A row with seq_len 0 gets a zero output.
  * out: [B, n_heads, head_dim], LK_F32 or LK_BF16.
- * n_split: number of sequence splits per (b, h); 0 picks one for the GPU.
- *   The result does not depend on it beyond float rounding.
- * workspace: lk_latent_decode_workspace_bytes(...) bytes, 256-B aligned; its
- *   first region holds per-(b, h) arrival counters that must be zero before
- *   the first call and that every completed call leaves zero.
+ * n_split: about how many pieces each (b, h) is cut into (grid = B * n_heads
+ *   * n_split CTAs, at most one per 224-token stage); 0 picks a grid that
+ *   fills the GPU.  The result does not depend on it beyond float rounding.
+ * workspace: lk_latent_decode_workspace_bytes(...) bytes, 256-B aligned.
+ *   Its first round_up(4 * B * n_heads, 256) bytes are per-(b, h) arrival
+ *   counters that must read zero at entry (a fresh zeroed buffer); every
+ *   completed call leaves them zero, so a replayed launch (CUDA graph) also
+ *   starts clean.  The partials that follow may cover the counters of a call
+ *   with another B * n_heads: clear that region before reusing a workspace
+ *   for another shape.  Calls sharing a workspace must not overlap on the GPU.
  */
 lk_status lk_latent_decode_attn(const lk_latent_cache* k_cache, const lk_latent_cache* v_cache,
                                 const void* q, lk_dtype q_dtype, const void* B_K,
@@ -205,8 +212,9 @@ size_t lk_latent_decode_workspace_bytes(const lk_latent_cache* k_cache,
  *    lower n_split or use lk_latent_decode_attn with a workspace.
  *  - All calls share the one array: calls that overlap on the GPU (other
  *    streams, other host threads) race on it.  Serialise them.
- *  - The counters start at zero when the library loads; after each launch
- *    the call clears them again on `stream`.
+ *  - The arrival counters in the array start at zero when the library loads
+ *    and every completed call leaves them zero; a call whose B * n_heads
+ *    differs from the device's previous call first clears them on `stream`.
  */
 #define LK_DECODE_NOALLOC_SCRATCH_BYTES (4u << 20)
 lk_status lk_latent_decode_attn_noalloc(const lk_latent_cache* k_cache, const lk_latent_cache* v_cache,

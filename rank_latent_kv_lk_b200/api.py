@@ -124,7 +124,9 @@ def latent_decode_attn(k_cache, v_cache, q, B_K, B_V, seq_len, max_seq_len, soft
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     need = lib.lk_latent_decode_workspace_bytes(k_cache.desc(), v_cache.desc(), int(max_seq_len), int(n_split))
-    ws = workspaces.get("decode", need, q.device)
+    # one buffer per B * n_heads: the counters at its start must read zero, and
+    # the partials of another shape could cover them
+    ws = workspaces.get(("decode", k_cache.batch * len(k_cache.ranks)), need, q.device)
     check(lib.lk_latent_decode_attn(
         k_cache.desc(), v_cache.desc(), _ptr(q), _dtype_code(q), _ptr(B_K), _ptr(B_V), _dtype_code(B_K), H,
         _ptr(seq_len), int(max_seq_len), float(softmax_scale), _ptr(out), _dtype_code(out), int(n_split),

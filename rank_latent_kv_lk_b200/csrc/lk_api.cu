@@ -73,9 +73,7 @@ lk_status check_cache(const lk_latent_cache* c, const char* name, bool need_buff
 size_t decode_ws_bytes(const lk_latent_cache* k, const lk_latent_cache* v, int max_seq_len, int n_split) {
   int rv_max = 0;
   for (int h = 0; h < v->n_heads; ++h) rv_max = std::max(rv_max, v->ranks[h]);
-  const int stages = std::max(1, (max_seq_len + 127) / 128);
-  const int s = n_split > 0 ? std::min(n_split, stages) : stages;
-  return lk::decode_workspace_bytes(k->batch, k->n_heads, rv_max, s);
+  return lk::decode_workspace_bytes(k->batch * k->n_heads, rv_max, max_seq_len, n_split);
 }
 
 }  // namespace
@@ -256,8 +254,7 @@ lk_status lk_latent_decode_attn(const lk_latent_cache* k, const lk_latent_cache*
   a.b_bf16 = b_dtype == LK_BF16;
   a.out_bf16 = out_dtype == LK_BF16;
   a.max_len = max_seq_len;
-  const int stages = std::max(1, (max_seq_len + 127) / 128);
-  a.n_split = n_split > 0 ? std::min(n_split, stages) : 0;
+  a.n_split = n_split;
   a.num_sms = num_sms();
   a.softmax_scale = softmax_scale;
   cudaError_t e = lk::launch_decode_attn(a, reinterpret_cast<cudaStream_t>(stream));

@@ -202,3 +202,13 @@ LK_DEVICE void lk_bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes,
 }
 
 static constexpr uint64_t LK_WAIT_LIMIT_NS = 2000000000ull;  // 2 s
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may start while
+// the previous kernel on its stream still runs; it must call lk_grid_dep_wait
+// before touching anything that kernel writes (the wait returns once the
+// previous grid has completed and its memory is visible; without the launch
+// attribute it returns at once).  lk_grid_dep_launch lets such a dependent
+// kernel be scheduled early.
+LK_DEVICE void lk_grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+LK_DEVICE void lk_grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }

@@ -1,48 +1,69 @@
-// Latent decode attention, split-K over the sequence (sm_100a).
+// Latent decode attention on B200 (sm_100a): a persistent, stream-K
+// flash-decode over the per-head latent cache.
 //
-// Per (batch row b, head h, split s) one CTA of 256 threads:
-//   1. absorbs q into latent space, q~ = B_K^h q * softmax_scale * log2(e)
-//      (WSVD page §2C: the fused kernel works from the per-head latents;
-//      without positional rotation (q B_K^T) C^T equals q K^T), and writes
-//      q~ as a three-term int8 expansion q~ = a (t0 + t1/254 + t2/254^2)
-//      (error <= 6e-8 of max|q~|, i.e. float32 level);
-//   2. streams its slice of the latent cache (K codes, V codes and their
-//      scales) HBM -> shared memory with bulk copies on the TMA engine,
-//      2 or 3 stages deep, one mbarrier per stage;
-//   3. per stage of 256 tokens (three block barriers):
-//      a. one token per thread: s_t = sigma_K (c_K . q~) with exact int32
-//         dp4a dot products against the expansion;
-//      b. a CTA-uniform running max, p_t = 2^(s_t - max), running sum;
-//      c. u += p_t sigma_V c_V: the stage's weights w_t = p_t sigma_V[t] are
-//         written as a three-term int8 expansion relative to
-//         W = max_t p_t * max_t sigma_V[t] >= every w_t (both maxima come out
-//         of the score reduction; error <= 6e-8 W per weight), and each
-//         lane takes exact int32 dp4a sums over 4 (int8) or 8 (int4) tokens
-//         of one latent dim at a time from the dimension-major V layout; one
-//         float fold per stage;
-//   4. reduces (max, sum, u) over the CTA into a partial in latent space; the
-//      last CTA of the (b, h) to arrive (atomic ticket, no waiting) merges
-//      all partials and applies out = (u / sum) B_V^h.
-// K and V are never formed; the per-token traffic is the latent codes and
-// their scales.
+// What it computes (WSVD page, technical summary §2A and §2C): for every batch
+// row b and head h, softmax(q K^T / sqrt(H)) V with K = dequant(C_K) B_K and
+// V = dequant(C_V) B_V, without forming K or V.  Without positional rotation
+// q K^T = (B_K q)^T dequant(C_K)^T, so q is absorbed once per head
+// (q~ = B_K q) and scores are taken against the latent codes; the
+// probability-weighted latent sum u = sum_t p_t dequant(c_V[t]) is up-projected
+// once, out = (u / sum_t p_t) B_V.
+//
+// Work split.  A (b, h) pair is a unit; a unit's tokens are cut into stages
+// of 224.  The (unit, stage) items, in unit order, are dealt out in equal
+// contiguous ranges to a fixed grid of CTAs (two per SM by default), so every
+// SM streams the same number of bytes and each CTA pays its start-up once.  A
+// CTA walks its range: at a unit boundary it absorbs the next q (its q and B_K
+// copies were prefetched while the previous unit streamed), then streams the
+// unit's stages through an NS-deep ring of shared-memory buffers filled with
+// bulk copies (TMA engine) by a producer warp.  A unit that lies inside one
+// CTA is finished there; a unit cut by range boundaries leaves one partial
+// (m, l, u) per piece, and the piece that arrives last (atomic ticket, no
+// waiting) merges them and writes the output.
+//
+// Per stage, each of 7 consumer warps takes 32 tokens:
+//   a. score, one token per lane: s_t = sigma_K[t] (c_K[t] . q~), exact int32
+//      dp4a sums against a three-term int8 expansion of q~
+//      (q~ = a (t0 + t1/254 + t2/254^2), error <= 6e-8 max|q~|);
+//   b. running max by warp vote, p_t = 2^(s_t - m);
+//   c. w_t = p_t sigma_V[t] as four int8 terms relative to a reference scale,
+//      then u_d += sum_t w_t c_V[t][d] as exact int8 tensor-core products
+//      [4 terms x 32 tokens] x [32 tokens x 8 dims] (mma.sync m16n8k32),
+//      folded into float only when the max or the reference changes.
+// Every wait on a shared-memory barrier is bounded (2 s); an expired wait
+// sets the library status word, stops the math and lets the CTA finish its
+// protocol steps, so no other CTA waits on it.
+#include <atomic>
+#include <map>
+#include <mutex>
+#include <tuple>
+
 #include "lk_common.cuh"
 #include "lk_internal.h"
 
-#include <cooperative_groups.h>
-namespace cg = cooperative_groups;
-
 namespace {
 
-constexpr int kCW = 8;                          // consumer warps
+// 7 consumer warps + 1 producer warp: two CTAs of 8 warps fill an SM with 4
+// warps per scheduler and leave each thread 128 registers (a ninth warp would
+// put 5 warps on one scheduler and cap every thread at 96)
+constexpr int kCW = 7;                           // consumer warps
 constexpr int kConsumerThreads = kCW * 32;
-constexpr int kWTerms = 4;                      // int8 terms of the weight expansion
 constexpr int kThreads = kConsumerThreads + 32;  // + one producer warp
-constexpr int kStageT = 256;   // tokens per pipeline stage: one per thread in the score phase
-constexpr int kMaxStages = 8;  // pipeline depth chosen at launch (2 .. 8)
+constexpr int kStageT = 32 * kCW;                // tokens per stage (224): 32 per consumer warp
+constexpr int kMaxStages = 8;                    // ring depth chosen at launch (2 .. 8)
 constexpr int kMaxR = LK_MAX_RANK;
-constexpr int kMaxWords = kMaxR / 4;  // 32-bit words of q~ terms (int8 per dim)
-constexpr int kMaxGroups = 8;
-constexpr int kMaxSplit = 256;
+constexpr int kAutoCtaBound = 1024;              // grid bound of the automatic split (sizes the workspace)
+
+// Per-head geometry, computed on the host (prefix sums over the heads of a
+// batch row).
+struct HeadInfo {
+  uint8_t rk, rv;     // ranks
+  uint8_t ngk, ngv;   // scale groups per token (1 for int8)
+  uint8_t gk, gv;     // effective group sizes (int4; = rank for int8)
+  uint16_t pk, pv;    // code bytes of the heads before this one (one batch row)
+  uint16_t pgk, pgv;  // scale groups of the heads before this one
+  uint16_t prk, prv;  // ranks of the heads before this one (offset of B_K^h / B_V^h rows)
+};
 
 struct DecodeParams {
   const uint8_t* codes_k;
@@ -54,28 +75,29 @@ struct DecodeParams {
   const void* BV;
   const int32_t* seq_len;
   void* out;
-  float* partials;    // [B * n_heads][n_split][part_stride]
-  int32_t* counters;  // [B * n_heads]
-  int batch, n_heads, head_dim, capacity;
-  int group_k, group_v;  // int4 requested group size (effective min(g, r))
+  float* partials;    // [G][2][part_stride]: a CTA's first and last unit pieces
+  int32_t* counters;  // [units] arrival tickets, zero at entry, left zero
+  int n_heads, head_dim, capacity;
+  int tk, tv, tgk, tgv;  // code bytes / scale groups of one batch row (all heads)
   int q_bf16, b_bf16, out_bf16;
-  int n_split, stages_per_split, part_stride, max_len;
+  int max_len;
+  int S;   // stages per unit: ceil(max_len / kStageT)
+  int W;   // items: units * S
+  int G;   // CTAs
+  int part_stride;
   float qscale;  // softmax_scale * log2(e)
   // bytes of the shared-memory regions (max over heads), multiples of 128
-  int st_kc, st_vc, st_ks, st_vs;
-  int st_q, st_bk, st_bv, st_tw;
+  int st_kc, st_vc, st_ks, st_vs, st_q, st_bk, st_bv, st_fr;
   int nstages;
   int q_size, b_size;  // element sizes of q and of the factors
-  int cluster_merge;   // the n_split CTAs of a head form one thread-block cluster
-  uint8_t rk[LK_MAX_HEADS];
-  uint8_t rv[LK_MAX_HEADS];
+  HeadInfo head[LK_MAX_HEADS];
 };
 
 struct HeadGeom {
   int rk, rv;      // ranks
   int rbk, rbv;    // code bytes per token
-  int ngk, ngv;    // scale groups per token (1 for int8)
-  int gk, gv;      // effective group size (int4)
+  int ngk, ngv;    // scale groups per token
+  int gk, gv;      // effective group sizes
   int64_t kc_off;  // byte offset of this (b, h) K code plane
   int64_t vc_off;
   int64_t ks_off;  // element offset of this (b, h) K scale plane
@@ -85,52 +107,47 @@ struct HeadGeom {
 };
 
 template <int KIND>
-LK_DEVICE int row_bytes(int r) { return KIND == 0 ? r : r / 2; }
-template <int KIND>
-LK_DEVICE int n_groups(int r, int g) { return KIND == 0 ? 1 : (r + g - 1) / g; }
-
-// Prefix sums over heads, computed by each warp with strided lanes + shuffles.
-template <int KIND>
-LK_DEVICE HeadGeom head_geometry(const DecodeParams& p, int b, int h) {
-  int lane = threadIdx.x & 31;
-  int pk = 0, pv = 0, tk = 0, tv = 0, pgk = 0, pgv = 0, tgk = 0, tgv = 0, prk = 0, prv = 0;
-  for (int i = lane; i < p.n_heads; i += 32) {
-    int rk = p.rk[i], rv = p.rv[i];
-    int bk = row_bytes<KIND>(rk), bv = row_bytes<KIND>(rv);
-    int gk = n_groups<KIND>(rk, min(p.group_k, rk)), gv = n_groups<KIND>(rv, min(p.group_v, rv));
-    tk += bk; tv += bv; tgk += gk; tgv += gv;
-    if (i < h) { pk += bk; pv += bv; pgk += gk; pgv += gv; prk += rk; prv += rv; }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    pk += __shfl_xor_sync(0xffffffffu, pk, o);
-    pv += __shfl_xor_sync(0xffffffffu, pv, o);
-    tk += __shfl_xor_sync(0xffffffffu, tk, o);
-    tv += __shfl_xor_sync(0xffffffffu, tv, o);
-    pgk += __shfl_xor_sync(0xffffffffu, pgk, o);
-    pgv += __shfl_xor_sync(0xffffffffu, pgv, o);
-    tgk += __shfl_xor_sync(0xffffffffu, tgk, o);
-    tgv += __shfl_xor_sync(0xffffffffu, tgv, o);
-    prk += __shfl_xor_sync(0xffffffffu, prk, o);
-    prv += __shfl_xor_sync(0xffffffffu, prv, o);
-  }
+LK_DEVICE HeadGeom unit_geometry(const DecodeParams& p, int b, int h) {
+  const HeadInfo& hi = p.head[h];
   HeadGeom g;
-  g.rk = p.rk[h];
-  g.rv = p.rv[h];
-  g.rbk = row_bytes<KIND>(g.rk);
-  g.rbv = row_bytes<KIND>(g.rv);
-  g.gk = KIND == 0 ? g.rk : min(p.group_k, g.rk);
-  g.gv = KIND == 0 ? g.rv : min(p.group_v, g.rv);
-  g.ngk = n_groups<KIND>(g.rk, g.gk);
-  g.ngv = n_groups<KIND>(g.rv, g.gv);
+  g.rk = hi.rk;
+  g.rv = hi.rv;
+  g.rbk = KIND == 0 ? g.rk : g.rk / 2;
+  g.rbv = KIND == 0 ? g.rv : g.rv / 2;
+  g.ngk = hi.ngk;
+  g.ngv = hi.ngv;
+  g.gk = hi.gk;
+  g.gv = hi.gv;
   const int64_t cap = p.capacity;
-  g.kc_off = ((int64_t)b * tk + pk) * cap;
-  g.vc_off = ((int64_t)b * tv + pv) * cap;
-  g.ks_off = ((int64_t)b * tgk + pgk) * cap;
-  g.vs_off = ((int64_t)b * tgv + pgv) * cap;
-  g.bk_off = (int64_t)prk * p.head_dim;
-  g.bv_off = (int64_t)prv * p.head_dim;
+  g.kc_off = ((int64_t)b * p.tk + hi.pk) * cap;
+  g.vc_off = ((int64_t)b * p.tv + hi.pv) * cap;
+  g.ks_off = ((int64_t)b * p.tgk + hi.pgk) * cap;
+  g.vs_off = ((int64_t)b * p.tgv + hi.pgv) * cap;
+  g.bk_off = (int64_t)hi.prk * p.head_dim;
+  g.bv_off = (int64_t)hi.prv * p.head_dim;
   return g;
+}
+
+LK_DEVICE int unit_len(const DecodeParams& p, int b) { return max(0, min(p.seq_len[b], p.max_len)); }
+
+// First item of CTA c, and the CTA that holds item i.
+LK_DEVICE int cta_first(const DecodeParams& p, int c) { return (int)((int64_t)c * p.W / p.G); }
+LK_DEVICE int cta_of(const DecodeParams& p, int i) { return (int)(((int64_t)(i + 1) * p.G - 1) / p.W); }
+
+// Barrier over the consumer warps only (the producer warp never joins).
+LK_DEVICE void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory"); }
+// The same barrier, returning whether any consumer thread passed `pred`.
+LK_DEVICE bool consumer_sync_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "n"(kConsumerThreads)
+      : "memory");
+  return r != 0;
 }
 
 // Loads the code chunk `c` (CS bytes) of local token `tl` from a staged
@@ -171,25 +188,7 @@ LK_DEVICE float ld_f(const uint8_t* base, int i, int is_bf16) {
                  : reinterpret_cast<const float*>(base)[i];
 }
 
-// Expands code word `wd` into fp32 values: 4 signed bytes (int8) or 8 signed
-// nibbles (int4, low nibble = even dim).  Exact integers.
-template <int KIND>
-LK_DEVICE void expand_word(uint32_t wd, float* f) {
-  if (KIND == 0) {
-    const uint32_t x = wd ^ 0x80808080u;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) f[k] = lk_s8_from_xored(x, k);
-  } else {
-    const uint32_t x = wd ^ 0x88888888u;        // each nibble n -> c + 8
-    const uint32_t ev = x & 0x0F0F0F0Fu;         // dims 0, 2, 4, 6
-    const uint32_t od = (x >> 4) & 0x0F0F0F0Fu;  // dims 1, 3, 5, 7
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      f[2 * k] = __uint_as_float(__byte_perm(ev, 0x4B000000u, 0x7540u | k)) - 8388616.0f;
-      f[2 * k + 1] = __uint_as_float(__byte_perm(od, 0x4B000000u, 0x7540u | k)) - 8388616.0f;
-    }
-  }
-}
+
 
 // Signed int4 nibbles of a word as signed int8 bytes: `ev` gets the low
 // nibbles (elements 0, 2, 4, 6), `od` the high ones (1, 3, 5, 7).  Setting
@@ -204,12 +203,91 @@ LK_DEVICE void nibbles_to_s8(uint32_t x, int& ev, int& od) {
 constexpr float kInv254 = 1.0f / 254.0f;
 constexpr float kInv254sq = 1.0f / (254.0f * 254.0f);
 
+constexpr float kInv254cu = 1.0f / (254.0f * 254.0f * 254.0f);
+
+// Four int8 terms t_i of x in [0, 127]: x = t0 + t1/254 + t2/254^2 + t3/254^3
+// up to 127/254^4 (each remainder lies in [-1/2, 1/2], so |t_i| <= 127),
+// packed little-endian into one word (byte i = t_i).
+LK_DEVICE uint32_t expand_weight(float x) {
+  x = fminf(x, 127.0f);
+  const float t0 = rintf(x);
+  x = (x - t0) * 254.0f;
+  const float t1 = rintf(x);
+  x = (x - t1) * 254.0f;
+  const float t2 = rintf(x);
+  x = (x - t2) * 254.0f;
+  const float t3 = rintf(x);
+  const uint32_t lo = __byte_perm((uint32_t)(int)t0, (uint32_t)(int)t1, 0x0040u);
+  const uint32_t hi = __byte_perm((uint32_t)(int)t2, (uint32_t)(int)t3, 0x0040u);
+  return __byte_perm(lo, hi, 0x5410u);
+}
+
+// Lane L holds the four terms of k position L (byte i = term i).  Returns the
+// A fragments of an m16n8k32 int8 product whose row i (< 4) is term i over
+// the 32 positions: a0 = row gid, positions 4 tig .. 4 tig + 3; a2 = the same
+// row, positions 16 + 4 tig ..; rows 4..15 are zero.  A 4 x 4 byte transpose
+// inside each quad of lanes (two exchanges) puts term c of positions
+// 4q .. 4q + 3 in lane 4q + c; two shuffles fetch the fragments.
+LK_DEVICE void weight_frags(uint32_t w, uint32_t sel1, uint32_t sel2, int gid, int tig, uint32_t& a0,
+                            uint32_t& a2) {
+  w = __byte_perm(w, __shfl_xor_sync(0xffffffffu, w, 1), sel1);
+  w = __byte_perm(w, __shfl_xor_sync(0xffffffffu, w, 2), sel2);
+  a0 = __shfl_sync(0xffffffffu, w, (4 * tig + gid) & 31);
+  a2 = __shfl_sync(0xffffffffu, w, (16 + 4 * tig + gid) & 31);
+  if (gid >= 4) a0 = a2 = 0u;
+}
+
+// D = A B + C for a 16 x 32 int8 A (rows gid + 8 zero: a1 = a3 = 0) and a
+// 32 x 8 int8 B; exact int32.  Only the rows < 8 of C/D are carried.
+LK_DEVICE void mma_s8_rows8(uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1, int& c0, int& c1) {
+  int d2, d3;
+  asm(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %11, %12, %13};"
+      : "=r"(c0), "=r"(c1), "=r"(d2), "=r"(d3)
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "r"(c0), "r"(c1), "r"(0), "r"(0));
+  (void)d2;
+  (void)d3;
+}
+
+// B fragment word of the V product: the codes of latent dim d for the four
+// k positions 4 tig .. 4 tig + 3 of one 16-token block (dimension-major
+// block layout).  int4: positions 4 tig + m are tokens 8 (tig / 2) + 2 m +
+// (tig % 2), i.e. the low (even tokens) or high (odd tokens) nibbles of one
+// word, sign-extended to bytes.
+template <int KIND>
+LK_DEVICE uint32_t v_frag(const uint8_t* blk, int d, int tig) {
+  if (KIND == 0) return *reinterpret_cast<const uint32_t*>(blk + d * 16 + tig * 4);
+  const uint32_t w = *reinterpret_cast<const uint32_t*>(blk + d * 8 + (tig >> 1) * 4);
+  const uint32_t x = (w >> ((tig & 1) * 4)) & 0x0F0F0F0Fu;
+  return x | ((x & 0x08080808u) * 0x1Eu);
+}
+
+// Loads N consecutive 32-bit words from shared memory (16-byte aligned for
+// N >= 4, 8-byte for N = 2).
+template <int N>
+LK_DEVICE void lds_words(const void* p, uint32_t (&w)[N]) {
+  if constexpr (N == 1) {
+    w[0] = *reinterpret_cast<const uint32_t*>(p);
+  } else if constexpr (N == 2) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    w[0] = v.x; w[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const uint4 v = reinterpret_cast<const uint4*>(p)[i];
+      w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+    }
+  }
+}
+
 // Score of one token in log2 units: sum over groups g of
 //   sigma_g * a * (D0 + D1/254 + D2/254^2),  D_i = c . t_i  (exact dp4a sums)
-// (int8 keys: one group and one scale per token).
+// with the q~ terms t_i read from shared memory (the same words for every
+// lane: broadcast loads).  int8 keys: one group and one scale per token.
 template <int KIND, int CS>
 LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom& g, int tl,
-                            const uint32_t (&qw)[3][kMaxWords], float qa) {
+                            const int8_t* qterm, float qa) {
   constexpr int WPC = CS / 4;  // words per chunk
   constexpr int MAXCH = (KIND == 0 ? kMaxR : kMaxR / 2) / CS;
   const int nch = g.rbk / CS;
@@ -220,12 +298,15 @@ LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom
       if (c < nch) {
         Chunk<CS> ch;
         ch.load(kc, g.rbk, tl, c);
+        uint32_t t0[WPC], t1[WPC], t2[WPC];
+        lds_words<WPC>(qterm + 0 * kMaxR + c * CS, t0);
+        lds_words<WPC>(qterm + 1 * kMaxR + c * CS, t1);
+        lds_words<WPC>(qterm + 2 * kMaxR + c * CS, t2);
 #pragma unroll
         for (int wi = 0; wi < WPC; ++wi) {
-          const int w = c * WPC + wi;
-          d0 = __dp4a((int)ch.w[wi], (int)qw[0][w], d0);
-          d1 = __dp4a((int)ch.w[wi], (int)qw[1][w], d1);
-          d2 = __dp4a((int)ch.w[wi], (int)qw[2][w], d2);
+          d0 = __dp4a((int)ch.w[wi], (int)t0[wi], d0);
+          d1 = __dp4a((int)ch.w[wi], (int)t1[wi], d1);
+          d2 = __dp4a((int)ch.w[wi], (int)t2[wi], d2);
         }
       }
     }
@@ -235,12 +316,17 @@ LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom
     float s = 0.0f;
     int d0 = 0, d1 = 0, d2 = 0;
     int cur_g = 0;
-    // code word w holds dims 8w .. 8w+7; groups are multiples of 8 dims
+    // code word w holds dims 8w .. 8w+7 (q~ bytes 8w .. 8w+7: even dims, then
+    // odd dims); groups are multiples of 8 dims
 #pragma unroll
     for (int c = 0; c < MAXCH; ++c) {
       if (c < nch) {
         Chunk<CS> ch;
         ch.load(kc, g.rbk, tl, c);
+        uint32_t t0[2 * WPC], t1[2 * WPC], t2[2 * WPC];
+        lds_words<2 * WPC>(qterm + 0 * kMaxR + c * 2 * CS, t0);
+        lds_words<2 * WPC>(qterm + 1 * kMaxR + c * 2 * CS, t1);
+        lds_words<2 * WPC>(qterm + 2 * kMaxR + c * 2 * CS, t2);
 #pragma unroll
         for (int wi = 0; wi < WPC; ++wi) {
           const int w = c * WPC + wi;
@@ -253,9 +339,9 @@ LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom
           }
           int ev, od;
           nibbles_to_s8(ch.w[wi], ev, od);
-          d0 = __dp4a(od, (int)qw[0][2 * w + 1], __dp4a(ev, (int)qw[0][2 * w], d0));
-          d1 = __dp4a(od, (int)qw[1][2 * w + 1], __dp4a(ev, (int)qw[1][2 * w], d1));
-          d2 = __dp4a(od, (int)qw[2][2 * w + 1], __dp4a(ev, (int)qw[2][2 * w], d2));
+          d0 = __dp4a(od, (int)t0[2 * wi + 1], __dp4a(ev, (int)t0[2 * wi], d0));
+          d1 = __dp4a(od, (int)t1[2 * wi + 1], __dp4a(ev, (int)t1[2 * wi], d1));
+          d2 = __dp4a(od, (int)t2[2 * wi + 1], __dp4a(ev, (int)t2[2 * wi], d2));
         }
       }
     }
@@ -264,23 +350,23 @@ LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom
   }
 }
 
+
 struct SmemLayout {
   int stage_bytes;
   int off_kc, off_vc, off_ks, off_vs;  // within a stage
-  int off_q, off_bk, off_bv;           // q^h, B_K^h, B_V^h staged once per CTA
-  int off_tw;                          // per consumer warp: weight expansion bytes [ngv][3][32]
+  int off_q, off_bk;                   // factor slot: q^h and B_K^h of the current or next unit
+  int off_bv;                          // B_V^h of the current unit
+  int off_fr;                          // per consumer warp: V weight fragments [ngv][32 lanes] (several groups)
   int off_qt;                          // q~ [kMaxR] floats
   int off_qterm;                       // q~ expansion bytes [3][kMaxR]
   int off_wst;                         // per consumer warp: (m, l, u[kMaxR])
-  int off_cta;                         // CTA partial [2 + kMaxR]
-  int off_mw;                          // merge weights [kMaxSplit]
-  int off_bar;                         // full[kMaxStages], empty[kMaxStages], factor barrier
-  int off_misc;
-  int total;
+  int off_cta;                         // CTA state of the unit [2 + kMaxR]
+  int off_bar;                         // full[kMaxStages], empty[kMaxStages], factor full, factor empty, B_V full
+  int off_misc;                        // abort flag, ticket flag, q~ expansion scale
 };
 
-constexpr int kSmemFixed = kMaxR * 4 + 3 * kMaxR + kCW * (2 + kMaxR) * 4 + (2 + kMaxR) * 4 + kMaxSplit * 4 +
-                           (2 * kMaxStages + 1) * 8 + 16;
+constexpr int kSmemFixed = kMaxR * 4 + 3 * kMaxR + kCW * (2 + kMaxR) * 4 + (2 + kMaxR) * 4 +
+                           (2 * kMaxStages + 4) * 8 + 16;
 
 LK_DEVICE SmemLayout smem_layout(const DecodeParams& p) {
   SmemLayout L;
@@ -292,84 +378,144 @@ LK_DEVICE SmemLayout smem_layout(const DecodeParams& p) {
   L.off_q = p.nstages * L.stage_bytes;
   L.off_bk = L.off_q + p.st_q;
   L.off_bv = L.off_bk + p.st_bk;
-  L.off_tw = L.off_bv + p.st_bv;
-  L.off_qt = L.off_tw + p.st_tw;
+  L.off_fr = L.off_bv + p.st_bv;
+  L.off_qt = L.off_fr + p.st_fr;
   L.off_qterm = L.off_qt + kMaxR * 4;
   L.off_wst = L.off_qterm + 3 * kMaxR;
   L.off_cta = L.off_wst + kCW * (2 + kMaxR) * 4;
-  L.off_mw = L.off_cta + (2 + kMaxR) * 4;
-  L.off_bar = L.off_mw + kMaxSplit * 4;
-  L.off_misc = L.off_bar + (2 * kMaxStages + 1) * 8;
-  L.total = L.off_misc + 16;
+  L.off_bar = L.off_cta + (2 + kMaxR) * 4;
+  L.off_misc = L.off_bar + (2 * kMaxStages + 4) * 8;
   return L;
 }
 
 inline int smem_bytes_for(const DecodeParams& p) {
   const int stage = p.st_kc + p.st_vc + p.st_ks + p.st_vs;
-  return p.nstages * stage + p.st_q + p.st_bk + p.st_bv + p.st_tw + kSmemFixed;
+  return p.nstages * stage + p.st_q + p.st_bk + p.st_bv + p.st_fr + kSmemFixed;
 }
 
-template <int KIND, int CSK, int CSV>
-LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* smem, const SmemLayout& L,
-                           int b, int h, int split, int len, int first_stage, int n_my) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int H = p.head_dim;
+struct Bars {
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* fbar;    // factor slot filled
+  uint64_t* fempty;  // factor slot released by every consumer warp
+  uint64_t* vbar;    // B_V slot filled
+  volatile int* abort_flag;
+  int* ticket_flag;
+  float* qa;
+};
+
+LK_DEVICE Bars bars_of(uint8_t* smem, const SmemLayout& L) {
+  Bars B;
+  B.full = reinterpret_cast<uint64_t*>(smem + L.off_bar);
+  B.empty = B.full + kMaxStages;
+  B.fbar = B.full + 2 * kMaxStages;
+  B.fempty = B.fbar + 1;
+  B.vbar = B.fbar + 2;
+  B.abort_flag = reinterpret_cast<volatile int*>(smem + L.off_misc);
+  B.ticket_flag = reinterpret_cast<int*>(smem + L.off_misc) + 1;
+  B.qa = reinterpret_cast<float*>(smem + L.off_misc) + 2;
+  return B;
+}
+
+// ------------------------------------------------------------------ producer
+// One thread: for every unit of the CTA's range, the factor copies (q^h,
+// B_K^h) once the consumers released the slot, then each non-empty stage once
+// its ring buffer is free.
+template <int KIND>
+LK_DEVICE void produce(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, int i0, int i1) {
+  const Bars B = bars_of(smem, L);
   const int NS = p.nstages;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.off_bar);
-  uint64_t* empty = full + kMaxStages;
-  uint64_t* fbar = full + 2 * kMaxStages;
+  const int H = p.head_dim;
+  const int ssz = KIND == 0 ? 4 : 2;
+  int u = i0 / p.S, s = i0 - u * p.S;
+  int it = i0, k = 0, nunit = 0, nf = 0;  // stages issued, units begun, factor copies issued
+  bool ok = true;
+  while (it < i1) {
+    const int s_end = min(p.S, s + (i1 - it));
+    const int b = u / p.n_heads, h = u - b * p.n_heads;
+    const HeadGeom g = unit_geometry<KIND>(p, b, h);
+    const int len = unit_len(p, b);
+    if (ok && nunit > 0 && !lk_mbar_wait_bounded(B.fempty, (uint32_t)((nunit - 1) & 1), LK_WAIT_LIMIT_NS)) {
+      *B.abort_flag = 1;
+      ok = false;
+    }
+    if (ok) {
+      const uint32_t qb = H * p.q_size, bkb = g.rk * H * p.b_size;
+      lk_mbar_arrive_expect_tx(B.fbar, qb + bkb);
+      lk_bulk_g2s(smem + L.off_q, static_cast<const uint8_t*>(p.q) + (int64_t)(b * p.n_heads + h) * H * p.q_size, qb,
+                  B.fbar);
+      lk_bulk_g2s(smem + L.off_bk, static_cast<const uint8_t*>(p.BK) + g.bk_off * p.b_size, bkb, B.fbar);
+      ++nf;
+    }
+    ++nunit;
+    const int64_t end = min((int64_t)((len + 15) & ~15), (int64_t)p.capacity);
+    for (int ss = s; ss < s_end && ok; ++ss) {
+      const int64_t t0 = (int64_t)ss * kStageT;
+      if (t0 >= len) break;  // this and the unit's later stages hold no tokens
+      if (*B.abort_flag) {
+        ok = false;
+        break;
+      }
+      const int buf = k % NS;
+      if (k >= NS && !lk_mbar_wait_bounded(&B.empty[buf], (uint32_t)(((k / NS) - 1) & 1), LK_WAIT_LIMIT_NS)) {
+        *B.abort_flag = 1;
+        ok = false;
+        break;
+      }
+      const int ntok = (int)min((int64_t)kStageT, end - t0);
+      uint8_t* st = smem + buf * L.stage_bytes;
+      const uint32_t bkc = ntok * g.rbk, bvc = ntok * g.rbv;
+      const uint32_t bks = ntok * g.ngk * ssz, bvs = ntok * g.ngv * ssz;
+      lk_mbar_arrive_expect_tx(&B.full[buf], bkc + bvc + bks + bvs);
+      lk_bulk_g2s(st + L.off_kc, p.codes_k + g.kc_off + t0 * g.rbk, bkc, &B.full[buf]);
+      lk_bulk_g2s(st + L.off_vc, p.codes_v + g.vc_off + t0 * g.rbv, bvc, &B.full[buf]);
+      lk_bulk_g2s(st + L.off_ks, p.scales_k + (g.ks_off + t0 * g.ngk) * ssz, bks, &B.full[buf]);
+      lk_bulk_g2s(st + L.off_vs, p.scales_v + (g.vs_off + t0 * g.ngv) * ssz, bvs, &B.full[buf]);
+      ++k;
+    }
+    it += s_end - s;
+    ++u;
+    s = 0;
+  }
+  // before the CTA may finish, every copy this CTA started has landed
+  for (int j = max(0, k - NS); j < k; ++j)
+    if (!lk_mbar_wait_bounded(&B.full[j % NS], (uint32_t)((j / NS) & 1), LK_WAIT_LIMIT_NS))
+      lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
+  if (nf > 0 && !lk_mbar_wait_bounded(B.fbar, (uint32_t)((nf - 1) & 1), LK_WAIT_LIMIT_NS))
+    lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
+}
+
+// ------------------------------------------------------------------ consumers
+// q~ of unit (b, h) from the staged q^h and B_K^h, then its three-term int8
+// expansion (warp 0).  `n` counts the units this CTA has begun.
+template <int KIND>
+LK_DEVICE void absorb_q(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, const HeadGeom& g, int n) {
+  const Bars B = bars_of(smem, L);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int H = p.head_dim;
   float* qt_s = reinterpret_cast<float*>(smem + L.off_qt);
   int8_t* qterm = reinterpret_cast<int8_t*>(smem + L.off_qterm);
-  float* wst = reinterpret_cast<float*>(smem + L.off_wst);
-  float* cta = reinterpret_cast<float*>(smem + L.off_cta);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.off_misc);
-  int* flag = reinterpret_cast<int*>(smem + L.off_misc) + 1;
-  float* qa_s = reinterpret_cast<float*>(smem + L.off_misc) + 2;
-  const int ssz = KIND == 0 ? 4 : 2;
-  const int64_t bh = (int64_t)b * p.n_heads + h;
-
-  auto issue = [&](int j) {  // stage j of this split -> buffer j % NS
-    const int buf = j % NS;
-    const int64_t t0 = (int64_t)(first_stage + j) * kStageT;
-    const int64_t end = min((int64_t)((len + 15) & ~15), (int64_t)p.capacity);
-    const int ntok = (int)min((int64_t)kStageT, end - t0);
-    uint8_t* st = smem + buf * L.stage_bytes;
-    const uint32_t bkc = ntok * g.rbk, bvc = ntok * g.rbv;
-    const uint32_t bks = ntok * g.ngk * ssz, bvs = ntok * g.ngv * ssz;
-    lk_mbar_arrive_expect_tx(&full[buf], bkc + bvc + bks + bvs);
-    lk_bulk_g2s(st + L.off_kc, p.codes_k + g.kc_off + t0 * g.rbk, bkc, &full[buf]);
-    lk_bulk_g2s(st + L.off_vc, p.codes_v + g.vc_off + t0 * g.rbv, bvc, &full[buf]);
-    lk_bulk_g2s(st + L.off_ks, p.scales_k + (g.ks_off + t0 * g.ngk) * ssz, bks, &full[buf]);
-    lk_bulk_g2s(st + L.off_vs, p.scales_v + (g.vs_off + t0 * g.ngv) * ssz, bvs, &full[buf]);
-  };
-  // the producer starts the copies at once: B_V^h, then the first stages (the
-  // buffers are free), so they stream in while q is absorbed
-  if (tid == kConsumerThreads) {
-    const uint32_t qb = H * p.q_size, bkb = g.rk * H * p.b_size, bvb = g.rv * H * p.b_size;
-    lk_mbar_arrive_expect_tx(fbar, qb + bkb + bvb);
-    lk_bulk_g2s(smem + L.off_q, static_cast<const uint8_t*>(p.q) + bh * H * p.q_size, qb, fbar);
-    lk_bulk_g2s(smem + L.off_bk, static_cast<const uint8_t*>(p.BK) + g.bk_off * p.b_size, bkb, fbar);
-    lk_bulk_g2s(smem + L.off_bv, static_cast<const uint8_t*>(p.BV) + g.bv_off * p.b_size, bvb, fbar);
-    for (int j = 0; j < min(NS, n_my); ++j) issue(j);
+  if (threadIdx.x == 0 && !*B.abort_flag) {
+    // B_V^h is read when the unit ends; the previous unit's output is done
+    // (the slot is free) and its copy was waited for
+    const uint32_t bvb = g.rv * H * p.b_size;
+    lk_mbar_arrive_expect_tx(B.vbar, bvb);
+    lk_bulk_g2s(smem + L.off_bv, static_cast<const uint8_t*>(p.BV) + g.bv_off * p.b_size, bvb, B.vbar);
   }
-
-  // ---- absorb q (consumer warps): q~[i] = qscale * sum_d B_K[i][d] q[d] from the
-  //      staged copies of q^h and B_K^h
-  if (warp < kCW) {
-    if (!lk_mbar_wait_bounded(fbar, 0, LK_WAIT_LIMIT_NS)) *abort_flag = 1;
+  if (!*B.abort_flag && !lk_mbar_wait_bounded(B.fbar, (uint32_t)(n & 1), LK_WAIT_LIMIT_NS)) *B.abort_flag = 1;
+  if (!*B.abort_flag) {
     const uint8_t* qs = smem + L.off_q;
     const uint8_t* bks = smem + L.off_bk;
-    if (!*abort_flag) {
-      for (int i = warp; i < g.rk; i += kCW) {
-        float acc = 0.0f;
-        for (int d = lane; d < H; d += 32) acc = fmaf(ld_f(qs, d, p.q_bf16), ld_f(bks, i * H + d, p.b_bf16), acc);
-        acc = lk_warp_sum(acc);
-        if (lane == 0) qt_s[i] = acc * p.qscale;
-      }
+    for (int i = warp; i < g.rk; i += kCW) {
+      float acc = 0.0f;
+      for (int d = lane; d < H; d += 32) acc = fmaf(ld_f(qs, d, p.q_bf16), ld_f(bks, i * H + d, p.b_bf16), acc);
+      acc = lk_warp_sum(acc);
+      if (lane == 0) qt_s[i] = acc * p.qscale;
     }
   }
-  __syncthreads();
-  // ---- three-term int8 expansion of q~ (warp 0): q~ = a (t0 + t1/254 + t2/254^2)
+  __syncwarp();
+  if (lane == 0) lk_mbar_arrive(B.fempty);  // this warp is done with the factor slot
+  consumer_sync();
   if (warp == 0) {
     const float v0 = lane < g.rk ? qt_s[lane] : 0.0f;
     const float v1 = lane + 32 < g.rk ? qt_s[lane + 32] : 0.0f;
@@ -391,304 +537,358 @@ LK_DEVICE void decode_body(const DecodeParams& p, const HeadGeom& g, uint8_t* sm
       qterm[1 * kMaxR + pos] = (int8_t)(live ? (int)t1 : 0);
       qterm[2 * kMaxR + pos] = (int8_t)(live ? (int)t2 : 0);
     }
-    if (lane == 0) *qa_s = a;
+    if (lane == 0) *B.qa = a;
   }
-  __syncthreads();
+  consumer_sync();
+}
 
-  if (warp == kCW) {
-    // ================= producer warp: bulk copies, gated by the empty barriers
-    if (lane == 0) {
-      int issued = min(NS, n_my);
-      for (int j = issued; j < n_my; ++j) {
-        if (*abort_flag) break;
-        if (j >= NS) {  // the consumers released this buffer's previous stage
-          if (!lk_mbar_wait_bounded(&empty[j % NS], (uint32_t)(((j / NS) - 1) & 1), LK_WAIT_LIMIT_NS)) {
-            *abort_flag = 1;
-            break;
-          }
-        }
-        issue(j);
-        issued = j + 1;
-      }
-      // before the CTA may finish, every copy this CTA started has landed
-      for (int j = max(0, issued - NS); j < issued; ++j) {
-        if (!lk_mbar_wait_bounded(&full[j % NS], (uint32_t)((j / NS) & 1), LK_WAIT_LIMIT_NS)) {
-          lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
-          *abort_flag = 1;
-        }
-      }
-      if (!lk_mbar_wait_bounded(fbar, 0, LK_WAIT_LIMIT_NS)) {
-        lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
-        *abort_flag = 1;
+// The stages [s0, s1) of one unit (tokens below len), then this warp's state
+// (m, l, u) in shared memory.  buf / phase: ring position and parity of the
+// CTA's next stage, carried across units.  NM = ceil(r_V / 8) V products per
+// stage, fixed at compile time (runtime bounds on these loops cost more
+// instructions than the products themselves).
+template <int KIND, int CSK, int NM, bool VG1>
+LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, const HeadGeom& g, int len,
+                        int s0, int s1, int& buf, uint32_t& phase) {
+  const Bars B = bars_of(smem, L);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int NS = p.nstages;
+  const int8_t* qterm = reinterpret_cast<const int8_t*>(smem + L.off_qterm);
+  float* wst = reinterpret_cast<float*>(smem + L.off_wst);
+  const float qa = *B.qa;
+  const int gid = lane >> 2, tig = lane & 3;
+  // Score phase: lane L takes token tok(L) of the warp's 32 (int4: the even
+  // tokens of each octet before the odd ones), so that lane order is the k
+  // order of the V products.
+  const int tok = KIND == 0 ? lane : (lane & 16) | (((lane >> 3) & 1) << 3) | ((lane & 3) << 1) | ((lane >> 2) & 1);
+  const int tl = 32 * warp + tok;  // this lane's token within a stage
+  const uint32_t sel1 = (lane & 1) ? 0x3715u : 0x6240u;
+  const uint32_t sel2 = (lane & 2) ? 0x3276u : 0x5410u;
+  const float fterm = gid == 0 ? 1.0f : gid == 1 ? kInv254 : gid == 2 ? kInv254sq : gid == 3 ? kInv254cu : 0.0f;
+  uint2* fr = reinterpret_cast<uint2*>(smem + L.off_fr) + warp * (p.st_fr / (kCW * 8));
+  int acc[NM][2];
+#pragma unroll
+  for (int j = 0; j < NM; ++j) acc[j][0] = acc[j][1] = 0;
+  float u[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};  // lanes < 16: MMAs j = gid and gid + 4
+  float m_run = -INFINITY, l_run = 0.0f;
+  float wref = 0.0f;  // every weight of the open accumulation is <= wref
+  float inv = 0.0f;   // 127 / wref
+  auto fold = [&](float alpha) {
+    const float sc = wref * (1.0f / 127.0f);
+#pragma unroll
+    for (int j = 0; j < NM; ++j) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float x = (float)acc[j][e] * fterm;
+        x += __shfl_xor_sync(0xffffffffu, x, 4);
+        x += __shfl_xor_sync(0xffffffffu, x, 8);
+        acc[j][e] = 0;
+        if ((j & 3) == gid) u[j >> 2][e] = (u[j >> 2][e] + sc * x) * alpha;
       }
     }
-  } else {
-    // ================= consumer warp: tokens 32 * warp .. 32 * warp + 31 of every stage
-    const float qa = *qa_s;
-    uint32_t qw[3][kMaxWords];
-#pragma unroll
-    for (int i = 0; i < 3; ++i)
-#pragma unroll
-      for (int w = 0; w < kMaxWords; ++w) qw[i][w] = reinterpret_cast<const uint32_t*>(qterm + i * kMaxR)[w];
-    // weight-expansion bytes of this warp: [group][term][32 tokens]
-    int8_t* tw = reinterpret_cast<int8_t*>(smem + L.off_tw) + warp * (p.st_tw / kCW);
-    const int tl = 32 * warp + lane;  // this lane's token within a stage
-    // int4 values: even and odd tokens of an octet live in separate words
-    const int tpos = KIND == 0 ? lane : (lane & ~7) + ((lane & 1) ? 4 : 0) + ((lane & 7) >> 1);
-    // V: this lane owns latent dims lane and lane + 32; exact int32 sums of
-    // (expanded weight term) x code, folded into float only when the running
-    // max or the reference scale changes
-    int A[2][kWTerms];
-    float u[2] = {0.0f, 0.0f};
-#pragma unroll
-    for (int k = 0; k < 2; ++k)
-#pragma unroll
-      for (int i = 0; i < kWTerms; ++i) A[k][i] = 0;
-    float m_run = -INFINITY, l_run = 0.0f;
-    float wref = 0.0f;  // every weight of the open accumulation is <= wref
-    auto fold = [&](float alpha) {
-      const float sc = wref * (1.0f / 127.0f);
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        float x = (float)A[k][kWTerms - 1];
-#pragma unroll
-        for (int i = kWTerms - 2; i >= 0; --i) x = fmaf(x, kInv254, (float)A[k][i]);
-        u[k] = (u[k] + sc * x) * alpha;
-#pragma unroll
-        for (int i = 0; i < kWTerms; ++i) A[k][i] = 0;
-      }
-    };
+  };
 
-    for (int j = 0; j < n_my; ++j) {
-      const int buf = j % NS;
-      if (!lk_mbar_wait_bounded(&full[buf], (uint32_t)((j / NS) & 1), LK_WAIT_LIMIT_NS)) *abort_flag = 1;
-      if (*abort_flag) break;
-      const uint8_t* st = smem + buf * L.stage_bytes;
-      const uint8_t* vs = st + L.off_vs;
-      const bool valid = (first_stage + j) * kStageT + tl < len;
-      // a. score; a new running max (warp vote) folds the open sums
-      float s = -INFINITY;
-      if (valid) s = token_score<KIND, CSK>(st + L.off_kc, st + L.off_ks, g, tl, qw, qa);
-      if (__any_sync(0xffffffffu, s > m_run)) {
-        const float m_new = fmaxf(m_run, lk_warp_max(s));
-        const float alpha = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - m_new);
-        fold(alpha);
-        l_run *= alpha;
-        m_run = m_new;
+  const int tl_end = len - s0 * kStageT - tl;  // token (s0 + j) * kStageT + tl is valid iff j * kStageT < tl_end
+  for (int j = 0; j < s1 - s0; ++j) {
+    if ((s0 + j) * kStageT >= len) break;  // no copies were issued for the unit's later stages
+    if (*B.abort_flag) break;
+    if (!lk_mbar_wait_bounded(&B.full[buf], phase, LK_WAIT_LIMIT_NS)) *B.abort_flag = 1;
+    if (*B.abort_flag) break;
+    const uint8_t* st = smem + buf * L.stage_bytes;
+    const uint8_t* vs = st + L.off_vs;
+    const bool valid = j * kStageT < tl_end;
+    // a. score; a new running max (warp vote) folds the open sums
+    float s = -INFINITY;
+    if (valid) s = token_score<KIND, CSK>(st + L.off_kc, st + L.off_ks, g, tl, qterm, qa);
+    if (__any_sync(0xffffffffu, s > m_run)) {
+      const float m_new = fmaxf(m_run, lk_warp_max(s));
+      const float alpha = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - m_new);
+      fold(alpha);
+      l_run *= alpha;
+      m_run = m_new;
+    }
+    const float pr = valid ? exp2f(s - m_run) : 0.0f;
+    l_run += pr;
+    // b. V scales: a larger one (warp vote) folds, then raises wref; the
+    //    weights w = p sigma_V become four int8 terms of w * 127 / wref
+    const uint8_t* vc = st + L.off_vc + 2 * warp * 16 * g.rbv;  // the warp's two 16-token blocks
+    const uint8_t* vc1 = vc + 16 * g.rbv;
+    if (VG1) {
+      const float sg = valid ? load_scale(vs, tl, KIND) : 0.0f;
+      if (__any_sync(0xffffffffu, sg > wref)) {  // then some sg > 0, so wref > 0 below
+        fold(1.0f);
+        wref = fmaxf(wref, lk_warp_max(sg));
+        inv = 127.0f / wref;
       }
-      const float pr = valid ? exp2f(s - m_run) : 0.0f;
-      l_run += pr;
-      // b. reference scale: a larger V scale (warp vote) folds, then raises wref
+      uint32_t a0, a2;
+      weight_frags(expand_weight(pr * sg * inv), sel1, sel2, gid, tig, a0, a2);
+      // c. acc[jm] += terms x codes of dims 8 jm .. 8 jm + 7 (dims >= r_V only
+      //    in the last product, when r_V % 8 != 0)
+#pragma unroll
+      for (int jm = 0; jm < NM; ++jm) {
+        const int d = 8 * jm + gid;
+        const bool live = jm < NM - 1 || d < g.rv;
+        const uint32_t b0 = live ? v_frag<KIND>(vc, d, tig) : 0u;
+        const uint32_t b1 = live ? v_frag<KIND>(vc1, d, tig) : 0u;
+        mma_s8_rows8(a0, a2, b0, b1, acc[jm][0], acc[jm][1]);
+      }
+    } else {
       float smax_t = 0.0f;
       for (int gi = 0; gi < g.ngv; ++gi) smax_t = fmaxf(smax_t, valid ? load_scale(vs, tl * g.ngv + gi, KIND) : 0.0f);
       if (__any_sync(0xffffffffu, smax_t > wref)) {
         fold(1.0f);
         wref = fmaxf(wref, lk_warp_max(smax_t));
+        inv = 127.0f / wref;
       }
-      //    weights w = p sigma_V as a four-term int8 expansion of w * 127 / wref
-      const float inv = wref > 0.0f ? 127.0f / wref : 0.0f;
       for (int gi = 0; gi < g.ngv; ++gi) {
         const float sg = valid ? load_scale(vs, tl * g.ngv + gi, KIND) : 0.0f;
-        float x = fminf(pr * sg * inv, 127.0f);
-        int8_t* tg = tw + gi * (kWTerms * 32);
-#pragma unroll
-        for (int i = 0; i < kWTerms; ++i) {
-          const float t = fminf(fmaxf(rintf(x), -127.0f), 127.0f);
-          tg[32 * i + tpos] = (int8_t)(int)t;
-          x = (x - t) * 254.0f;
-        }
+        uint32_t a0, a2;
+        weight_frags(expand_weight(pr * sg * inv), sel1, sel2, gid, tig, a0, a2);
+        fr[gi * 32 + lane] = make_uint2(a0, a2);
       }
       __syncwarp();
-      // c. A[d][i] += sum over the warp's 32 tokens of term_i(t) * c_{t,d}
-      const uint8_t* vc = st + L.off_vc;
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int d = lane + 32 * k;
-        if (d < g.rv) {
-          const int gi = KIND == 0 ? 0 : d / g.gv;
-          const uint32_t* T = reinterpret_cast<const uint32_t*>(tw + gi * (kWTerms * 32));
-#pragma unroll
-          for (int blk = 0; blk < 2; ++blk) {  // the warp's two 16-token blocks
-            const int b16 = 2 * warp + blk;
-            if (KIND == 0) {
-              const uint4 v = *reinterpret_cast<const uint4*>(vc + b16 * 16 * g.rbv + d * 16);
-              const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-              for (int qd = 0; qd < 4; ++qd)
-#pragma unroll
-                for (int i = 0; i < kWTerms; ++i) A[k][i] = __dp4a((int)vw[qd], (int)T[8 * i + 4 * blk + qd], A[k][i]);
-            } else {
-              const uint2 v = *reinterpret_cast<const uint2*>(vc + b16 * 16 * g.rbv + d * 8);
-              const uint32_t vw[2] = {v.x, v.y};
-#pragma unroll
-              for (int oc = 0; oc < 2; ++oc) {
-                int ev, od;
-                nibbles_to_s8(vw[oc], ev, od);
-                const int o = 2 * blk + oc;  // octet of the warp's tokens
-#pragma unroll
-                for (int i = 0; i < kWTerms; ++i)
-                  A[k][i] = __dp4a(od, (int)T[8 * i + 2 * o + 1], __dp4a(ev, (int)T[8 * i + 2 * o], A[k][i]));
-              }
-            }
-          }
-        }
+      for (int jm = 0; jm < NM; ++jm) {
+        const uint2 a = fr[((8 * jm) / g.gv) * 32 + lane];
+        const int d = 8 * jm + gid;
+        const bool live = jm < NM - 1 || d < g.rv;
+        const uint32_t b0 = live ? v_frag<KIND>(vc, d, tig) : 0u;
+        const uint32_t b1 = live ? v_frag<KIND>(vc1, d, tig) : 0u;
+        mma_s8_rows8(a.x, a.y, b0, b1, acc[jm][0], acc[jm][1]);
       }
-      __syncwarp();  // this warp is done with the stage buffer and its weight bytes
-      if (lane == 0) lk_mbar_arrive(&empty[buf]);
     }
-    fold(1.0f);
-    // per-warp state (m, l, u)
-    const float lw = lk_warp_sum(l_run);
-    float* ws = wst + warp * (2 + kMaxR);
-    if (lane == 0) {
-      ws[0] = m_run;
-      ws[1] = lw;
+    __syncwarp();  // this warp is done with the stage buffer (and its fragment store)
+    if (lane == 0) lk_mbar_arrive(&B.empty[buf]);
+    if (++buf == NS) {
+      buf = 0;
+      phase ^= 1u;
     }
-    if (lane < g.rv) ws[2 + lane] = u[0];
-    if (lane + 32 < g.rv) ws[2 + lane + 32] = u[1];
+    if ((j & 255) == 255) fold(1.0f);  // int32 sums stay far from overflow
   }
-  __syncthreads();
-  const bool aborted = *abort_flag != 0;
-  if (aborted && tid == 0) lk_dev_fail(LK_DEV_TIMEOUT_PIPE);
-
-  // ---- merge the consumer warps' states into the CTA partial
-  {
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kCW; ++w) M = fmaxf(M, wst[w * (2 + kMaxR)]);
-    const int idx = (tid < g.rv) ? 2 + tid : (tid == kMaxR ? 1 : -1);
-    float acc = 0.0f;
-    if (idx >= 0 && M != -INFINITY && !aborted) {
-#pragma unroll
-      for (int w = 0; w < kCW; ++w) {
-        const float mw = wst[w * (2 + kMaxR)];
-        if (mw != -INFINITY) acc += wst[w * (2 + kMaxR) + idx] * exp2f(mw - M);
-      }
-    }
-    if (idx >= 0) cta[idx] = acc;
-    if (tid == 0) cta[0] = aborted ? -INFINITY : M;
+  fold(1.0f);
+  const float lw = lk_warp_sum(l_run);
+  float* ws = wst + warp * (2 + kMaxR);
+  if (lane == 0) {
+    ws[0] = m_run;
+    ws[1] = lw;
   }
-  __syncthreads();
-
-  const int idx = (tid < g.rv) ? 2 + tid : (tid == kMaxR ? 1 : -1);
-  if (p.cluster_merge) {
-    // the head's splits form one cluster: rank 0 merges the partials straight
-    // from the other CTAs' shared memory
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    const unsigned nrank = cluster.num_blocks();
-    const bool lead = cluster.block_rank() == 0;
-    float acc = 0.0f, Mg = -INFINITY;
-    if (lead) {
-      for (unsigned q = 0; q < nrank; ++q) Mg = fmaxf(Mg, cluster.map_shared_rank(cta, q)[0]);
-      if (idx >= 0 && Mg != -INFINITY) {
-        for (unsigned q = 0; q < nrank; ++q) {
-          const float* pq = cluster.map_shared_rank(cta, q);
-          const float mq = pq[0];
-          if (mq != -INFINITY) acc += pq[idx] * exp2f(mq - Mg);
-        }
+  if (gid < 4) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int jm = gid + 4 * k;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int d = 8 * jm + 2 * tig + e;
+        if (jm < NM && d < g.rv) ws[2 + d] = u[k][e];
       }
     }
-    cluster.sync();  // every rank's partial has been read
-    if (!lead) return;
-    if (idx >= 0) cta[idx] = acc;
-    if (tid == 0) cta[0] = Mg;
-    __syncthreads();
-  } else if (p.n_split > 1) {
-    float* part = p.partials + (bh * p.n_split + split) * p.part_stride;
-    for (int i = tid; i < 2 + g.rv; i += kThreads) part[i] = cta[i];
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-      const int ticket = atomicAdd(&p.counters[bh], 1);
-      *flag = (ticket == p.n_split - 1);
-    }
-    __syncthreads();
-    if (!*flag) return;
-    __threadfence();
-    // last arriver: merge every split's partial (all visible in L2), all
-    // splits' loads in flight at once
-    float* mw = reinterpret_cast<float*>(smem + L.off_mw);
-    const float* P0 = p.partials + bh * p.n_split * p.part_stride;
-    for (int s2 = tid; s2 < p.n_split; s2 += kThreads) mw[s2] = __ldcg(P0 + (int64_t)s2 * p.part_stride);
-    __syncthreads();
-    float Mg = -INFINITY;
-    for (int s2 = 0; s2 < p.n_split; ++s2) Mg = fmaxf(Mg, mw[s2]);
-    __syncthreads();
-    for (int s2 = tid; s2 < p.n_split; s2 += kThreads)
-      mw[s2] = (mw[s2] == -INFINITY || Mg == -INFINITY) ? 0.0f : exp2f(mw[s2] - Mg);
-    __syncthreads();
-    float acc = 0.0f;
-    if (idx >= 0) {
-      int s2 = 0;
-      for (; s2 + 4 <= p.n_split; s2 += 4) {
-        const float v0 = __ldcg(P0 + (int64_t)(s2 + 0) * p.part_stride + idx);
-        const float v1 = __ldcg(P0 + (int64_t)(s2 + 1) * p.part_stride + idx);
-        const float v2 = __ldcg(P0 + (int64_t)(s2 + 2) * p.part_stride + idx);
-        const float v3 = __ldcg(P0 + (int64_t)(s2 + 3) * p.part_stride + idx);
-        acc += v0 * mw[s2] + v1 * mw[s2 + 1] + v2 * mw[s2 + 2] + v3 * mw[s2 + 3];
-      }
-      for (; s2 < p.n_split; ++s2) acc += __ldcg(P0 + (int64_t)s2 * p.part_stride + idx) * mw[s2];
-    }
-    __syncthreads();
-    if (idx >= 0) cta[idx] = acc;
-    if (tid == 0) {
-      cta[0] = Mg;
-      p.counters[bh] = 0;  // ready for the next call
-    }
-    __syncthreads();
   }
+}
 
-  // ---- out = (u / l) B_V^h, B_V^h from shared memory
+template <int KIND, int CSK, bool VG1>
+LK_DEVICE void run_unit_nm(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, const HeadGeom& g, int len,
+                           int s0, int s1, int& buf, uint32_t& phase) {
+  switch ((g.rv + 7) >> 3) {
+    case 1: run_unit<KIND, CSK, 1, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
+    case 2: run_unit<KIND, CSK, 2, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
+    case 3: run_unit<KIND, CSK, 3, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
+    case 4: run_unit<KIND, CSK, 4, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
+    case 5: run_unit<KIND, CSK, 5, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
+    case 6: run_unit<KIND, CSK, 6, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
+    case 7: run_unit<KIND, CSK, 7, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
+    default: run_unit<KIND, CSK, 8, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
+  }
+}
+
+// Block-wide max over the consumer threads (red: kCW floats of shared memory).
+LK_DEVICE float consumer_max(float v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = lk_warp_max(v);
+  if (lane == 0) red[warp] = v;
+  consumer_sync();
+  float m = red[0];
+#pragma unroll
+  for (int w = 1; w < kCW; ++w) m = fmaxf(m, red[w]);
+  consumer_sync();  // red is free again
+  return m;
+}
+
+// out^h = (u / l) B_V^h from the CTA state, B_V^h staged in shared memory.
+LK_DEVICE void write_output(const DecodeParams& p, const uint8_t* bvs, const float* cta, const HeadGeom& g,
+                            int64_t bh, bool aborted) {
+  const int H = p.head_dim;
   const float lsum = cta[1];
   const float inv = (cta[0] == -INFINITY || lsum == 0.0f || aborted) ? 0.0f : 1.0f / lsum;
-  const uint8_t* bvs = smem + L.off_bv;
-  const int64_t ooff = bh * H;
-  for (int d = tid; d < H; d += kThreads) {
+  for (int d = threadIdx.x; d < H; d += kConsumerThreads) {
     float o = 0.0f;
     for (int j = 0; j < g.rv; ++j) o = fmaf(cta[2 + j], ld_f(bvs, j * H + d, p.b_bf16), o);
     o *= inv;
-    if (p.out_bf16) reinterpret_cast<uint16_t*>(p.out)[ooff + d] = lk_f32_to_bf16(o);
-    else reinterpret_cast<float*>(p.out)[ooff + d] = o;
+    if (p.out_bf16) reinterpret_cast<uint16_t*>(p.out)[bh * H + d] = lk_f32_to_bf16(o);
+    else reinterpret_cast<float*>(p.out)[bh * H + d] = o;
+  }
+}
+
+// Merges the warps' states into the unit's CTA state; then writes the output
+// (unit whole inside this CTA) or this piece's partial, and the last piece of
+// the unit to arrive merges every piece and writes the output.
+template <int KIND>
+LK_DEVICE void finish_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, const HeadGeom& g, int b,
+                           int h, int u, int seg_first, int seg_end, int i0, int c, int n) {
+  const Bars B = bars_of(smem, L);
+  const int tid = threadIdx.x;
+  float* wst = reinterpret_cast<float*>(smem + L.off_wst);
+  float* cta = reinterpret_cast<float*>(smem + L.off_cta);
+  // this unit's B_V copy has landed long ago; waiting here also keeps the next
+  // unit's copy from starting while this one is in flight
+  if (!*B.abort_flag && !lk_mbar_wait_bounded(B.vbar, (uint32_t)(n & 1), LK_WAIT_LIMIT_NS)) *B.abort_flag = 1;
+  const bool aborted = consumer_sync_or(*B.abort_flag != 0);  // every warp's state is written
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kCW; ++w) M = fmaxf(M, wst[w * (2 + kMaxR)]);
+  if (tid < 2 + g.rv) {
+    float acc = M;
+    if (tid > 0) {
+      acc = 0.0f;
+      if (M != -INFINITY && !aborted) {
+#pragma unroll
+        for (int w = 0; w < kCW; ++w) {
+          const float mw = wst[w * (2 + kMaxR)];
+          if (mw != -INFINITY) acc += wst[w * (2 + kMaxR) + tid] * exp2f(mw - M);
+        }
+      }
+    } else if (aborted) {
+      acc = -INFINITY;
+    }
+    cta[tid] = acc;
+  }
+  consumer_sync();  // cta[] is written; wst is free for the merge below
+  const int64_t bh = (int64_t)b * p.n_heads + h;
+  const int u0 = u * p.S, u1 = u0 + p.S;
+  if (seg_first == u0 && seg_end == u1) {  // the whole unit ran here
+    write_output(p, smem + L.off_bv, cta, g, bh, aborted);
+    consumer_sync();  // cta[] and the B_V slot are free for the next unit
+    return;
+  }
+  const int slot = seg_first == i0 ? 0 : 1;
+  float* part = p.partials + ((int64_t)c * 2 + slot) * p.part_stride;
+  if (tid < 2 + g.rv) part[tid] = cta[tid];
+  __threadfence();
+  consumer_sync();
+  const int c0 = cta_of(p, u0), c1 = cta_of(p, u1 - 1);
+  if (tid == 0) *B.ticket_flag = atomicAdd(&p.counters[u], 1) == c1 - c0;
+  consumer_sync();
+  const bool last = *B.ticket_flag != 0;
+  consumer_sync();  // every thread read the flag before the next unit may set it
+  if (!last) return;
+  __threadfence();
+  // last piece: merge every piece of the unit (partials visible in L2).  The
+  // pieces are CTAs c0 .. c1; only c0 may hold the unit in its second slot.
+  const int slot0 = cta_first(p, c0) >= u0 ? 0 : 1;
+  auto piece = [&](int cc) {
+    return p.partials + ((int64_t)cc * 2 + (cc == c0 ? slot0 : 0)) * p.part_stride;
+  };
+  float mloc = -INFINITY;
+  for (int cc = c0 + tid; cc <= c1; cc += kConsumerThreads) mloc = fmaxf(mloc, __ldcg(piece(cc)));
+  const float Mg = consumer_max(mloc, wst);
+  // warp w sums pieces w, w + kCW, ... (lanes over the state), then the warps'
+  // sums meet in shared memory
+  {
+    const int lane = tid & 31, warp = tid >> 5;
+    float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f;
+    if (Mg != -INFINITY) {
+      for (int cc = c0 + warp; cc <= c1; cc += kCW) {
+        const float* pc = piece(cc);
+        const float mc = __ldcg(pc);
+        const float v0 = lane < 2 + g.rv ? __ldcg(pc + lane) : 0.0f;
+        const float v1 = lane + 32 < 2 + g.rv ? __ldcg(pc + lane + 32) : 0.0f;
+        const float v2 = lane + 64 < 2 + g.rv ? __ldcg(pc + lane + 64) : 0.0f;
+        const float w = mc == -INFINITY ? 0.0f : exp2f(mc - Mg);
+        a0 = fmaf(w, v0, a0);
+        a1 = fmaf(w, v1, a1);
+        a2 = fmaf(w, v2, a2);
+      }
+    }
+    float* ws = wst + warp * (2 + kMaxR);
+    if (lane < 2 + g.rv) ws[lane] = a0;
+    if (lane + 32 < 2 + g.rv) ws[lane + 32] = a1;
+    if (lane + 64 < 2 + g.rv) ws[lane + 64] = a2;
+  }
+  consumer_sync();
+  if (tid == 0) {
+    cta[0] = Mg;
+    p.counters[u] = 0;  // ready for the next call (and for a replay of this launch)
+  } else if (tid < 2 + g.rv) {
+    float acc = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kCW; ++w) acc += wst[w * (2 + kMaxR) + tid];
+    cta[tid] = acc;
+  }
+  consumer_sync();
+  write_output(p, smem + L.off_bv, cta, g, bh, aborted);
+  consumer_sync();
+}
+
+template <int KIND>
+LK_DEVICE void consume(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, int i0, int i1, int c) {
+  int u = i0 / p.S, s = i0 - u * p.S;
+  int it = i0, n = 0, buf = 0;
+  uint32_t phase = 0u;
+  while (it < i1) {
+    const int s_end = min(p.S, s + (i1 - it));
+    const int seg_end = it + (s_end - s);
+    const int b = u / p.n_heads, h = u - b * p.n_heads;
+    const HeadGeom g = unit_geometry<KIND>(p, b, h);
+    const int len = unit_len(p, b);
+    absorb_q<KIND>(p, smem, L, g, n);
+    const int csk = lk_chunk_bytes(g.rbk);
+    if (KIND == 0 || g.ngv == 1) {
+      if (csk == 16) run_unit_nm<KIND, 16, true>(p, smem, L, g, len, s, s_end, buf, phase);
+      else if (csk == 8) run_unit_nm<KIND, 8, true>(p, smem, L, g, len, s, s_end, buf, phase);
+      else run_unit_nm<KIND, 4, true>(p, smem, L, g, len, s, s_end, buf, phase);
+    } else if constexpr (KIND == 1) {
+      if (csk == 16) run_unit_nm<KIND, 16, false>(p, smem, L, g, len, s, s_end, buf, phase);
+      else if (csk == 8) run_unit_nm<KIND, 8, false>(p, smem, L, g, len, s, s_end, buf, phase);
+      else run_unit_nm<KIND, 4, false>(p, smem, L, g, len, s, s_end, buf, phase);
+    }
+    finish_unit<KIND>(p, smem, L, g, b, h, u, it, seg_end, i0, c, n);
+    it = seg_end;
+    ++u;
+    ++n;
+    s = 0;
   }
 }
 
 template <int KIND>
 __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const SmemLayout L = smem_layout(p);
-  const HeadGeom g = head_geometry<KIND>(p, b, h);
-  int len = p.seq_len[b];
-  len = max(0, min(len, p.max_len));
-
-  const int total_stages = (len + kStageT - 1) / kStageT;
-  const int first_stage = split * p.stages_per_split;
-  const int n_my = max(0, min(p.stages_per_split, total_stages - first_stage));
-
+  const int c = blockIdx.x;
+  const int i0 = cta_first(p, c), i1 = cta_first(p, c + 1);
   if (threadIdx.x == 0) {
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.off_bar);
-    for (int i = 0; i < kMaxStages; ++i) lk_mbar_init(&bars[i], 1);                       // full
-    for (int i = kMaxStages; i < 2 * kMaxStages; ++i) lk_mbar_init(&bars[i], kCW);       // empty
-    lk_mbar_init(&bars[2 * kMaxStages], 1);                                              // factor
+    const Bars B = bars_of(smem, L);
+    for (int i = 0; i < kMaxStages; ++i) {
+      lk_mbar_init(&B.full[i], 1);
+      lk_mbar_init(&B.empty[i], kCW);
+    }
+    lk_mbar_init(B.fbar, 1);
+    lk_mbar_init(B.fempty, kCW);
+    lk_mbar_init(B.vbar, 1);
     lk_fence_mbar_init();
-    *reinterpret_cast<int*>(smem + L.off_misc) = 0;
+    *B.abort_flag = 0;
   }
   __syncthreads();
-
-  const int csk = lk_chunk_bytes(g.rbk), csv = lk_chunk_bytes(g.rbv);
-#define LK_BODY(A, B_) decode_body<KIND, A, B_>(p, g, smem, L, b, h, split, len, first_stage, n_my)
-  if (csk == 16) {
-    if (csv == 16) LK_BODY(16, 16); else if (csv == 8) LK_BODY(16, 8); else LK_BODY(16, 4);
-  } else if (csk == 8) {
-    if (csv == 16) LK_BODY(8, 16); else if (csv == 8) LK_BODY(8, 8); else LK_BODY(8, 4);
-  } else {
-    if (csv == 16) LK_BODY(4, 16); else if (csv == 8) LK_BODY(4, 8); else LK_BODY(4, 4);
+  // launched with programmatic stream serialisation, this CTA may run while
+  // the previous kernel on the stream (e.g. the latent append) finishes:
+  // nothing before this point reads global memory
+  lk_grid_dep_wait();
+  if (i0 >= i1) return;
+  if (threadIdx.x >= kConsumerThreads) {
+    if (threadIdx.x == kConsumerThreads) produce<KIND>(p, smem, L, i0, i1);
+    return;
   }
-#undef LK_BODY
+  consume<KIND>(p, smem, L, i0, i1, c);
+  if (threadIdx.x == 0 && *bars_of(smem, L).abort_flag) lk_dev_fail(LK_DEV_TIMEOUT_PIPE);
 }
-
-int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 }  // namespace
 
@@ -696,22 +896,48 @@ LK_DEFINE_STATUS_ACCESSOR(lk_decode_status_word)
 
 namespace lk {
 
-int decode_pick_split(int units, int max_len, int num_sms) {
-  const int stages = (max_len + kStageT - 1) / kStageT;
-  if (stages <= 1) return 1;
-  // splitting only pays while the (batch, head) units leave SMs idle: with
-  // two resident CTAs per SM, aim for about one full wave
-  if (units >= num_sms) return 1;
-  const int target = num_sms * 2;
-  int s = (target + units - 1) / units;
-  s = std::max(1, std::min(std::min(s, stages), 8));  // <= 8: the splits merge inside one cluster
-  return s;
-}
+namespace {
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-size_t decode_workspace_bytes(int batch, int n_heads, int rv_max, int n_split) {
-  const size_t counters = (size_t)round_up(batch * n_heads * 4, 256);
+// Resident CTAs per SM of the decode kernel for `smem` bytes of shared memory
+// (cached per device, kind and size; the query costs a few microseconds).
+int decode_occupancy(int kind, int smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  const auto key = std::make_tuple(dev, kind, smem);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int occ = 0;
+  cudaError_t e = kind == 0
+                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_attn_kernel<0>, kThreads, smem)
+                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_attn_kernel<1>, kThreads, smem);
+  if (e != cudaSuccess || occ < 1) occ = 1;
+  cache[key] = occ;
+  return occ;
+}
+int decode_stages(int max_len) { return std::max(1, (max_len + kStageT - 1) / kStageT); }
+// CTAs of the split (never more than items).  n_split > 0 asks for about
+// n_split pieces per (b, h) unit.  Automatic (n_split = 0), `cap` = CTAs that
+// fit on the GPU at once: with fewer units than that, each unit is cut into
+// the same number k = cap / units of pieces, so that no CTA straddles two
+// units (a straddling CTA pays a second q absorption and its pieces a merge);
+// with more units, `cap` CTAs share all items evenly (stream-K).
+int64_t decode_ctas(int units, int max_len, int n_split, int64_t cap) {
+  const int64_t W = (int64_t)units * decode_stages(max_len);
+  if (n_split > 0) return std::min(W, (int64_t)units * n_split);
+  if (units >= cap) return std::min(W, cap);
+  return std::min(W, (int64_t)units * (cap / units));
+}
+}  // namespace
+
+size_t decode_workspace_bytes(int units, int rv_max, int max_len, int n_split) {
+  const size_t counters = (size_t)round_up(units * 4, 256);
   const size_t stride = (size_t)round_up(2 + rv_max, 4);
-  return counters + (size_t)batch * n_heads * n_split * stride * 4;
+  const int64_t G = decode_ctas(units, max_len, n_split, kAutoCtaBound);
+  return counters + (size_t)G * 2 * stride * 4;
 }
 
 cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
@@ -725,29 +951,49 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   p.BV = a.BV;
   p.seq_len = a.seq_len;
   p.out = a.out;
-  p.batch = a.batch;
   p.n_heads = a.n_heads;
   p.head_dim = a.head_dim;
   p.capacity = a.capacity;
-  p.group_k = a.group_k;
-  p.group_v = a.group_v;
   p.q_bf16 = a.q_bf16;
   p.b_bf16 = a.b_bf16;
   p.out_bf16 = a.out_bf16;
   p.max_len = a.max_len;
   p.qscale = a.softmax_scale * 1.4426950408889634f;
   int rk_max = 0, rv_max = 0, ngk_max = 1, ngv_max = 1;
+  int pk = 0, pv = 0, pgk = 0, pgv = 0, prk = 0, prv = 0;
   for (int h = 0; h < a.n_heads; ++h) {
-    p.rk[h] = (uint8_t)a.ranks_k[h];
-    p.rv[h] = (uint8_t)a.ranks_v[h];
-    rk_max = std::max(rk_max, a.ranks_k[h]);
-    rv_max = std::max(rv_max, a.ranks_v[h]);
-    if (a.kind == 1) {
-      const int gk = std::min(a.group_k, a.ranks_k[h]), gv = std::min(a.group_v, a.ranks_v[h]);
-      ngk_max = std::max(ngk_max, (a.ranks_k[h] + gk - 1) / gk);
-      ngv_max = std::max(ngv_max, (a.ranks_v[h] + gv - 1) / gv);
-    }
+    const int rk = a.ranks_k[h], rv = a.ranks_v[h];
+    const int gk = a.kind == 0 ? rk : std::min(a.group_k, rk);
+    const int gv = a.kind == 0 ? rv : std::min(a.group_v, rv);
+    const int ngk = (rk + gk - 1) / gk, ngv = (rv + gv - 1) / gv;
+    HeadInfo& hi = p.head[h];
+    hi.rk = (uint8_t)rk;
+    hi.rv = (uint8_t)rv;
+    hi.ngk = (uint8_t)ngk;
+    hi.ngv = (uint8_t)ngv;
+    hi.gk = (uint8_t)gk;
+    hi.gv = (uint8_t)gv;
+    hi.pk = (uint16_t)pk;
+    hi.pv = (uint16_t)pv;
+    hi.pgk = (uint16_t)pgk;
+    hi.pgv = (uint16_t)pgv;
+    hi.prk = (uint16_t)prk;
+    hi.prv = (uint16_t)prv;
+    pk += a.kind == 0 ? rk : rk / 2;
+    pv += a.kind == 0 ? rv : rv / 2;
+    pgk += ngk;
+    pgv += ngv;
+    prk += rk;
+    prv += rv;
+    rk_max = std::max(rk_max, rk);
+    rv_max = std::max(rv_max, rv);
+    ngk_max = std::max(ngk_max, ngk);
+    ngv_max = std::max(ngv_max, ngv);
   }
+  p.tk = pk;
+  p.tv = pv;
+  p.tgk = pgk;
+  p.tgv = pgv;
   const int rbk_max = a.kind == 0 ? rk_max : rk_max / 2;
   const int rbv_max = a.kind == 0 ? rv_max : rv_max / 2;
   const int ssz = a.kind == 0 ? 4 : 2;
@@ -760,52 +1006,47 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   p.st_q = round_up(a.head_dim * p.q_size, 128);
   p.st_bk = round_up(rk_max * a.head_dim * p.b_size, 128);
   p.st_bv = round_up(rv_max * a.head_dim * p.b_size, 128);
-  p.st_tw = kCW * round_up(ngv_max * kWTerms * 32, 16);
-  // as many stages as fit while two CTAs share an SM (about 64 KB of copies
-  // in flight per SM keeps HBM busy), between 2 and kMaxStages
+  p.st_fr = ngv_max > 1 ? kCW * ngv_max * 32 * 8 : 0;  // per-warp V fragments of each scale group
+  // as many stages as fit while two CTAs share an SM (about 64 KB of copies in
+  // flight per SM keeps HBM busy), between 2 and kMaxStages
   {
     p.nstages = 0;
     const int stage = p.st_kc + p.st_vc + p.st_ks + p.st_vs;
-    const int room = 110 * 1024 - (smem_bytes_for(p));  // smem_bytes_for counts 0 stages here
+    const int room = 110 * 1024 - smem_bytes_for(p);  // smem_bytes_for counts 0 stages here
     p.nstages = std::max(2, std::min(kMaxStages, room / std::max(stage, 1)));
   }
-  const int stages = std::max(1, (a.max_len + kStageT - 1) / kStageT);
-  int n_split = a.n_split;
-  if (n_split <= 0) n_split = decode_pick_split(a.batch * a.n_heads, a.max_len, a.num_sms);
-  n_split = std::max(1, std::min(std::min(n_split, stages), kMaxSplit));
-  p.stages_per_split = (stages + n_split - 1) / n_split;
-  n_split = (stages + p.stages_per_split - 1) / p.stages_per_split;
-  p.n_split = n_split;
+  const int units = a.batch * a.n_heads;
+  p.S = decode_stages(a.max_len);
+  const int64_t W = (int64_t)units * p.S;
+  const int smem = smem_bytes_for(p);
+  cudaError_t e = a.kind == 0
+                      ? cudaFuncSetAttribute(decode_attn_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+                      : cudaFuncSetAttribute(decode_attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int resident = decode_occupancy(a.kind, smem) * a.num_sms;
+  const int64_t G = decode_ctas(units, a.max_len, a.n_split, std::min(resident, kAutoCtaBound));
+  if (W > INT32_MAX || G < 1) return cudaErrorInvalidValue;
+  p.W = (int)W;
+  p.G = (int)G;
   p.part_stride = round_up(2 + rv_max, 4);
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
   p.counters = reinterpret_cast<int32_t*>(ws);
-  p.partials = reinterpret_cast<float*>(ws + round_up(a.batch * a.n_heads * 4, 256));
+  p.partials = reinterpret_cast<float*>(ws + round_up(units * 4, 256));
 
-  // up to eight splits of a head merge inside a cluster (portable cluster size)
-  p.cluster_merge = (n_split > 1 && n_split <= 8) ? 1 : 0;
-  const int smem = smem_bytes_for(p);
+  // programmatic stream serialisation: the launch and the barrier set-up
+  // overlap the tail of the previous kernel (the kernel waits for it before
+  // its first global read)
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_split, a.n_heads, a.batch);
+  cfg.gridDim = dim3((unsigned)G, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = p.cluster_merge ? n_split : 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e;
-  if (a.kind == 0) {
-    e = cudaFuncSetAttribute(decode_attn_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    e = cudaLaunchKernelEx(&cfg, decode_attn_kernel<0>, p);
-  } else {
-    e = cudaFuncSetAttribute(decode_attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    e = cudaLaunchKernelEx(&cfg, decode_attn_kernel<1>, p);
-  }
+  e = a.kind == 0 ? cudaLaunchKernelEx(&cfg, decode_attn_kernel<0>, p) : cudaLaunchKernelEx(&cfg, decode_attn_kernel<1>, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -830,6 +1071,7 @@ namespace {
 constexpr int kNoallocMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+int g_noalloc_units[kNoallocMaxDevices] = {};  // B * n_heads of the device's last call (0: none)
 }  // namespace
 
 extern "C" lk_status lk_latent_decode_attn_noalloc(const lk_latent_cache* k, const lk_latent_cache* v,
@@ -851,6 +1093,8 @@ extern "C" lk_status lk_latent_decode_attn_noalloc(const lk_latent_cache* k, con
     return lk::set_error(LK_ERR_CUDA, msg);
   }
   void* scratch = nullptr;
+  bool clear = false;
+  const int units = k->batch * k->n_heads;
   {
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
     if (!g_noalloc_ptr[dev]) {
@@ -865,16 +1109,14 @@ extern "C" lk_status lk_latent_decode_attn_noalloc(const lk_latent_cache* k, con
       g_noalloc_ptr[dev] = p;
     }
     scratch = g_noalloc_ptr[dev];
+    // the partials of a call with another B * n_heads may cover this call's
+    // counters: clear them first (every completed call leaves them zero)
+    clear = g_noalloc_units[dev] != units;
+    g_noalloc_units[dev] = units;
   }
   int rv_max = 0;
   for (int h = 0; h < v->n_heads; ++h) rv_max = std::max(rv_max, (int)v->ranks[h]);
-  int num_sms = 0;
-  if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || num_sms <= 0)
-    num_sms = 148;
-  const int stages = std::max(1, (max_seq_len + kStageT - 1) / kStageT);
-  int n_eff = n_split > 0 ? std::min(n_split, stages) : lk::decode_pick_split(k->batch * k->n_heads, max_seq_len, num_sms);
-  n_eff = std::max(1, std::min(std::min(n_eff, stages), kMaxSplit));
-  const size_t need = lk::decode_workspace_bytes(k->batch, k->n_heads, rv_max, n_eff);
+  const size_t need = lk::decode_workspace_bytes(k->batch * k->n_heads, rv_max, max_seq_len, n_split);
   if (need > LK_DECODE_NOALLOC_SCRATCH_BYTES) {
     snprintf(msg, sizeof(msg),
              "lk_latent_decode_attn_noalloc: needs %zu bytes of scratch, the static array holds %u; "
@@ -882,17 +1124,16 @@ extern "C" lk_status lk_latent_decode_attn_noalloc(const lk_latent_cache* k, con
              need, (unsigned)LK_DECODE_NOALLOC_SCRATCH_BYTES);
     return lk::set_error(LK_ERR_WORKSPACE, msg);
   }
+  if (clear) {
+    e = cudaMemsetAsync(scratch, 0, (size_t)(units * 4 + 255) / 256 * 256, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+      snprintf(msg, sizeof(msg), "lk_latent_decode_attn_noalloc: clearing counters: %s", cudaGetErrorString(e));
+      return lk::set_error(LK_ERR_CUDA, msg);
+    }
+  }
   const lk_status st = lk_latent_decode_attn(k, v, q, q_dtype, B_K, B_V, b_dtype, head_dim, seq_len, max_seq_len,
-                                             softmax_scale, out, out_dtype, n_eff, scratch,
+                                             softmax_scale, out, out_dtype, n_split, scratch,
                                              LK_DECODE_NOALLOC_SCRATCH_BYTES, stream);
   if (st != LK_OK) return st;
-  // leave the arrival counters zero for the next call (the kernel already does;
-  // this also covers a call cut short)
-  const size_t counters = (size_t)((k->batch * k->n_heads * 4 + 255) / 256 * 256);
-  e = cudaMemsetAsync(scratch, 0, counters, reinterpret_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) {
-    snprintf(msg, sizeof(msg), "lk_latent_decode_attn_noalloc: clearing counters: %s", cudaGetErrorString(e));
-    return lk::set_error(LK_ERR_CUDA, msg);
-  }
   return LK_OK;
 }

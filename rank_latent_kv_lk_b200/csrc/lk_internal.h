@@ -33,8 +33,10 @@ struct DecodeLaunch {
   int max_len, n_split, num_sms;
   float softmax_scale;
 };
-int decode_pick_split(int units, int max_len, int num_sms);
-size_t decode_workspace_bytes(int batch, int n_heads, int rv_max, int n_split);
+// Workspace of a decode call: arrival counters for the units plus two partial
+// slots per CTA; n_split > 0 asks for about n_split pieces per unit, 0 for a
+// grid that fills the GPU (at most 1024 CTAs).
+size_t decode_workspace_bytes(int units, int rv_max, int max_len, int n_split);
 cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream);
 
 // ---------------------------------------------------------------- projection

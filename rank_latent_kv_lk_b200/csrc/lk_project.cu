@@ -184,6 +184,7 @@ LK_DEVICE void append_values(const FinalizeParams& p, int grow, int j, float v0,
 
 // Prefill epilogue: one warp per (row, head); the last CTA advances seq_len.
 __global__ void __launch_bounds__(128) proj_finalize_kernel(const __grid_constant__ FinalizeParams p) {
+  lk_grid_dep_launch();  // a decode launched next may start its set-up now
   const int n_heads_tot = p.k.n_heads + p.v.n_heads;
   const int64_t item = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
   if (item < (int64_t)p.rows * n_heads_tot) {
@@ -219,10 +220,16 @@ struct ClusterProjParams {
   const void* A;
   int M, E, slice;
   int32_t* done_cnt;
+  int off_A, off_x, off_bar;  // staged variant: shared-memory offsets of the A and x slices and the barrier
 };
 
-template <int XT, int MT>
+// ST (staged, M <= 8): the CTA's whole slice of A (r rows x slice) and of x
+// is brought into shared memory by bulk copies issued at once, so all of the
+// CTA's bytes are in flight together; the dot products then read shared
+// memory.  Otherwise each warp streams its A rows from global memory.
+template <int XT, int MT, bool ST>
 __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid_constant__ ClusterProjParams p) {
+  lk_grid_dep_launch();  // a decode launched next may start its set-up now
   using T = typename XTraits<XT>::T;
   constexpr int VE = XTraits<XT>::VE;
   constexpr bool INT = XT == lk::X_I8;
@@ -241,6 +248,71 @@ __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid
   const T* x = static_cast<const T*>(p.x);  // read through L1: every warp of the CTA uses the same slice
   const T* A = static_cast<const T*>(p.A);
 
+  if constexpr (ST) {
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + p.off_bar);
+    const T* As = reinterpret_cast<const T*>(smem_raw + p.off_A);
+    const T* xs = reinterpret_cast<const T*>(smem_raw + p.off_x);
+    if (threadIdx.x == 0) {
+      lk_mbar_init(bar, 1);
+      lk_fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && elen > 0) {
+      const uint32_t rowb = (uint32_t)(elen * sizeof(T));
+      lk_mbar_arrive_expect_tx(bar, (uint32_t)(r + M) * rowb);
+      for (int n = 0; n < r; ++n)
+        lk_bulk_g2s(smem_raw + p.off_A + (size_t)n * p.slice * sizeof(T), A + (int64_t)(col0 + n) * p.E + e0, rowb, bar);
+      for (int m = 0; m < M; ++m)
+        lk_bulk_g2s(smem_raw + p.off_x + (size_t)m * p.slice * sizeof(T), x + (int64_t)m * p.E + e0, rowb, bar);
+    }
+    const bool ok = elen == 0 || lk_mbar_wait_bounded(bar, 0, LK_WAIT_LIMIT_NS);
+    if (!ok && threadIdx.x == 0) lk_dev_fail(LK_DEV_TIMEOUT_PIPE);
+    for (int n = warp; n < r; n += kGemvThreads / 32) {
+      float facc[MT];
+      int iacc[MT];
+#pragma unroll
+      for (int i = 0; i < MT; ++i) { facc[i] = 0.0f; iacc[i] = 0; }
+      for (int cc = lane; ok && cc < chunks; cc += 32) {
+        const uint4 wv = *reinterpret_cast<const uint4*>(As + (size_t)n * p.slice + cc * VE);
+        float wf[VE];
+        if (!INT) expand16<XT>(wv, wf);
+#pragma unroll
+        for (int i = 0; i < MT; ++i) {
+          if (i < M) {
+            const uint4 xv4 = *reinterpret_cast<const uint4*>(xs + (size_t)i * p.slice + cc * VE);
+            if (INT) {
+              int a = iacc[i];
+              a = __dp4a((int)xv4.x, (int)wv.x, a);
+              a = __dp4a((int)xv4.y, (int)wv.y, a);
+              a = __dp4a((int)xv4.z, (int)wv.z, a);
+              a = __dp4a((int)xv4.w, (int)wv.w, a);
+              iacc[i] = a;
+            } else {
+              float xf[VE];
+              expand16<XT>(xv4, xf);
+              float a = facc[i];
+#pragma unroll
+              for (int k = 0; k < VE; ++k) a = fmaf(xf[k], wf[k], a);
+              facc[i] = a;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < MT; ++i) {
+        uint32_t val;
+        if (INT) {
+          int a = iacc[i];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+          val = (uint32_t)a;
+        } else {
+          val = __float_as_uint(lk_warp_sum(facc[i]));
+        }
+        if (lane == 0 && i < M) part[n * M + i] = val;
+      }
+    }
+  } else
   for (int cb = warp * kProjNC; cb < r; cb += (kGemvThreads / 32) * kProjNC) {
     for (int m0 = 0; m0 < M; m0 += MT) {
       const int mt = min(MT, M - m0);
@@ -437,7 +509,16 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
     d.E = a.embed_dim;
     d.slice = cluster_slice(a.embed_dim, a.xtype);
     d.done_cnt = static_cast<int32_t*>(a.workspace);
-    const size_t smem = (size_t)LK_MAX_RANK * rows * 4;
+    size_t smem = (size_t)LK_MAX_RANK * rows * 4;
+    // staged variant: A rows of the widest head and the x rows, one slice each
+    int r_max = 0;
+    for (int j = 0; j < heads_tot; ++j) r_max = std::max(r_max, (int)f.rank[j]);
+    const size_t slice_b = (size_t)d.slice * x_size(a.xtype);
+    d.off_A = round_up((int)smem, 128);
+    d.off_x = d.off_A + round_up((int)(r_max * slice_b), 128);
+    d.off_bar = d.off_x + round_up((int)(rows * slice_b), 16);
+    const bool staged = rows <= 8 && (size_t)d.off_bar + 8 <= 200 * 1024;
+    if (staged) smem = (size_t)d.off_bar + 8;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kClusterE, heads_tot, 1);
     cfg.blockDim = dim3(kGemvThreads, 1, 1);
@@ -451,12 +532,17 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const int mt = rows <= 1 ? 1 : (rows <= 2 ? 2 : (rows <= 4 ? 4 : 8));
-#define LK_PROJ_LAUNCH(XTV, MTV)                                                                         \
+#define LK_PROJ_LAUNCH2(XTV, MTV, STV)                                                                   \
   do {                                                                                                \
-    e = cudaFuncSetAttribute(proj_cluster_kernel<XTV, MTV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+    e = cudaFuncSetAttribute(proj_cluster_kernel<XTV, MTV, STV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              (int)smem);                                                             \
     if (e != cudaSuccess) return e;                                                                   \
-    e = cudaLaunchKernelEx(&cfg, proj_cluster_kernel<XTV, MTV>, d);                                  \
+    e = cudaLaunchKernelEx(&cfg, proj_cluster_kernel<XTV, MTV, STV>, d);                             \
+  } while (0)
+#define LK_PROJ_LAUNCH(XTV, MTV)                         \
+  do {                                                   \
+    if (staged) LK_PROJ_LAUNCH2(XTV, MTV, true);         \
+    else LK_PROJ_LAUNCH2(XTV, MTV, false);               \
   } while (0)
 #define LK_PROJ_MT(XTV)                          \
   do {                                           \
@@ -470,6 +556,7 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
     else LK_PROJ_MT(X_I8);
 #undef LK_PROJ_MT
 #undef LK_PROJ_LAUNCH
+#undef LK_PROJ_LAUNCH2
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }

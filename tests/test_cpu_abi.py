@@ -90,11 +90,14 @@ def test_decode_validation(L):
 
 def test_decode_workspace_size_formula(L):
     k, v = cache(L), cache(L)
-    # counters (1 * 2 heads * 4 B, rounded to 256) + partials (1 * 2 * stages * (2 + 16) floats)
+    # counters (1 * 2 heads * 4 B, rounded to 256) + two partial slots per CTA of
+    # (2 + 16) floats rounded to 20; items = units * ceil(max_len / 224)
     n = L.lib.lk_latent_decode_workspace_bytes(C.byref(k), C.byref(v), 64, 0)
-    assert n == 256 + 1 * 2 * 1 * 20 * 4
+    assert n == 256 + 2 * 2 * 20 * 4            # 2 items -> at most 2 CTAs
     n = L.lib.lk_latent_decode_workspace_bytes(C.byref(k), C.byref(v), 1000, 3)
-    assert n == 256 + 1 * 2 * 3 * 20 * 4
+    assert n == 256 + 6 * 2 * 20 * 4            # 10 items, about 3 pieces per unit -> 6 CTAs
+    n = L.lib.lk_latent_decode_workspace_bytes(C.byref(k), C.byref(v), 64 * 1024, 0)
+    assert n == 256 + 586 * 2 * 20 * 4          # 586 items, automatic grid (at most 1024 CTAs)
 
 
 def project(L, k, v, x=FAKE + 0x800000, xdt=None, E=512, n_new=1, host_len=(0,), ws_bytes=1 << 24,
