@@ -244,30 +244,57 @@ __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid
   const int e0 = rank * p.slice;
   const int elen = max(0, min(p.slice, p.E - e0));
   const int chunks = elen / VE;
-  uint32_t* part = reinterpret_cast<uint32_t*>(smem_raw);  // [kMaxR][M]
+  // every CTA's partials go straight into rank 0's shared memory:
+  // part[q][n][m] for slice q, latent column n, row m
+  uint32_t* part = reinterpret_cast<uint32_t*>(smem_raw);
+  uint32_t* mine = cluster.map_shared_rank(part, 0) + (size_t)rank * LK_MAX_RANK * M;
+  // a peer's shared memory may be written only once that CTA runs: arrive now,
+  // wait just before the first remote write
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  bool joined = false;
+  auto join = [&]() {
+    if (!joined) {
+      asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+      joined = true;
+    }
+  };
   const T* x = static_cast<const T*>(p.x);  // read through L1: every warp of the CTA uses the same slice
   const T* A = static_cast<const T*>(p.A);
 
   if constexpr (ST) {
+    // rows in groups of 8 (x with group 0), one barrier each, so the first
+    // rows are worked on while the later ones are still arriving
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + p.off_bar);
     const T* As = reinterpret_cast<const T*>(smem_raw + p.off_A);
     const T* xs = reinterpret_cast<const T*>(smem_raw + p.off_x);
+    const int ngroups = (r + 7) / 8;
     if (threadIdx.x == 0) {
-      lk_mbar_init(bar, 1);
+      for (int gi = 0; gi < ngroups; ++gi) lk_mbar_init(&bar[gi], 1);
       lk_fence_mbar_init();
     }
     __syncthreads();
     if (threadIdx.x == 0 && elen > 0) {
       const uint32_t rowb = (uint32_t)(elen * sizeof(T));
-      lk_mbar_arrive_expect_tx(bar, (uint32_t)(r + M) * rowb);
-      for (int n = 0; n < r; ++n)
-        lk_bulk_g2s(smem_raw + p.off_A + (size_t)n * p.slice * sizeof(T), A + (int64_t)(col0 + n) * p.E + e0, rowb, bar);
-      for (int m = 0; m < M; ++m)
-        lk_bulk_g2s(smem_raw + p.off_x + (size_t)m * p.slice * sizeof(T), x + (int64_t)m * p.E + e0, rowb, bar);
+      for (int gi = 0; gi < ngroups; ++gi) {
+        const int n0 = 8 * gi, n1 = min(r, n0 + 8);
+        lk_mbar_arrive_expect_tx(&bar[gi], (uint32_t)(n1 - n0 + (gi == 0 ? M : 0)) * rowb);
+        if (gi == 0)
+          for (int m = 0; m < M; ++m)
+            lk_bulk_g2s(smem_raw + p.off_x + (size_t)m * p.slice * sizeof(T), x + (int64_t)m * p.E + e0, rowb, &bar[0]);
+        for (int n = n0; n < n1; ++n)
+          lk_bulk_g2s(smem_raw + p.off_A + (size_t)n * p.slice * sizeof(T), A + (int64_t)(col0 + n) * p.E + e0, rowb,
+                      &bar[gi]);
+      }
     }
-    const bool ok = elen == 0 || lk_mbar_wait_bounded(bar, 0, LK_WAIT_LIMIT_NS);
-    if (!ok && threadIdx.x == 0) lk_dev_fail(LK_DEV_TIMEOUT_PIPE);
+    bool ok = true;
+    int waited = 0;  // groups this thread has seen land
     for (int n = warp; n < r; n += kGemvThreads / 32) {
+      for (; ok && elen > 0 && waited <= n / 8; ++waited) {
+        if (!lk_mbar_wait_bounded(&bar[waited], 0, LK_WAIT_LIMIT_NS)) {
+          ok = false;
+          if (lane == 0) lk_dev_fail(LK_DEV_TIMEOUT_PIPE);
+        }
+      }
       float facc[MT];
       int iacc[MT];
 #pragma unroll
@@ -309,9 +336,16 @@ __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid
         } else {
           val = __float_as_uint(lk_warp_sum(facc[i]));
         }
-        if (lane == 0 && i < M) part[n * M + i] = val;
+        if (i < M) {
+          join();
+          if (lane == 0) mine[n * M + i] = val;
+        }
       }
     }
+    // copies of groups no warp waited for (r not a multiple of the warps' stride)
+    // have landed before the CTA may finish
+    for (int gi = waited; ok && elen > 0 && gi < ngroups; ++gi)
+      if (!lk_mbar_wait_bounded(&bar[gi], 0, LK_WAIT_LIMIT_NS)) ok = false;
   } else
   for (int cb = warp * kProjNC; cb < r; cb += (kGemvThreads / 32) * kProjNC) {
     for (int m0 = 0; m0 < M; m0 += MT) {
@@ -382,14 +416,16 @@ __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid
           } else {
             val = __float_as_uint(lk_warp_sum(facc[jj][i]));
           }
-          if (lane == 0 && i < mt && cb + jj < r) part[(cb + jj) * M + m0 + i] = val;
+          join();
+          if (lane == 0 && i < mt && cb + jj < r) mine[(cb + jj) * M + m0 + i] = val;
         }
       }
     }
   }
-  cluster.sync();  // every CTA's partials are visible to the cluster
-
-  if (rank == 0) {
+  join();  // (warps without columns)
+  cluster.sync();  // every CTA's partials are in rank 0's shared memory
+  if (rank != 0) return;
+  {
     for (int m = warp; m < M; m += kGemvThreads / 32) {
       float vals[2];
 #pragma unroll
@@ -401,11 +437,11 @@ __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid
           if (INT) {
             int acc = 0;
 #pragma unroll
-            for (int q = 0; q < kClusterE; ++q) acc += (int)cluster.map_shared_rank(part, q)[d * M + m];
+            for (int q = 0; q < kClusterE; ++q) acc += (int)part[((size_t)q * LK_MAX_RANK + d) * M + m];
             val = __fmul_rn(__fmul_rn((float)acc, f.x_scale[m]), lk_f16_to_f32(f.a_scale[n]));
           } else {
 #pragma unroll
-            for (int q = 0; q < kClusterE; ++q) val += __uint_as_float(cluster.map_shared_rank(part, q)[d * M + m]);
+            for (int q = 0; q < kClusterE; ++q) val += __uint_as_float(part[((size_t)q * LK_MAX_RANK + d) * M + m]);
           }
         }
         vals[q2] = val;
@@ -413,9 +449,8 @@ __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid
       append_values(f, m, j, vals[0], vals[1]);
     }
   }
-  cluster.sync();  // the other CTAs keep their partials until rank 0 has read them
-
-  if (rank == 0 && threadIdx.x == 0) {
+  __syncthreads();  // every append of this head is written
+  if (threadIdx.x == 0) {
     __threadfence();
     const int n_heads_tot = f.k.n_heads + f.v.n_heads;
     if (atomicAdd(p.done_cnt, 1) == n_heads_tot - 1) {  // every head appended: advance the rows
@@ -509,7 +544,7 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
     d.E = a.embed_dim;
     d.slice = cluster_slice(a.embed_dim, a.xtype);
     d.done_cnt = static_cast<int32_t*>(a.workspace);
-    size_t smem = (size_t)LK_MAX_RANK * rows * 4;
+    size_t smem = (size_t)kClusterE * LK_MAX_RANK * rows * 4;
     // staged variant: A rows of the widest head and the x rows, one slice each
     int r_max = 0;
     for (int j = 0; j < heads_tot; ++j) r_max = std::max(r_max, (int)f.rank[j]);
@@ -517,8 +552,8 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
     d.off_A = round_up((int)smem, 128);
     d.off_x = d.off_A + round_up((int)(r_max * slice_b), 128);
     d.off_bar = d.off_x + round_up((int)(rows * slice_b), 16);
-    const bool staged = rows <= 8 && (size_t)d.off_bar + 8 <= 200 * 1024;
-    if (staged) smem = (size_t)d.off_bar + 8;
+    const bool staged = rows <= 8 && (size_t)d.off_bar + 8 * 8 <= 200 * 1024;
+    if (staged) smem = (size_t)d.off_bar + 8 * 8;  // up to 8 row groups (r <= 64)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kClusterE, heads_tot, 1);
     cfg.blockDim = dim3(kGemvThreads, 1, 1);
