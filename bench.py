@@ -48,6 +48,9 @@ def parse_args(argv=None):
     ap.add_argument("--workload", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--attn-only", action="store_true",
+                    help="time the latent decode attention alone on one layer of the workload, "
+                         "its cache filled with seeded random codes (no prefill)")
     return ap.parse_args(argv)
 
 
@@ -461,6 +464,82 @@ def run_ours(args):
     return 0
 
 
+def run_attn_only(args):
+    """Latent decode attention alone on one layer of a workload (throughput of
+    the cache stream at the large shapes).  The cache holds seeded random codes
+    and positive scales; q and the factors follow the workload's recipe."""
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    import rank_latent_kv_lk_b200 as lk
+    from rank_latent_kv_lk_b200 import synth
+    from rank_latent_kv_lk_b200.configs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    rk, rv = synth.ranks(w)
+    rk, rv = rk[0], rv[0]
+    _, BK, BV = synth.factors(w, 0, rk, rv)
+    BK, BV = BK.to(device), BV.to(device)
+    T = w.context + 1
+    g = torch.Generator(device=device)
+    g.manual_seed(synth.seed_for(w, synth.CONTEXT))
+    caches = []
+    for ranks in (rk, rv):
+        c = lk.LatentCache(w.batch, ranks, w.capacity, w.kind, w.group, device, role="k" if not caches else "v")
+        c.codes.copy_(torch.randint(0, 256, c.codes.shape, dtype=torch.uint8, device=device, generator=g))
+        sc = torch.rand(c.scales.shape, device=device, generator=g) * 0.02 + 0.01
+        c.scales.copy_(sc.to(c.scales.dtype))
+        caches.append(c)
+    ck, cv = caches
+    q = synth.queries(w, 0)[0].to(device)
+    seq = torch.full((w.batch,), T, dtype=torch.int32, device=device)
+    out = torch.empty(w.batch, w.n_heads, w.head_dim, dtype=torch.bfloat16, device=device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    for _ in range(max(3, args.warmup)):
+        lk.latent_decode_attn(ck, cv, q, BK, BV, seq, T, out=out)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(1e8))
+    with ClockSampler(local) as clocks:
+        for i in range(K):
+            flush.fill_(1)
+            ev[i][0].record(stream)
+            lk.latent_decode_attn(ck, cv, q, BK, BV, seq, T, out=out)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    lk.device_status()
+    ms = [e[0].elapsed_time(e[1]) for e in ev]
+    total_ms = max_over_ranks(sum(ms), world, device)
+    rb = lambda r: r if w.kind == "i8" else r // 2
+    sb = lambda r: 4 if w.kind == "i8" else 2 * (-(-r // min(w.group, r)))
+    per_tok = sum(rb(r) + sb(r) for r in rk) + sum(rb(r) + sb(r) for r in rv)
+    nbytes = w.batch * T * per_tok + (sum(rk) + sum(rv)) * w.head_dim * 2 + 2 * w.batch * w.n_heads * w.head_dim * 2
+    us = total_ms / K * 1e3
+    gbs = nbytes / (us * 1e-6) / 1e9
+    hbm, peak_kind = peaks()
+    if rank == 0:
+        print(json.dumps({
+            "mode": "attn-only", "metric": "latent-attn HBM GB/s", "value": gbs * world, "unit": "GB/s",
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "us_per_launch": us, "higher_is_better": True,
+            "scaling": "weak", "dtype": "int8/f32" if w.kind == "i8" else "int4/f32",
+            "data": "synthetic (seeded random latent codes and scales; shapes of the workload)",
+            "config": {"workload": w.name, "layer": 0, "batch": w.batch, "tokens": T,
+                       "l2": "flushed before every launch (256 MiB write, untimed)"},
+            "algorithmic_bytes_per_launch": nbytes,
+            "roofline": {"kernel": "latent_decode_attn", "bound": "hbm", "achieved": gbs, "peak": hbm,
+                         "unit": "GB/s", "frac": gbs / hbm, "peak_kind": peak_kind,
+                         "frac_of_8tbs": gbs / 8000.0,
+                         "traffic": profiled_traffic("decode_attn_kernel", f"{w.key}-attn")},
+            "gpu_launches": K, "clocks": clocks.summary()}), flush=True)
+    _finish(world)
+    return 0
+
+
 def _finish(world):
     if world > 1 and torch.distributed.is_initialized():
         torch.distributed.destroy_process_group()
@@ -472,6 +551,8 @@ def main(argv=None):
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.attn_only:
+        return run_attn_only(args)
     return run_ours(args)
 
 
