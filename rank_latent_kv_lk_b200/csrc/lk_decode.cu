@@ -316,6 +316,8 @@ LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom
     float s = 0.0f;
     int d0 = 0, d1 = 0, d2 = 0;
     int cur_g = 0;
+    const int wpg = g.gk >> 3;  // code words per scale group
+    int wleft = wpg;            // words left in the current group
     // code word w holds dims 8w .. 8w+7 (q~ bytes 8w .. 8w+7: even dims, then
     // odd dims); groups are multiples of 8 dims
 #pragma unroll
@@ -329,14 +331,14 @@ LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom
         lds_words<2 * WPC>(qterm + 2 * kMaxR + c * 2 * CS, t2);
 #pragma unroll
         for (int wi = 0; wi < WPC; ++wi) {
-          const int w = c * WPC + wi;
-          const int gw = (8 * w) / g.gk;
-          if (gw != cur_g) {  // flush the finished group (uniform branch)
+          if (wleft == 0) {  // flush the finished group (uniform branch)
             const float x = fmaf((float)d2, kInv254sq, fmaf((float)d1, kInv254, (float)d0));
             s = fmaf(load_scale(ks, tl * g.ngk + cur_g, 1), qa * x, s);
             d0 = d1 = d2 = 0;
-            cur_g = gw;
+            ++cur_g;
+            wleft = wpg;
           }
+          --wleft;
           int ev, od;
           nibbles_to_s8(ch.w[wi], ev, od);
           d0 = __dp4a(od, (int)t0[2 * wi + 1], __dp4a(ev, (int)t0[2 * wi], d0));
@@ -936,7 +938,9 @@ int64_t decode_ctas(int units, int max_len, int n_split, int64_t cap) {
 size_t decode_workspace_bytes(int units, int rv_max, int max_len, int n_split) {
   const size_t counters = (size_t)round_up(units * 4, 256);
   const size_t stride = (size_t)round_up(2 + rv_max, 4);
-  const int64_t G = decode_ctas(units, max_len, n_split, kAutoCtaBound);
+  // the automatic grid never exceeds min(items, kAutoCtaBound)
+  const int64_t G = n_split > 0 ? decode_ctas(units, max_len, n_split, kAutoCtaBound)
+                                 : std::min((int64_t)units * decode_stages(max_len), (int64_t)kAutoCtaBound);
   return counters + (size_t)G * 2 * stride * 4;
 }
 
@@ -961,6 +965,7 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   p.qscale = a.softmax_scale * 1.4426950408889634f;
   int rk_max = 0, rv_max = 0, ngk_max = 1, ngv_max = 1;
   int pk = 0, pv = 0, pgk = 0, pgv = 0, prk = 0, prv = 0;
+
   for (int h = 0; h < a.n_heads; ++h) {
     const int rk = a.ranks_k[h], rv = a.ranks_v[h];
     const int gk = a.kind == 0 ? rk : std::min(a.group_k, rk);
@@ -979,6 +984,7 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
     hi.pgv = (uint16_t)pgv;
     hi.prk = (uint16_t)prk;
     hi.prv = (uint16_t)prv;
+
     pk += a.kind == 0 ? rk : rk / 2;
     pv += a.kind == 0 ? rv : rv / 2;
     pgk += ngk;
@@ -1018,6 +1024,7 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   const int units = a.batch * a.n_heads;
   p.S = decode_stages(a.max_len);
   const int64_t W = (int64_t)units * p.S;
+
   const int smem = smem_bytes_for(p);
   cudaError_t e = a.kind == 0
                       ? cudaFuncSetAttribute(decode_attn_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
