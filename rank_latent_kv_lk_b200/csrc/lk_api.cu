@@ -9,6 +9,7 @@
 cudaError_t lk_quant_status_word(unsigned int* value, int reset);
 cudaError_t lk_project_status_word(unsigned int* value, int reset);
 cudaError_t lk_lowrank_status_word(unsigned int* value, int reset);
+cudaError_t lk_gemm_tc_status_word(unsigned int* value, int reset);
 
 namespace {
 
@@ -368,8 +369,9 @@ lk_status lk_device_status(int32_t reset) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "lk_device_status");
   unsigned int words[4] = {0, 0, 0, 0};
-  cudaError_t (*fns[4])(unsigned int*, int) = {lk_decode_status_word, lk_quant_status_word,
-                                                lk_project_status_word, lk_lowrank_status_word};
+  cudaError_t (*fns[5])(unsigned int*, int) = {lk_decode_status_word, lk_quant_status_word,
+                                                lk_project_status_word, lk_lowrank_status_word,
+                                                lk_gemm_tc_status_word};
   unsigned int any = 0;
   for (int i = 0; i < 4; ++i) {
     e = fns[i](&words[i], reset);

@@ -103,6 +103,12 @@ cudaError_t launch_rowquant(int mode, const void* x, const void* x2, int x_bf16,
 
 // ---------------------------------------------------------------- generic int8 GEMM
 // C[m][n] = sum_k A[m][k] * B[n][k]  (int32), A, B row-major with given row strides (bytes)
+// tcgen05 bf16 GEMM with TMEM accumulators (lk_gemm_tc.cu): same contract as
+// launch_gemm_f with bf16 operands; needs lda, ldb multiples of 8 and
+// 16-byte aligned operands.
+bool gemm_bf16_tc_supported(const void* A, int lda, const void* B, int ldb, int K);
+cudaError_t launch_gemm_bf16_tc(const void* A, int lda, const void* B, int ldb, float* C, int ldc, int M, int N,
+                                int K, cudaStream_t stream);
 cudaError_t launch_gemm_i8(const int8_t* A, int lda, const int8_t* B, int ldb, int32_t* C, int ldc,
                            int M, int N, int K, cudaStream_t stream);
 

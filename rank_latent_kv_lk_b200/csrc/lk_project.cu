@@ -606,9 +606,14 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
       e = launch_gemm_i8(reinterpret_cast<const int8_t*>(xr), a.embed_dim,
                          static_cast<const int8_t*>(a.A), a.embed_dim,
                          reinterpret_cast<int32_t*>(f.ws), a.n_tot, nr, a.n_tot, a.embed_dim, stream);
+    } else if (a.xtype == X_BF16) {
+      // a dense bf16 contraction: tcgen05 with TMEM accumulators
+      if (!gemm_bf16_tc_supported(xr, a.embed_dim, a.A, a.embed_dim, a.embed_dim)) return cudaErrorInvalidValue;
+      e = launch_gemm_bf16_tc(xr, a.embed_dim, a.A, a.embed_dim, reinterpret_cast<float*>(f.ws), a.n_tot, nr,
+                              a.n_tot, a.embed_dim, stream);
     } else {
       e = launch_gemm_f(xr, a.embed_dim, a.A, a.embed_dim, reinterpret_cast<float*>(f.ws), a.n_tot, nr,
-                        a.n_tot, a.embed_dim, a.xtype == X_BF16, stream);
+                        a.n_tot, a.embed_dim, false, stream);
     }
     if (e != cudaSuccess) return e;
     f.n_ksplit = 1;
