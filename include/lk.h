@@ -225,6 +225,29 @@ lk_status lk_latent_decode_attn_noalloc(const lk_latent_cache* k_cache, const lk
                                         int32_t n_split, lk_stream_t stream);
 
 /*
+ * One decode step of the latent-KV attention: lk_latent_project_append of
+ * one new token per batch row (x: [B, embed_dim]), then
+ * lk_latent_decode_attn over positions [0, seq_len_host[b] + 1) (the new
+ * token included; max_seq_len = max_b seq_len_host[b] + 1).  The arguments
+ * mean what they mean for those two calls.
+ * The attention kernel is launched so that it may start while the append
+ * still runs: it fetches q, B_K and B_V (and absorbs q) before it waits for
+ * the append, and reads the cache and seq_len only after.  q, B_K and B_V
+ * must therefore be complete before this call's first kernel starts (they
+ * are never written by the append).  All arguments are validated before
+ * anything is launched.
+ */
+lk_status lk_latent_decode_step(const lk_latent_cache* k_cache, const lk_latent_cache* v_cache,
+                                const void* x, lk_dtype x_dtype, const float* x_scale,
+                                const void* A, lk_dtype a_dtype, const uint16_t* a_scale,
+                                int32_t embed_dim, int32_t* seq_len, const int32_t* seq_len_host,
+                                const void* q, lk_dtype q_dtype, const void* B_K, const void* B_V,
+                                lk_dtype b_dtype, int32_t head_dim, float softmax_scale, void* out,
+                                lk_dtype out_dtype, int32_t n_split, void* project_workspace,
+                                size_t project_workspace_bytes, void* decode_workspace,
+                                size_t decode_workspace_bytes, lk_stream_t stream);
+
+/*
  * LASER hybrid dense + low-rank linear, W8A8 (LASER technical summary §3:
  * selected input channels go through SVD factors, the rest stay dense; both
  * branches RTN-quantised).

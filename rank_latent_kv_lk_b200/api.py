@@ -134,6 +134,33 @@ def latent_decode_attn(k_cache, v_cache, q, B_K, B_V, seq_len, max_seq_len, soft
     return out
 
 
+def latent_decode_step(k_cache, v_cache, x, A, seq_len, seq_len_host, q, B_K, B_V, x_scale=None, a_scale=None,
+                       softmax_scale=None, out=None, out_dtype=None, n_split=0, stream=None):
+    """One decode step: append one token per row (x: [B, E]), then attend over
+    the caches including it.  The attention launch overlaps the append (its
+    q absorption runs while the append finishes).  seq_len (device) advances
+    by one; seq_len_host is the host copy before the step."""
+    H = q.shape[-1]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(H)
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    E = x.shape[-1]
+    xdt = _dtype_code(x)
+    host = (C.c_int32 * k_cache.batch)(*[int(v) for v in seq_len_host])
+    pneed = lib.lk_latent_project_workspace_bytes(k_cache.desc(), v_cache.desc(), E, 1, xdt)
+    pws = workspaces.get("project", pneed, x.device)
+    max_len = max(int(v) for v in seq_len_host) + 1
+    dneed = lib.lk_latent_decode_workspace_bytes(k_cache.desc(), v_cache.desc(), max_len, int(n_split))
+    dws = workspaces.get(("decode", k_cache.batch * len(k_cache.ranks)), dneed, q.device)
+    check(lib.lk_latent_decode_step(
+        k_cache.desc(), v_cache.desc(), _ptr(x), xdt, _ptr(x_scale), _ptr(A), _dtype_code(A), _ptr(a_scale), E,
+        _ptr(seq_len), host, _ptr(q), _dtype_code(q), _ptr(B_K), _ptr(B_V), _dtype_code(B_K), H,
+        float(softmax_scale), _ptr(out), _dtype_code(out), int(n_split), _ptr(pws), pws.numel(), _ptr(dws),
+        dws.numel(), _stream(stream)))
+    return out
+
+
 class LowrankWeight:
     """Device weights of one LASER hybrid linear (int8, fp16 scales)."""
 

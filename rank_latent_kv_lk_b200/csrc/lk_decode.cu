@@ -80,6 +80,7 @@ struct DecodeParams {
   int n_heads, head_dim, capacity;
   int tk, tv, tgk, tgv;  // code bytes / scale groups of one batch row (all heads)
   int q_bf16, b_bf16, out_bf16;
+  int early_inputs;  // q, B_K, B_V are read before waiting for the previous kernel on the stream
   int max_len;
   int S;   // stages per unit: ceil(max_len / kStageT)
   int W;   // items: units * S
@@ -436,7 +437,6 @@ LK_DEVICE void produce(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
     const int s_end = min(p.S, s + (i1 - it));
     const int b = u / p.n_heads, h = u - b * p.n_heads;
     const HeadGeom g = unit_geometry<KIND>(p, b, h);
-    const int len = unit_len(p, b);
     if (ok && nunit > 0 && !lk_mbar_wait_bounded(B.fempty, (uint32_t)((nunit - 1) & 1), LK_WAIT_LIMIT_NS)) {
       *B.abort_flag = 1;
       ok = false;
@@ -449,7 +449,9 @@ LK_DEVICE void produce(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
       lk_bulk_g2s(smem + L.off_bk, static_cast<const uint8_t*>(p.BK) + g.bk_off * p.b_size, bkb, B.fbar);
       ++nf;
     }
+    if (nunit == 0 && p.early_inputs) lk_grid_dep_wait();  // the cache and seq_len are the previous kernel's
     ++nunit;
+    const int len = unit_len(p, b);
     const int64_t end = min((int64_t)((len + 15) & ~15), (int64_t)p.capacity);
     for (int ss = s; ss < s_end && ok; ++ss) {
       const int64_t t0 = (int64_t)ss * kStageT;
@@ -840,8 +842,9 @@ LK_DEVICE void consume(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
     const int seg_end = it + (s_end - s);
     const int b = u / p.n_heads, h = u - b * p.n_heads;
     const HeadGeom g = unit_geometry<KIND>(p, b, h);
-    const int len = unit_len(p, b);
     absorb_q<KIND>(p, smem, L, g, n);
+    if (n == 0 && p.early_inputs) lk_grid_dep_wait();  // the cache and seq_len are the previous kernel's
+    const int len = unit_len(p, b);
     const int csk = lk_chunk_bytes(g.rbk);
     if (KIND == 0 || g.ngv == 1) {
       if (csk == 16) run_unit_nm<KIND, 16, true>(p, smem, L, g, len, s, s_end, buf, phase);
@@ -880,9 +883,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const __grid_c
   }
   __syncthreads();
   // launched with programmatic stream serialisation, this CTA may run while
-  // the previous kernel on the stream (e.g. the latent append) finishes:
-  // nothing before this point reads global memory
-  lk_grid_dep_wait();
+  // the previous kernel on the stream (e.g. the latent append) finishes.
+  // Nothing before this point reads global memory; with early_inputs the
+  // first unit's q, B_K and B_V are fetched before the wait (in produce and
+  // absorb_q), everything else after it.
+  if (!p.early_inputs) lk_grid_dep_wait();
   if (i0 >= i1) return;
   if (threadIdx.x >= kConsumerThreads) {
     if (threadIdx.x == kConsumerThreads) produce<KIND>(p, smem, L, i0, i1);
@@ -961,6 +966,7 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   p.q_bf16 = a.q_bf16;
   p.b_bf16 = a.b_bf16;
   p.out_bf16 = a.out_bf16;
+  p.early_inputs = a.early_inputs;
   p.max_len = a.max_len;
   p.qscale = a.softmax_scale * 1.4426950408889634f;
   int rk_max = 0, rv_max = 0, ngk_max = 1, ngv_max = 1;

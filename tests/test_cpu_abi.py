@@ -100,6 +100,18 @@ def test_decode_workspace_size_formula(L):
     assert n == 256 + 586 * 2 * 20 * 4          # 586 items, automatic grid (at most 1024 CTAs)
 
 
+def test_step_validates_attention_before_launching(L):
+    k, v = cache(L), cache(L)
+    hl = (C.c_int32 * 1)(0)
+    st = L.lib.lk_latent_decode_step(C.byref(k), C.byref(v), C.c_void_p(FAKE + 0x800000), L.LK_BF16, None,
+                                     C.c_void_p(FAKE + 0xA00000), L.LK_BF16, None, 512, C.c_void_p(FAKE + 0xB00000),
+                                     hl, C.c_void_p(FAKE + 0x300000), L.LK_BF16, C.c_void_p(FAKE + 0x400000),
+                                     C.c_void_p(FAKE + 0x500000), L.LK_BF16, 60, 0.125, C.c_void_p(FAKE + 0x700000),
+                                     L.LK_F32, 0, C.c_void_p(FAKE + 0x900000), 1 << 24, C.c_void_p(FAKE + 0x200000),
+                                     1 << 20, None)
+    assert st == L.LK_ERR_SHAPE  # head_dim 60: rejected before the append is launched
+
+
 def project(L, k, v, x=FAKE + 0x800000, xdt=None, E=512, n_new=1, host_len=(0,), ws_bytes=1 << 24,
             ws=FAKE + 0x900000, x_scale=None, a_scale=None):
     hl = (C.c_int32 * len(host_len))(*host_len)
