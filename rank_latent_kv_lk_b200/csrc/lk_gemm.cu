@@ -1,7 +1,7 @@
-// Tiled CUDA-core GEMMs, C[m][n] = sum_k A[m][k] * B[n][k] with both operands
-// K-contiguous.  Used for the large-M (prefill) latent projection and for the
-// W8A8 hybrid linear; exact int32 accumulation for int8 (dp4a), fp32 for
-// fp32 / bf16 operands.
+// C[m][n] = sum_k A[m][k] * B[n][k] with both operands K-contiguous.  fp32
+// operands (the fp32 prefill projection): a tiled CUDA-core GEMM with fp32
+// accumulation.  int8 operands (the W8A8 linears and the int8 prefill
+// projection): the tcgen05 kernels of lk_gemm_tc.cu, exact int32.
 #include "lk_common.cuh"
 #include "lk_internal.h"
 
@@ -9,58 +9,6 @@ namespace {
 
 constexpr int kBM = 64, kBN = 64;
 constexpr int kThreads = 256;  // 16 x 16 threads, 4 x 4 outputs each
-
-// ---- int8: K tile of 64 bytes = 16 words per row
-__global__ void __launch_bounds__(kThreads) gemm_i8_kernel(const int8_t* __restrict__ A, int lda,
-                                                          const int8_t* __restrict__ B, int ldb,
-                                                          int32_t* __restrict__ C, int ldc, int M, int N,
-                                                          int K) {
-  __shared__ int32_t As[16][kBM + 4];
-  __shared__ int32_t Bs[16][kBN + 4];
-  const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
-  const int m0 = blockIdx.y * kBM, n0 = blockIdx.x * kBN;
-  const int lrow = tid >> 2, lq = tid & 3;  // loader: row 0..63, 16-byte quarter 0..3
-  int32_t acc[4][4] = {};
-  for (int k0 = 0; k0 < K; k0 += 64) {
-    const int kk = k0 + lq * 16;
-    uint4 av = make_uint4(0, 0, 0, 0), bv = make_uint4(0, 0, 0, 0);
-    if (m0 + lrow < M && kk < K) av = *reinterpret_cast<const uint4*>(A + (int64_t)(m0 + lrow) * lda + kk);
-    if (n0 + lrow < N && kk < K) bv = *reinterpret_cast<const uint4*>(B + (int64_t)(n0 + lrow) * ldb + kk);
-    __syncthreads();
-    As[lq * 4 + 0][lrow] = (int32_t)av.x;
-    As[lq * 4 + 1][lrow] = (int32_t)av.y;
-    As[lq * 4 + 2][lrow] = (int32_t)av.z;
-    As[lq * 4 + 3][lrow] = (int32_t)av.w;
-    Bs[lq * 4 + 0][lrow] = (int32_t)bv.x;
-    Bs[lq * 4 + 1][lrow] = (int32_t)bv.y;
-    Bs[lq * 4 + 2][lrow] = (int32_t)bv.z;
-    Bs[lq * 4 + 3][lrow] = (int32_t)bv.w;
-    __syncthreads();
-#pragma unroll
-    for (int w = 0; w < 16; ++w) {
-      int a[4], b[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[w][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = Bs[w][tx * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = __dp4a(a[i], b[j], acc[i][j]);
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + ty * 4 + i;
-    if (m >= M) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx * 4 + j;
-      if (n < N) C[(int64_t)m * ldc + n] = acc[i][j];
-    }
-  }
-}
 
 // ---- fp32 / bf16 operands, fp32 accumulate: K tile of 16 elements
 template <bool BF16>
@@ -136,13 +84,19 @@ __global__ void __launch_bounds__(kThreads) gemm_f_kernel(const void* __restrict
 
 namespace lk {
 
-// Requires K % 16 == 0 and 16-byte aligned rows (lda, ldb multiples of 16).
+// int8 products run on the tensor cores (lk_gemm_tc.cu); they need 16-byte
+// aligned operands with lda, ldb multiples of 16.
 cudaError_t launch_gemm_i8(const int8_t* A, int lda, const int8_t* B, int ldb, int32_t* C, int ldc,
                            int M, int N, int K, cudaStream_t stream) {
   if (M == 0 || N == 0) return cudaSuccess;
-  dim3 grid((N + kBN - 1) / kBN, (M + kBM - 1) / kBM);
-  gemm_i8_kernel<<<grid, kThreads, 0, stream>>>(A, lda, B, ldb, C, ldc, M, N, K);
-  return cudaGetLastError();
+  if (!gemm_i8_tc_supported(A, lda, B, ldb, K)) return cudaErrorInvalidValue;
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      sms = 148;
+  }
+  return launch_gemm_i8_tc(A, lda, B, ldb, C, ldc, M, N, K, sms, stream);
 }
 
 // Requires K % 4 == 0 (fp32) / K % 4 == 0 (bf16) with 16 / 8-byte aligned rows.

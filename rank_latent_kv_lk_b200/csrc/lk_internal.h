@@ -110,6 +110,11 @@ cudaError_t launch_rowquant(int mode, const void* x, const void* x2, int x_bf16,
 bool gemm_bf16_tc_supported(const void* A, int lda, const void* B, int ldb, int K);
 cudaError_t launch_gemm_bf16_tc(const void* A, int lda, const void* B, int ldb, float* C, int ldc, int M, int N,
                                 int K, cudaStream_t stream);
+// tcgen05 int8 GEMM (exact int32), K split over CTAs with integer atomics;
+// needs lda, ldb multiples of 16 and 16-byte aligned operands.
+bool gemm_i8_tc_supported(const void* A, int lda, const void* B, int ldb, int K);
+cudaError_t launch_gemm_i8_tc(const int8_t* A, int lda, const int8_t* B, int ldb, int32_t* C, int ldc, int M, int N,
+                              int K, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemm_i8(const int8_t* A, int lda, const int8_t* B, int ldb, int32_t* C, int ldc,
                            int M, int N, int K, cudaStream_t stream);
 
