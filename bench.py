@@ -49,6 +49,9 @@ def parse_args(argv=None):
     ap.add_argument("--workload", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layer", action="store_true",
+                    help="time one full W8A8 decoder-layer decode step (workload 5 shape); the latent cache "
+                         "holds seeded random codes (no prefill)")
     ap.add_argument("--attn-only", action="store_true",
                     help="time the latent decode attention alone on one layer of the workload, "
                          "its cache filled with seeded random codes (no prefill)")
@@ -548,6 +551,83 @@ def run_attn_only(args):
     return 0
 
 
+def run_layer(args):
+    """One W8A8 decoder-layer decode step (RMSNorm+quant, W_Q, latent append,
+    latent attention, quant, W_O + residual, RMSNorm+quant, hybrid gate/up,
+    SwiGLU+quant, hybrid down + residual), all through the C ABI."""
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    import rank_latent_kv_lk_b200 as lk
+    from rank_latent_kv_lk_b200 import synth
+    from rank_latent_kv_lk_b200.configs import WORKLOADS
+    from rank_latent_kv_lk_b200.layer import W8A8DecoderLayer
+    w = WORKLOADS[5]
+    rk, rv = synth.ranks(w)
+    rk, rv = rk[0], rv[0]
+    wts = synth.layer_weights_w8a8(w, rk, rv)
+    layer = W8A8DecoderLayer(wts, w.n_heads, w.head_dim, rk, rv, w.batch, w.capacity, w.ffn_inter, device)
+    g = torch.Generator(device=device)
+    g.manual_seed(synth.seed_for(w, synth.CONTEXT))
+    for c in (layer.cache_k, layer.cache_v):
+        c.codes.copy_(torch.randint(0, 256, c.codes.shape, dtype=torch.uint8, device=device, generator=g))
+        c.scales.copy_(torch.rand(c.scales.shape, device=device, generator=g) * 0.02 + 0.01)
+    xs = synth.decode_tokens(w, 0).to(device)  # [steps, B, E] bf16
+    seq = torch.full((w.batch,), w.context, dtype=torch.int32, device=device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    lens = [w.context] * w.batch
+    for i in range(max(3, args.warmup)):
+        layer.step(xs[i % w.steps], seq, lens)
+        seq.fill_(w.context)
+        lens = [w.context] * w.batch
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(2e8))
+    with ClockSampler(local) as clocks:
+        for i in range(K):
+            if i % w.steps == 0 and i:
+                seq.fill_(w.context)
+                lens = [w.context] * w.batch
+            flush.fill_(1)
+            ev[i][0].record(stream)
+            layer.step(xs[i % w.steps], seq, lens)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    lk.device_status()
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), world, device)
+    us = total_ms / K * 1e3
+    nbytes_w = sum(t.numel() * t.element_size() for t in (wts["W_Q"], wts["W_O"], wts["A"]))
+    for name in ("gate", "up", "down"):
+        d = wts[name]
+        nbytes_w += sum(d[k].numel() * d[k].element_size() for k in ("W_D", "U", "V"))
+    T = w.context + 1
+    nbytes_c = w.batch * T * sum(r + r + 8 for r in rk)
+    nbytes = nbytes_w + nbytes_c
+    gbs = nbytes / (us * 1e-6) / 1e9
+    hbm, peak_kind = peaks()
+    if rank == 0:
+        print(json.dumps({
+            "mode": "layer", "metric": "W8A8 decoder-layer decode tokens/s", "value": w.batch * world / (us * 1e-6),
+            "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup, "us_per_step": us,
+            "higher_is_better": True, "scaling": "weak", "dtype": "int8/f32",
+            "data": "synthetic (seeded W8A8 weights; random latent cache codes; shapes of the workload)",
+            "config": {"workload": w.name, "batch": w.batch, "tokens": T,
+                       "l2": "flushed before every step (256 MiB write, untimed)",
+                       "launches": "eager, one stream (about 30 kernel launches per step)"},
+            "algorithmic_bytes_per_step": {"weights": nbytes_w, "latent_cache": nbytes_c},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "peak_kind": peak_kind},
+            "clocks": clocks.summary()}), flush=True)
+    _finish(world)
+    return 0
+
+
 def _finish(world):
     if world > 1 and torch.distributed.is_initialized():
         torch.distributed.destroy_process_group()
@@ -561,6 +641,8 @@ def main(argv=None):
         return run_reference(args)
     if args.attn_only:
         return run_attn_only(args)
+    if args.layer:
+        return run_layer(args)
     return run_ours(args)
 
 

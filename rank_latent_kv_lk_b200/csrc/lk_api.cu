@@ -319,7 +319,7 @@ lk_status lk_lowrank_linear(const lk_lowrank_weight* w, const int8_t* x_q, const
     return fail(LK_ERR_SHAPE, "a low-rank branch needs both channels (%d) and rank (%d)", n_lr, w->rank);
   if (w->n_dense % 16 || n_lr % 16 || w->rank % 16)
     return fail(LK_ERR_ALIGN, "n_dense, k_in - n_dense and rank must be multiples of 16");
-  if (m < 0) return fail(LK_ERR_SHAPE, "m %d < 0", m);
+  if (m < 0 || m > 65535) return fail(LK_ERR_SHAPE, "m %d outside [0, 65535]", m);
   if (!x_q || !x_scale || !y) return fail(LK_ERR_INVALID_ARG, "null x_q, x_scale or y");
   if (y_dtype != LK_BF16 && y_dtype != LK_F32) return fail(LK_ERR_DTYPE, "y dtype must be LK_BF16 or LK_F32");
   if (w->n_dense > 0 && (!w->dense_idx || !w->W_D || !w->s_D))

@@ -55,19 +55,20 @@ __global__ void __launch_bounds__(256) requant_kernel(const int32_t* __restrict_
   }
 }
 
+// One CTA row per token row (blockIdx.y), columns strided over x.
 __global__ void lowrank_epilogue_kernel(const int32_t* __restrict__ accD, const int32_t* __restrict__ accV,
                                         const float* __restrict__ x_scale, const float* __restrict__ s_t,
                                         const uint16_t* __restrict__ s_D, const uint16_t* __restrict__ s_V,
                                         const uint16_t* __restrict__ residual, int m, int n, void* y,
                                         int y_bf16) {
-  const int64_t total = (int64_t)m * n;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = i / n;
-    const int col = (int)(i % n);
+  const int64_t row = blockIdx.y;
+  const float sx = accD ? x_scale[row] : 0.0f;
+  const float st = accV ? s_t[row] : 0.0f;
+  for (int col = blockIdx.x * blockDim.x + threadIdx.x; col < n; col += gridDim.x * blockDim.x) {
+    const int64_t i = row * n + col;
     float out = 0.0f;
-    if (accD) out = __fmul_rn(__fmul_rn((float)accD[i], x_scale[row]), lk_f16_to_f32(s_D[col]));
-    if (accV) out += __fmul_rn(__fmul_rn((float)accV[i], s_t[row]), lk_f16_to_f32(s_V[col]));
+    if (accD) out = __fmul_rn(__fmul_rn((float)accD[i], sx), lk_f16_to_f32(s_D[col]));
+    if (accV) out += __fmul_rn(__fmul_rn((float)accV[i], st), lk_f16_to_f32(s_V[col]));
     if (residual) out += lk_bf16_to_f32(residual[i]);
     if (y_bf16) static_cast<uint16_t*>(y)[i] = lk_f32_to_bf16(out);
     else static_cast<float*>(y)[i] = out;
@@ -141,10 +142,9 @@ cudaError_t launch_lowrank_linear(const LowrankLaunch& a, cudaStream_t stream) {
     e = launch_gemm_i8(t_q, ld_tq, a.V, a.rank, accV, a.n_out, a.m, a.n_out, a.rank, stream);
     if (e != cudaSuccess) return e;
   }
-  const int64_t total = (int64_t)a.m * a.n_out;
-  const int blocks = (int)std::min<int64_t>((total + 255) / 256, (int64_t)a.num_sms * 8);
-  lowrank_epilogue_kernel<<<blocks, 256, 0, stream>>>(accD, accV, a.x_scale, s_t, a.s_D, a.s_V, a.residual,
-                                                      a.m, a.n_out, a.y, a.y_bf16);
+  const dim3 egrid((unsigned)std::min((a.n_out + 255) / 256, 64), (unsigned)a.m);
+  lowrank_epilogue_kernel<<<egrid, 256, 0, stream>>>(accD, accV, a.x_scale, s_t, a.s_D, a.s_V, a.residual, a.m,
+                                                     a.n_out, a.y, a.y_bf16);
   return cudaGetLastError();
 }
 

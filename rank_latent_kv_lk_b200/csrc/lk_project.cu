@@ -30,7 +30,7 @@ namespace {
 constexpr int kGemvThreads = 256;
 constexpr int kColsPerWarp = 4;
 constexpr int kColsPerCta = kColsPerWarp * (kGemvThreads / 32);  // 32
-constexpr int kGemvMaxRows = 32;
+constexpr int kGemvMaxRows = 8;  // more rows: the tensor-core GEMM, then the quantise-and-append pass
 
 template <int XT> struct XTraits;
 template <> struct XTraits<lk::X_F32> { using T = float; static constexpr int VE = 4; };

@@ -72,14 +72,44 @@ __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(int mode, const v
   const T* xr = reinterpret_cast<const T*>(x) + row * k;
   const T* x2r = reinterpret_cast<const T*>(x2) + row * k;
   float ss = 0.0f;
-  for (int i = threadIdx.x; i < k; i += kRowThreads) {
-    float a = lk_load_f<T>(xr, i);
-    if (mode == 2) {
-      const float b = lk_load_f<T>(x2r, i);
-      a = __fmul_rn(__fdiv_rn(a, 1.0f + expf(-a)), b);
+  auto f = [&](float a, float b) { return mode == 2 ? __fmul_rn(__fdiv_rn(a, 1.0f + expf(-a)), b) : a; };
+  constexpr int VE = BF16 ? 8 : 4;  // elements per 16-byte vector
+  const bool vec = (k % VE) == 0 && ((reinterpret_cast<uintptr_t>(xr) | reinterpret_cast<uintptr_t>(x2r)) & 15) == 0;
+  if (vec) {
+    // 16-byte loads, several in flight per thread
+    const int nv = k / VE;
+#pragma unroll 4
+    for (int v = threadIdx.x; v < nv; v += kRowThreads) {
+      const uint4 xv = reinterpret_cast<const uint4*>(xr)[v];
+      uint4 yv = make_uint4(0, 0, 0, 0);
+      if (mode == 2) yv = reinterpret_cast<const uint4*>(x2r)[v];
+      float xa[VE], xb[VE];
+      if constexpr (BF16) {
+        const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w}, u[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          xa[2 * j] = lk_bf16lo(w[j]); xa[2 * j + 1] = lk_bf16hi(w[j]);
+          xb[2 * j] = lk_bf16lo(u[j]); xb[2 * j + 1] = lk_bf16hi(u[j]);
+        }
+      } else {
+        xa[0] = __uint_as_float(xv.x); xa[1] = __uint_as_float(xv.y);
+        xa[2] = __uint_as_float(xv.z); xa[3] = __uint_as_float(xv.w);
+        xb[0] = __uint_as_float(yv.x); xb[1] = __uint_as_float(yv.y);
+        xb[2] = __uint_as_float(yv.z); xb[3] = __uint_as_float(yv.w);
+      }
+#pragma unroll
+      for (int j = 0; j < VE; ++j) {
+        const float a = f(xa[j], xb[j]);
+        ys[v * VE + j] = a;
+        ss = fmaf(a, a, ss);
+      }
     }
-    ys[i] = a;
-    ss = fmaf(a, a, ss);
+  } else {
+    for (int i = threadIdx.x; i < k; i += kRowThreads) {
+      const float a = f(lk_load_f<T>(xr, i), mode == 2 ? lk_load_f<T>(x2r, i) : 0.0f);
+      ys[i] = a;
+      ss = fmaf(a, a, ss);
+    }
   }
   if (mode == 1) {
     const float tot = block_reduce(ss, scratch, false);

@@ -5,8 +5,8 @@ layer with unit RMSNorm weights, eps 1e-5, no positional rotation):
 
   x_q      = int8(RMSNorm(x))
   q        = x_q W_Q^T                      (W8A8 dense linear)
-  latents  = quant(x_q A^T) appended        (lk_latent_project_append)
-  a        = latent attention               (lk_latent_decode_attn)
+  latents  = quant(x_q A^T) appended        (lk_latent_decode_step: append,
+  a        = latent attention                 then attention)
   x2       = x + int8(a) W_O^T              (W8A8 dense linear + residual)
   h_q      = int8(RMSNorm(x2))
   g, u     = hybrid(h_q; gate), hybrid(h_q; up)     (LASER hybrid linear)
@@ -19,8 +19,8 @@ from __future__ import annotations
 
 import torch
 
-from .api import (LatentCache, LowrankWeight, latent_decode_attn, latent_project_append, lowrank_linear,
-                  quantize_rows_i8, rmsnorm_quant_i8, swiglu_quant_i8)
+from .api import (LatentCache, LowrankWeight, latent_decode_step, lowrank_linear, quantize_rows_i8,
+                  rmsnorm_quant_i8, swiglu_quant_i8)
 
 
 def dense_weight(W, s, device):
@@ -61,11 +61,13 @@ class W8A8DecoderLayer:
         B = x.shape[0]
         xq, sx = rmsnorm_quant_i8(x)
         q = lowrank_linear(self.wq, xq, sx)
-        latent_project_append(self.cache_k, self.cache_v, xq, self.A, seq_len, lens, sx, self.s_A)
+        # append the new token's latents, then attend (the attention launch
+        # overlaps the append)
+        attn = latent_decode_step(self.cache_k, self.cache_v, xq, self.A, seq_len, lens,
+                                  q.view(B, self.n_heads, self.head_dim), self.B_K, self.B_V, x_scale=sx,
+                                  a_scale=self.s_A, out_dtype=torch.bfloat16)
         for b in range(B):
             lens[b] += 1
-        attn = latent_decode_attn(self.cache_k, self.cache_v, q.view(B, self.n_heads, self.head_dim), self.B_K,
-                                  self.B_V, seq_len, max(lens), out_dtype=torch.bfloat16)
         aq, sa = quantize_rows_i8(attn.view(B, self.n_heads * self.head_dim))
         x2 = lowrank_linear(self.wo, aq, sa, residual=x)
         hq, sh = rmsnorm_quant_i8(x2)
