@@ -211,7 +211,7 @@ lk_status decode_attn_impl(const lk_latent_cache* k, const lk_latent_cache* v, c
                            const void* B_K, const void* B_V, lk_dtype b_dtype, int32_t head_dim,
                            const int32_t* seq_len, int32_t max_seq_len, float softmax_scale, void* out,
                            lk_dtype out_dtype, int32_t n_split, void* workspace, size_t workspace_bytes,
-                           lk_stream_t stream, bool launch, int early_inputs) {
+                           lk_stream_t stream, bool launch, int early_inputs, int stable_len) {
   lk_status s;
   if ((s = check_cache(k, "k_cache", true)) != LK_OK) return s;
   if ((s = check_cache(v, "v_cache", true)) != LK_OK) return s;
@@ -264,6 +264,7 @@ lk_status decode_attn_impl(const lk_latent_cache* k, const lk_latent_cache* v, c
   a.num_sms = num_sms();
   a.softmax_scale = softmax_scale;
   a.early_inputs = early_inputs;
+  a.stable_len = stable_len;
   if (!launch) return LK_OK;
   cudaError_t e = lk::launch_decode_attn(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "lk_latent_decode_attn");
@@ -277,7 +278,7 @@ lk_status lk_latent_decode_attn(const lk_latent_cache* k, const lk_latent_cache*
                                 float softmax_scale, void* out, lk_dtype out_dtype, int32_t n_split,
                                 void* workspace, size_t workspace_bytes, lk_stream_t stream) {
   return decode_attn_impl(k, v, q, q_dtype, B_K, B_V, b_dtype, head_dim, seq_len, max_seq_len, softmax_scale, out,
-                          out_dtype, n_split, workspace, workspace_bytes, stream, true, 0);
+                          out_dtype, n_split, workspace, workspace_bytes, stream, true, 0, 0);
 }
 
 lk_status lk_latent_decode_step(const lk_latent_cache* k, const lk_latent_cache* v, const void* x, lk_dtype x_dtype,
@@ -289,17 +290,21 @@ lk_status lk_latent_decode_step(const lk_latent_cache* k, const lk_latent_cache*
                                 void* decode_workspace, size_t decode_workspace_bytes, lk_stream_t stream) {
   if (!k || !seq_len_host) return fail(LK_ERR_INVALID_ARG, "null k_cache or seq_len_host");
   if (k->batch < 1) return fail(LK_ERR_SHAPE, "batch %d < 1", k->batch);
-  int max_len = 0;
-  for (int b = 0; b < k->batch; ++b) max_len = std::max(max_len, (int)seq_len_host[b] + 1);
+  int max_len = 0, stable_len = INT32_MAX;
+  for (int b = 0; b < k->batch; ++b) {
+    max_len = std::max(max_len, (int)seq_len_host[b] + 1);
+    stable_len = std::min(stable_len, (int)seq_len_host[b]);  // the append writes at or past it
+  }
   // the attention is validated first, so a rejected call launches nothing
   lk_status s = decode_attn_impl(k, v, q, q_dtype, B_K, B_V, b_dtype, head_dim, seq_len, max_len, softmax_scale,
-                                 out, out_dtype, n_split, decode_workspace, decode_workspace_bytes, stream, false, 1);
+                                 out, out_dtype, n_split, decode_workspace, decode_workspace_bytes, stream, false, 1,
+                                 stable_len);
   if (s != LK_OK) return s;
   s = lk_latent_project_append(k, v, x, x_dtype, x_scale, A, a_dtype, a_scale, embed_dim, 1, seq_len, seq_len_host,
                                project_workspace, project_workspace_bytes, stream);
   if (s != LK_OK) return s;
   return decode_attn_impl(k, v, q, q_dtype, B_K, B_V, b_dtype, head_dim, seq_len, max_len, softmax_scale, out,
-                          out_dtype, n_split, decode_workspace, decode_workspace_bytes, stream, true, 1);
+                          out_dtype, n_split, decode_workspace, decode_workspace_bytes, stream, true, 1, stable_len);
 }
 
 size_t lk_lowrank_workspace_bytes(const lk_lowrank_weight* w, int32_t m) {

@@ -81,6 +81,7 @@ struct DecodeParams {
   int tk, tv, tgk, tgv;  // code bytes / scale groups of one batch row (all heads)
   int q_bf16, b_bf16, out_bf16;
   int early_inputs;  // q, B_K, B_V are read before waiting for the previous kernel on the stream
+  int stable_len;    // with early_inputs: cache positions below it are final before the kernel starts
   int max_len;
   int S;   // stages per unit: ceil(max_len / kStageT)
   int W;   // items: units * S
@@ -433,6 +434,7 @@ LK_DEVICE void produce(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
   int u = i0 / p.S, s = i0 - u * p.S;
   int it = i0, k = 0, nunit = 0, nf = 0;  // stages issued, units begun, factor copies issued
   bool ok = true;
+  bool waited = !p.early_inputs;  // the previous kernel on the stream has completed
   while (it < i1) {
     const int s_end = min(p.S, s + (i1 - it));
     const int b = u / p.n_heads, h = u - b * p.n_heads;
@@ -449,12 +451,19 @@ LK_DEVICE void produce(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
       lk_bulk_g2s(smem + L.off_bk, static_cast<const uint8_t*>(p.BK) + g.bk_off * p.b_size, bkb, B.fbar);
       ++nf;
     }
-    if (nunit == 0 && p.early_inputs) lk_grid_dep_wait();  // the cache and seq_len are the previous kernel's
     ++nunit;
-    const int len = unit_len(p, b);
-    const int64_t end = min((int64_t)((len + 15) & ~15), (int64_t)p.capacity);
+    // until the wait, only stages below the stable prefix are read: they are
+    // full (every row is at least stable_len long) and final
+    int len = waited ? unit_len(p, b) : p.stable_len;
+    int64_t end = min((int64_t)((len + 15) & ~15), (int64_t)p.capacity);
     for (int ss = s; ss < s_end && ok; ++ss) {
       const int64_t t0 = (int64_t)ss * kStageT;
+      if (!waited && t0 + kStageT > p.stable_len) {  // the stage may hold what the append writes
+        lk_grid_dep_wait();
+        waited = true;
+        len = unit_len(p, b);
+        end = min((int64_t)((len + 15) & ~15), (int64_t)p.capacity);
+      }
       if (t0 >= len) break;  // this and the unit's later stages hold no tokens
       if (*B.abort_flag) {
         ok = false;
@@ -481,6 +490,7 @@ LK_DEVICE void produce(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
     ++u;
     s = 0;
   }
+  if (!waited) lk_grid_dep_wait();  // this grid never completes before the previous one
   // before the CTA may finish, every copy this CTA started has landed
   for (int j = max(0, k - NS); j < k; ++j)
     if (!lk_mbar_wait_bounded(&B.full[j % NS], (uint32_t)((j / NS) & 1), LK_WAIT_LIMIT_NS))
@@ -552,8 +562,8 @@ LK_DEVICE void absorb_q(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
 // stage, fixed at compile time (runtime bounds on these loops cost more
 // instructions than the products themselves).
 template <int KIND, int CSK, int NM, bool VG1>
-LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, const HeadGeom& g, int len,
-                        int s0, int s1, int& buf, uint32_t& phase) {
+LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, const HeadGeom& g, int b,
+                        int len, int s0, int s1, int& buf, uint32_t& phase, bool& waited) {
   const Bars B = bars_of(smem, L);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int NS = p.nstages;
@@ -592,8 +602,14 @@ LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
     }
   };
 
-  const int tl_end = len - s0 * kStageT - tl;  // token (s0 + j) * kStageT + tl is valid iff j * kStageT < tl_end
+  int tl_end = len - s0 * kStageT - tl;  // token (s0 + j) * kStageT + tl is valid iff j * kStageT < tl_end
   for (int j = 0; j < s1 - s0; ++j) {
+    if (!waited && (s0 + j + 1) * kStageT > p.stable_len) {  // past the stable prefix: the append's output
+      lk_grid_dep_wait();
+      waited = true;
+      len = unit_len(p, b);
+      tl_end = len - s0 * kStageT - tl;
+    }
     if ((s0 + j) * kStageT >= len) break;  // no copies were issued for the unit's later stages
     if (*B.abort_flag) break;
     if (!lk_mbar_wait_bounded(&B.full[buf], phase, LK_WAIT_LIMIT_NS)) *B.abort_flag = 1;
@@ -690,18 +706,20 @@ LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
 }
 
 template <int KIND, int CSK, bool VG1>
-LK_DEVICE void run_unit_nm(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, const HeadGeom& g, int len,
-                           int s0, int s1, int& buf, uint32_t& phase) {
+LK_DEVICE void run_unit_nm(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, const HeadGeom& g, int b,
+                           int len, int s0, int s1, int& buf, uint32_t& phase, bool& waited) {
+#define LK_RUN(NMV) run_unit<KIND, CSK, NMV, VG1>(p, smem, L, g, b, len, s0, s1, buf, phase, waited)
   switch ((g.rv + 7) >> 3) {
-    case 1: run_unit<KIND, CSK, 1, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
-    case 2: run_unit<KIND, CSK, 2, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
-    case 3: run_unit<KIND, CSK, 3, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
-    case 4: run_unit<KIND, CSK, 4, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
-    case 5: run_unit<KIND, CSK, 5, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
-    case 6: run_unit<KIND, CSK, 6, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
-    case 7: run_unit<KIND, CSK, 7, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
-    default: run_unit<KIND, CSK, 8, VG1>(p, smem, L, g, len, s0, s1, buf, phase); break;
+    case 1: LK_RUN(1); break;
+    case 2: LK_RUN(2); break;
+    case 3: LK_RUN(3); break;
+    case 4: LK_RUN(4); break;
+    case 5: LK_RUN(5); break;
+    case 6: LK_RUN(6); break;
+    case 7: LK_RUN(7); break;
+    default: LK_RUN(8); break;
   }
+#undef LK_RUN
 }
 
 // Block-wide max over the consumer threads (red: kCW floats of shared memory).
@@ -837,23 +855,24 @@ LK_DEVICE void consume(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
   int u = i0 / p.S, s = i0 - u * p.S;
   int it = i0, n = 0, buf = 0;
   uint32_t phase = 0u;
+  bool waited = !p.early_inputs;  // this thread waited for the previous kernel on the stream
   while (it < i1) {
     const int s_end = min(p.S, s + (i1 - it));
     const int seg_end = it + (s_end - s);
     const int b = u / p.n_heads, h = u - b * p.n_heads;
     const HeadGeom g = unit_geometry<KIND>(p, b, h);
     absorb_q<KIND>(p, smem, L, g, n);
-    if (n == 0 && p.early_inputs) lk_grid_dep_wait();  // the cache and seq_len are the previous kernel's
-    const int len = unit_len(p, b);
+    // before the wait, the stable prefix is the length every row has
+    const int len = waited ? unit_len(p, b) : p.stable_len;
     const int csk = lk_chunk_bytes(g.rbk);
     if (KIND == 0 || g.ngv == 1) {
-      if (csk == 16) run_unit_nm<KIND, 16, true>(p, smem, L, g, len, s, s_end, buf, phase);
-      else if (csk == 8) run_unit_nm<KIND, 8, true>(p, smem, L, g, len, s, s_end, buf, phase);
-      else run_unit_nm<KIND, 4, true>(p, smem, L, g, len, s, s_end, buf, phase);
+      if (csk == 16) run_unit_nm<KIND, 16, true>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      else if (csk == 8) run_unit_nm<KIND, 8, true>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      else run_unit_nm<KIND, 4, true>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
     } else if constexpr (KIND == 1) {
-      if (csk == 16) run_unit_nm<KIND, 16, false>(p, smem, L, g, len, s, s_end, buf, phase);
-      else if (csk == 8) run_unit_nm<KIND, 8, false>(p, smem, L, g, len, s, s_end, buf, phase);
-      else run_unit_nm<KIND, 4, false>(p, smem, L, g, len, s, s_end, buf, phase);
+      if (csk == 16) run_unit_nm<KIND, 16, false>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      else if (csk == 8) run_unit_nm<KIND, 8, false>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      else run_unit_nm<KIND, 4, false>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
     }
     finish_unit<KIND>(p, smem, L, g, b, h, u, it, seg_end, i0, c, n);
     it = seg_end;
@@ -861,6 +880,7 @@ LK_DEVICE void consume(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
     ++n;
     s = 0;
   }
+  if (!waited) lk_grid_dep_wait();  // this grid never completes before the previous one
 }
 
 template <int KIND>
@@ -967,6 +987,7 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   p.b_bf16 = a.b_bf16;
   p.out_bf16 = a.out_bf16;
   p.early_inputs = a.early_inputs;
+  p.stable_len = a.early_inputs ? std::max(0, std::min(a.stable_len, a.max_len)) : 0;
   p.max_len = a.max_len;
   p.qscale = a.softmax_scale * 1.4426950408889634f;
   int rk_max = 0, rv_max = 0, ngk_max = 1, ngv_max = 1;
@@ -1030,7 +1051,14 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   const int units = a.batch * a.n_heads;
   p.S = decode_stages(a.max_len);
   const int64_t W = (int64_t)units * p.S;
-
+  // a ring deeper than the stages a CTA streams only costs shared memory (and
+  // keeps the kernel off SMs the previous kernel still occupies): size it for
+  // the grid a full GPU would take
+  {
+    const int64_t g_full = decode_ctas(units, a.max_len, a.n_split, std::min(2 * a.num_sms, kAutoCtaBound));
+    const int64_t per_cta = (W + g_full - 1) / std::max<int64_t>(1, g_full) + 1;
+    p.nstages = (int)std::max<int64_t>(2, std::min<int64_t>(p.nstages, per_cta));
+  }
   const int smem = smem_bytes_for(p);
   cudaError_t e = a.kind == 0
                       ? cudaFuncSetAttribute(decode_attn_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)

@@ -32,6 +32,7 @@ struct DecodeLaunch {
   int q_bf16, b_bf16, out_bf16;
   int max_len, n_split, num_sms;
   int early_inputs;  // read q, B_K, B_V before waiting for the previous kernel (decode step entry point)
+  int stable_len;    // with early_inputs: positions below it are final before the kernel starts
   float softmax_scale;
 };
 // Workspace of a decode call: arrival counters for the units plus two partial
