@@ -155,10 +155,12 @@ size_t lk_latent_project_workspace_bytes(const lk_latent_cache* k_cache,
  *   s_t = softmax_scale * sigma_K[t] . (c_K[t] . q~)   (per group for int4)
  *   p = softmax(s);  u = sum_t p_t * sigma_V[t] * c_V[t]   (r_V values)
  *   out^h = u B_V^h                                  ([H])
- * computed split-K over t (flash-decoding): the (b, h, 224-token stage)
- * items are dealt out in equal ranges to a fixed grid of CTAs; a (b, h) cut
- * by a range boundary leaves partials (max, sum, u) that are merged in latent
- * space by the last piece to finish.  K and V are never formed.
+ * computed split-K over t (flash-decoding): the (b, h, stage) items
+ * (448-token stages, or 224 where two 448-token stages of the widest head
+ * do not fit in shared memory) are dealt out in equal ranges to a fixed
+ * grid of CTAs; a (b, h) cut by a range boundary leaves partials (max, sum,
+ * u) that are merged in latent space by the last piece to finish.  K and V
+ * are never formed.
  *
  * q: [B, n_heads, head_dim], q_dtype LK_F32 or LK_BF16; head_dim a multiple
  *   of 8 (<= LK_MAX_HEAD_DIM); q, B_K and B_V 16-byte aligned (they are
@@ -171,7 +173,7 @@ size_t lk_latent_project_workspace_bytes(const lk_latent_cache* k_cache,
  *   A row with seq_len 0 gets a zero output.
  * out: [B, n_heads, head_dim], LK_F32 or LK_BF16.
  * n_split: about how many pieces each (b, h) is cut into (grid = B * n_heads
- *   * n_split CTAs, at most one per 224-token stage); 0 picks a grid that
+ *   * n_split CTAs, at most one per stage); 0 picks a grid that
  *   fills the GPU.  The result does not depend on it beyond float rounding.
  * workspace: lk_latent_decode_workspace_bytes(...) bytes, 256-B aligned.
  *   Its first round_up(4 * B * n_heads, 256) bytes are per-(b, h) arrival

@@ -49,7 +49,9 @@ namespace {
 constexpr int kCW = 7;                           // consumer warps
 constexpr int kConsumerThreads = kCW * 32;
 constexpr int kThreads = kConsumerThreads + 32;  // + one producer warp
-constexpr int kStageT = 32 * kCW;                // tokens per stage (224): 32 per consumer warp
+// tokens per stage: TG groups of 32 per consumer warp (TG = 2 when two stages
+// of the widest head fit beside each other in ~110 KB, else 1)
+constexpr int kStageMin = 32 * kCW;  // 224 (TG = 1); 448 with TG = 2
 constexpr int kMaxStages = 8;                    // ring depth chosen at launch (2 .. 8)
 constexpr int kMaxR = LK_MAX_RANK;
 constexpr int kAutoCtaBound = 1024;              // grid bound of the automatic split (sizes the workspace)
@@ -83,7 +85,8 @@ struct DecodeParams {
   int early_inputs;  // q, B_K, B_V are read before waiting for the previous kernel on the stream
   int stable_len;    // with early_inputs: cache positions below it are final before the kernel starts
   int max_len;
-  int S;   // stages per unit: ceil(max_len / kStageT)
+  int ST;  // tokens per stage: 32 * TG * kCW
+  int S;   // stages per unit: ceil(max_len / ST)
   int W;   // items: units * S
   int G;   // CTAs
   int part_stride;
@@ -283,40 +286,49 @@ LK_DEVICE void lds_words(const void* p, uint32_t (&w)[N]) {
   }
 }
 
-// Score of one token in log2 units: sum over groups g of
+// Scores of two tokens (tl and tl + 32) in log2 units: sum over groups g of
 //   sigma_g * a * (D0 + D1/254 + D2/254^2),  D_i = c . t_i  (exact dp4a sums)
-// with the q~ terms t_i read from shared memory (the same words for every
-// lane: broadcast loads).  int8 keys: one group and one scale per token.
-template <int KIND, int CS>
-LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom& g, int tl,
-                            const int8_t* qterm, float qa) {
+// with the q~ terms t_i read from shared memory once for both tokens (the
+// same words for every lane: broadcast loads).  int8 keys: one group and one
+// scale per token.  The two tokens' chains are independent (instruction-level
+// parallelism for the warp).
+template <int KIND, int CS, int TG>
+LK_DEVICE void token_score2(const uint8_t* kc, const uint8_t* ks, const HeadGeom& g, int tl, const int8_t* qterm,
+                            float qa, float& sa, float& sb) {
   constexpr int WPC = CS / 4;  // words per chunk
   constexpr int MAXCH = (KIND == 0 ? kMaxR : kMaxR / 2) / CS;
   const int nch = g.rbk / CS;
+  const int tb = tl + 32;
   if (KIND == 0) {
-    int d0 = 0, d1 = 0, d2 = 0;
+    int a0 = 0, a1 = 0, a2 = 0, b0 = 0, b1 = 0, b2 = 0;
 #pragma unroll
     for (int c = 0; c < MAXCH; ++c) {
       if (c < nch) {
-        Chunk<CS> ch;
-        ch.load(kc, g.rbk, tl, c);
+        Chunk<CS> ca, cb;
+        ca.load(kc, g.rbk, tl, c);
+        if constexpr (TG == 2) cb.load(kc, g.rbk, tb, c);
         uint32_t t0[WPC], t1[WPC], t2[WPC];
         lds_words<WPC>(qterm + 0 * kMaxR + c * CS, t0);
         lds_words<WPC>(qterm + 1 * kMaxR + c * CS, t1);
         lds_words<WPC>(qterm + 2 * kMaxR + c * CS, t2);
 #pragma unroll
         for (int wi = 0; wi < WPC; ++wi) {
-          d0 = __dp4a((int)ch.w[wi], (int)t0[wi], d0);
-          d1 = __dp4a((int)ch.w[wi], (int)t1[wi], d1);
-          d2 = __dp4a((int)ch.w[wi], (int)t2[wi], d2);
+          a0 = __dp4a((int)ca.w[wi], (int)t0[wi], a0);
+          if constexpr (TG == 2) b0 = __dp4a((int)cb.w[wi], (int)t0[wi], b0);
+          a1 = __dp4a((int)ca.w[wi], (int)t1[wi], a1);
+          if constexpr (TG == 2) b1 = __dp4a((int)cb.w[wi], (int)t1[wi], b1);
+          a2 = __dp4a((int)ca.w[wi], (int)t2[wi], a2);
+          if constexpr (TG == 2) b2 = __dp4a((int)cb.w[wi], (int)t2[wi], b2);
         }
       }
     }
-    const float x = fmaf((float)d2, kInv254sq, fmaf((float)d1, kInv254, (float)d0));
-    return reinterpret_cast<const float*>(ks)[tl] * (qa * x);
+    const float xa = fmaf((float)a2, kInv254sq, fmaf((float)a1, kInv254, (float)a0));
+    const float xb = fmaf((float)b2, kInv254sq, fmaf((float)b1, kInv254, (float)b0));
+    sa = reinterpret_cast<const float*>(ks)[tl] * (qa * xa);
+    if constexpr (TG == 2) sb = reinterpret_cast<const float*>(ks)[tb] * (qa * xb);
   } else {
-    float s = 0.0f;
-    int d0 = 0, d1 = 0, d2 = 0;
+    float s_a = 0.0f, s_b = 0.0f;
+    int a0 = 0, a1 = 0, a2 = 0, b0 = 0, b1 = 0, b2 = 0;
     int cur_g = 0;
     const int wpg = g.gk >> 3;  // code words per scale group
     int wleft = wpg;            // words left in the current group
@@ -325,8 +337,9 @@ LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom
 #pragma unroll
     for (int c = 0; c < MAXCH; ++c) {
       if (c < nch) {
-        Chunk<CS> ch;
-        ch.load(kc, g.rbk, tl, c);
+        Chunk<CS> ca, cb;
+        ca.load(kc, g.rbk, tl, c);
+        if constexpr (TG == 2) cb.load(kc, g.rbk, tb, c);
         uint32_t t0[2 * WPC], t1[2 * WPC], t2[2 * WPC];
         lds_words<2 * WPC>(qterm + 0 * kMaxR + c * 2 * CS, t0);
         lds_words<2 * WPC>(qterm + 1 * kMaxR + c * 2 * CS, t1);
@@ -334,26 +347,34 @@ LK_DEVICE float token_score(const uint8_t* kc, const uint8_t* ks, const HeadGeom
 #pragma unroll
         for (int wi = 0; wi < WPC; ++wi) {
           if (wleft == 0) {  // flush the finished group (uniform branch)
-            const float x = fmaf((float)d2, kInv254sq, fmaf((float)d1, kInv254, (float)d0));
-            s = fmaf(load_scale(ks, tl * g.ngk + cur_g, 1), qa * x, s);
-            d0 = d1 = d2 = 0;
+            const float sg_a = load_scale(ks, tl * g.ngk + cur_g, 1);
+            s_a = fmaf(sg_a, qa * fmaf((float)a2, kInv254sq, fmaf((float)a1, kInv254, (float)a0)), s_a);
+            if constexpr (TG == 2) {
+              const float sg_b = load_scale(ks, tb * g.ngk + cur_g, 1);
+              s_b = fmaf(sg_b, qa * fmaf((float)b2, kInv254sq, fmaf((float)b1, kInv254, (float)b0)), s_b);
+            }
+            a0 = a1 = a2 = b0 = b1 = b2 = 0;
             ++cur_g;
             wleft = wpg;
           }
           --wleft;
-          int ev, od;
-          nibbles_to_s8(ch.w[wi], ev, od);
-          d0 = __dp4a(od, (int)t0[2 * wi + 1], __dp4a(ev, (int)t0[2 * wi], d0));
-          d1 = __dp4a(od, (int)t1[2 * wi + 1], __dp4a(ev, (int)t1[2 * wi], d1));
-          d2 = __dp4a(od, (int)t2[2 * wi + 1], __dp4a(ev, (int)t2[2 * wi], d2));
+          int eva, oda, evb = 0, odb = 0;
+          nibbles_to_s8(ca.w[wi], eva, oda);
+          if constexpr (TG == 2) nibbles_to_s8(cb.w[wi], evb, odb);
+          a0 = __dp4a(oda, (int)t0[2 * wi + 1], __dp4a(eva, (int)t0[2 * wi], a0));
+          if constexpr (TG == 2) b0 = __dp4a(odb, (int)t0[2 * wi + 1], __dp4a(evb, (int)t0[2 * wi], b0));
+          a1 = __dp4a(oda, (int)t1[2 * wi + 1], __dp4a(eva, (int)t1[2 * wi], a1));
+          if constexpr (TG == 2) b1 = __dp4a(odb, (int)t1[2 * wi + 1], __dp4a(evb, (int)t1[2 * wi], b1));
+          a2 = __dp4a(oda, (int)t2[2 * wi + 1], __dp4a(eva, (int)t2[2 * wi], a2));
+          if constexpr (TG == 2) b2 = __dp4a(odb, (int)t2[2 * wi + 1], __dp4a(evb, (int)t2[2 * wi], b2));
         }
       }
     }
-    const float x = fmaf((float)d2, kInv254sq, fmaf((float)d1, kInv254, (float)d0));
-    return fmaf(load_scale(ks, tl * g.ngk + cur_g, 1), qa * x, s);
+    sa = fmaf(load_scale(ks, tl * g.ngk + cur_g, 1), qa * fmaf((float)a2, kInv254sq, fmaf((float)a1, kInv254, (float)a0)), s_a);
+    if constexpr (TG == 2)
+      sb = fmaf(load_scale(ks, tb * g.ngk + cur_g, 1), qa * fmaf((float)b2, kInv254sq, fmaf((float)b1, kInv254, (float)b0)), s_b);
   }
 }
-
 
 struct SmemLayout {
   int stage_bytes;
@@ -457,8 +478,8 @@ LK_DEVICE void produce(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
     int len = waited ? unit_len(p, b) : p.stable_len;
     int64_t end = min((int64_t)((len + 15) & ~15), (int64_t)p.capacity);
     for (int ss = s; ss < s_end && ok; ++ss) {
-      const int64_t t0 = (int64_t)ss * kStageT;
-      if (!waited && t0 + kStageT > p.stable_len) {  // the stage may hold what the append writes
+      const int64_t t0 = (int64_t)ss * p.ST;
+      if (!waited && t0 + p.ST > p.stable_len) {  // the stage may hold what the append writes
         lk_grid_dep_wait();
         waited = true;
         len = unit_len(p, b);
@@ -475,7 +496,7 @@ LK_DEVICE void produce(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
         ok = false;
         break;
       }
-      const int ntok = (int)min((int64_t)kStageT, end - t0);
+      const int ntok = (int)min((int64_t)p.ST, end - t0);
       uint8_t* st = smem + buf * L.stage_bytes;
       const uint32_t bkc = ntok * g.rbk, bvc = ntok * g.rbv;
       const uint32_t bks = ntok * g.ngk * ssz, bvs = ntok * g.ngv * ssz;
@@ -561,7 +582,7 @@ LK_DEVICE void absorb_q(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
 // CTA's next stage, carried across units.  NM = ceil(r_V / 8) V products per
 // stage, fixed at compile time (runtime bounds on these loops cost more
 // instructions than the products themselves).
-template <int KIND, int CSK, int NM, bool VG1>
+template <int KIND, int CSK, int NM, bool VG1, int TG>
 LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, const HeadGeom& g, int b,
                         int len, int s0, int s1, int& buf, uint32_t& phase, bool& waited) {
   const Bars B = bars_of(smem, L);
@@ -575,7 +596,9 @@ LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
   // tokens of each octet before the odd ones), so that lane order is the k
   // order of the V products.
   const int tok = KIND == 0 ? lane : (lane & 16) | (((lane >> 3) & 1) << 3) | ((lane & 3) << 1) | ((lane >> 2) & 1);
-  const int tl = 32 * warp + tok;  // this lane's token within a stage
+  // two independent groups of 32 tokens per warp and stage: tokens tl and tl + 32
+  constexpr int ST = 32 * TG * kCW;
+  const int tl = 32 * TG * warp + tok;  // this lane's first token within a stage
   const uint32_t sel1 = (lane & 1) ? 0x3715u : 0x6240u;
   const uint32_t sel2 = (lane & 2) ? 0x3276u : 0x5410u;
   const float fterm = gid == 0 ? 1.0f : gid == 1 ? kInv254 : gid == 2 ? kInv254sq : gid == 3 ? kInv254cu : 0.0f;
@@ -602,79 +625,108 @@ LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
     }
   };
 
-  int tl_end = len - s0 * kStageT - tl;  // token (s0 + j) * kStageT + tl is valid iff j * kStageT < tl_end
+  int tl_end = len - s0 * ST - tl;  // token (s0 + j) * ST + tl is valid iff j * ST < tl_end
   for (int j = 0; j < s1 - s0; ++j) {
-    if (!waited && (s0 + j + 1) * kStageT > p.stable_len) {  // past the stable prefix: the append's output
+    if (!waited && (s0 + j + 1) * ST > p.stable_len) {  // past the stable prefix: the append's output
       lk_grid_dep_wait();
       waited = true;
       len = unit_len(p, b);
-      tl_end = len - s0 * kStageT - tl;
+      tl_end = len - s0 * ST - tl;
     }
-    if ((s0 + j) * kStageT >= len) break;  // no copies were issued for the unit's later stages
+    if ((s0 + j) * ST >= len) break;  // no copies were issued for the unit's later stages
     if (*B.abort_flag) break;
     if (!lk_mbar_wait_bounded(&B.full[buf], phase, LK_WAIT_LIMIT_NS)) *B.abort_flag = 1;
     if (*B.abort_flag) break;
     const uint8_t* st = smem + buf * L.stage_bytes;
     const uint8_t* vs = st + L.off_vs;
-    const bool valid = j * kStageT < tl_end;
-    // a. score; a new running max (warp vote) folds the open sums
-    float s = -INFINITY;
-    if (valid) s = token_score<KIND, CSK>(st + L.off_kc, st + L.off_ks, g, tl, qterm, qa);
-    if (__any_sync(0xffffffffu, s > m_run)) {
-      const float m_new = fmaxf(m_run, lk_warp_max(s));
+    const bool va = j * ST < tl_end, vb = TG == 2 && j * ST + 32 < tl_end;
+    // a. scores of the token groups; a new running max (warp vote) folds the open sums
+    float sa, sb = -INFINITY;
+    token_score2<KIND, CSK, TG>(st + L.off_kc, st + L.off_ks, g, tl, qterm, qa, sa, sb);
+    sa = va ? sa : -INFINITY;
+    sb = vb ? sb : -INFINITY;
+    const float smx = fmaxf(sa, sb);
+    if (__any_sync(0xffffffffu, smx > m_run)) {
+      const float m_new = fmaxf(m_run, lk_warp_max(smx));
       const float alpha = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - m_new);
       fold(alpha);
       l_run *= alpha;
       m_run = m_new;
     }
-    const float pr = valid ? exp2f(s - m_run) : 0.0f;
-    l_run += pr;
+    const float pa = va ? exp2f(sa - m_run) : 0.0f;
+    const float pb = vb ? exp2f(sb - m_run) : 0.0f;
+    l_run += pa + pb;
     // b. V scales: a larger one (warp vote) folds, then raises wref; the
     //    weights w = p sigma_V become four int8 terms of w * 127 / wref
-    const uint8_t* vc = st + L.off_vc + 2 * warp * 16 * g.rbv;  // the warp's two 16-token blocks
-    const uint8_t* vc1 = vc + 16 * g.rbv;
+    const uint8_t* vca = st + L.off_vc + 2 * TG * warp * 16 * g.rbv;  // the warp's 16-token blocks
+    const uint8_t* vca1 = vca + 16 * g.rbv;
+    const uint8_t* vcb = vca + 32 * g.rbv;
+    const uint8_t* vcb1 = vca + 48 * g.rbv;
     if (VG1) {
-      const float sg = valid ? load_scale(vs, tl, KIND) : 0.0f;
-      if (__any_sync(0xffffffffu, sg > wref)) {  // then some sg > 0, so wref > 0 below
+      const float ga = va ? load_scale(vs, tl, KIND) : 0.0f;
+      const float gb = TG == 2 && vb ? load_scale(vs, tl + 32, KIND) : 0.0f;
+      if (__any_sync(0xffffffffu, fmaxf(ga, gb) > wref)) {  // then some scale > 0, so wref > 0 below
         fold(1.0f);
-        wref = fmaxf(wref, lk_warp_max(sg));
+        wref = fmaxf(wref, lk_warp_max(fmaxf(ga, gb)));
         inv = 127.0f / wref;
       }
-      uint32_t a0, a2;
-      weight_frags(expand_weight(pr * sg * inv), sel1, sel2, gid, tig, a0, a2);
-      // c. acc[jm] += terms x codes of dims 8 jm .. 8 jm + 7 (dims >= r_V only
-      //    in the last product, when r_V % 8 != 0)
+      uint32_t a0a, a2a, a0b = 0u, a2b = 0u;
+      weight_frags(expand_weight(pa * ga * inv), sel1, sel2, gid, tig, a0a, a2a);
+      if constexpr (TG == 2) weight_frags(expand_weight(pb * gb * inv), sel1, sel2, gid, tig, a0b, a2b);
+      // c. acc[jm] += terms x codes of dims 8 jm .. 8 jm + 7, each group
+      //    (dims >= r_V only in the last product, when r_V % 8 != 0)
 #pragma unroll
       for (int jm = 0; jm < NM; ++jm) {
         const int d = 8 * jm + gid;
         const bool live = jm < NM - 1 || d < g.rv;
-        const uint32_t b0 = live ? v_frag<KIND>(vc, d, tig) : 0u;
-        const uint32_t b1 = live ? v_frag<KIND>(vc1, d, tig) : 0u;
-        mma_s8_rows8(a0, a2, b0, b1, acc[jm][0], acc[jm][1]);
+        const uint32_t b0 = live ? v_frag<KIND>(vca, d, tig) : 0u;
+        const uint32_t b1 = live ? v_frag<KIND>(vca1, d, tig) : 0u;
+        mma_s8_rows8(a0a, a2a, b0, b1, acc[jm][0], acc[jm][1]);
+        if constexpr (TG == 2) {
+          const uint32_t b2 = live ? v_frag<KIND>(vcb, d, tig) : 0u;
+          const uint32_t b3 = live ? v_frag<KIND>(vcb1, d, tig) : 0u;
+          mma_s8_rows8(a0b, a2b, b2, b3, acc[jm][0], acc[jm][1]);
+        }
       }
     } else {
       float smax_t = 0.0f;
-      for (int gi = 0; gi < g.ngv; ++gi) smax_t = fmaxf(smax_t, valid ? load_scale(vs, tl * g.ngv + gi, KIND) : 0.0f);
+      for (int gi = 0; gi < g.ngv; ++gi) {
+        smax_t = fmaxf(smax_t, va ? load_scale(vs, tl * g.ngv + gi, KIND) : 0.0f);
+        if (TG == 2) smax_t = fmaxf(smax_t, vb ? load_scale(vs, (tl + 32) * g.ngv + gi, KIND) : 0.0f);
+      }
       if (__any_sync(0xffffffffu, smax_t > wref)) {
         fold(1.0f);
         wref = fmaxf(wref, lk_warp_max(smax_t));
         inv = 127.0f / wref;
       }
       for (int gi = 0; gi < g.ngv; ++gi) {
-        const float sg = valid ? load_scale(vs, tl * g.ngv + gi, KIND) : 0.0f;
-        uint32_t a0, a2;
-        weight_frags(expand_weight(pr * sg * inv), sel1, sel2, gid, tig, a0, a2);
-        fr[gi * 32 + lane] = make_uint2(a0, a2);
+        const float ga = va ? load_scale(vs, tl * g.ngv + gi, KIND) : 0.0f;
+        uint32_t a0a, a2a;
+        weight_frags(expand_weight(pa * ga * inv), sel1, sel2, gid, tig, a0a, a2a);
+        fr[(gi * 2 + 0) * 32 + lane] = make_uint2(a0a, a2a);
+        if constexpr (TG == 2) {
+          const float gb = vb ? load_scale(vs, (tl + 32) * g.ngv + gi, KIND) : 0.0f;
+          uint32_t a0b, a2b;
+          weight_frags(expand_weight(pb * gb * inv), sel1, sel2, gid, tig, a0b, a2b);
+          fr[(gi * 2 + 1) * 32 + lane] = make_uint2(a0b, a2b);
+        }
       }
       __syncwarp();
 #pragma unroll
       for (int jm = 0; jm < NM; ++jm) {
-        const uint2 a = fr[((8 * jm) / g.gv) * 32 + lane];
+        const int gi = (8 * jm) / g.gv;
+        const uint2 fa = fr[(gi * 2 + 0) * 32 + lane];
         const int d = 8 * jm + gid;
         const bool live = jm < NM - 1 || d < g.rv;
-        const uint32_t b0 = live ? v_frag<KIND>(vc, d, tig) : 0u;
-        const uint32_t b1 = live ? v_frag<KIND>(vc1, d, tig) : 0u;
-        mma_s8_rows8(a.x, a.y, b0, b1, acc[jm][0], acc[jm][1]);
+        const uint32_t b0 = live ? v_frag<KIND>(vca, d, tig) : 0u;
+        const uint32_t b1 = live ? v_frag<KIND>(vca1, d, tig) : 0u;
+        mma_s8_rows8(fa.x, fa.y, b0, b1, acc[jm][0], acc[jm][1]);
+        if constexpr (TG == 2) {
+          const uint2 fb = fr[(gi * 2 + 1) * 32 + lane];
+          const uint32_t b2 = live ? v_frag<KIND>(vcb, d, tig) : 0u;
+          const uint32_t b3 = live ? v_frag<KIND>(vcb1, d, tig) : 0u;
+          mma_s8_rows8(fb.x, fb.y, b2, b3, acc[jm][0], acc[jm][1]);
+        }
       }
     }
     __syncwarp();  // this warp is done with the stage buffer (and its fragment store)
@@ -705,10 +757,10 @@ LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
   }
 }
 
-template <int KIND, int CSK, bool VG1>
+template <int KIND, int CSK, bool VG1, int TG>
 LK_DEVICE void run_unit_nm(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, const HeadGeom& g, int b,
                            int len, int s0, int s1, int& buf, uint32_t& phase, bool& waited) {
-#define LK_RUN(NMV) run_unit<KIND, CSK, NMV, VG1>(p, smem, L, g, b, len, s0, s1, buf, phase, waited)
+#define LK_RUN(NMV) run_unit<KIND, CSK, NMV, VG1, TG>(p, smem, L, g, b, len, s0, s1, buf, phase, waited)
   switch ((g.rv + 7) >> 3) {
     case 1: LK_RUN(1); break;
     case 2: LK_RUN(2); break;
@@ -850,7 +902,7 @@ LK_DEVICE void finish_unit(const DecodeParams& p, uint8_t* smem, const SmemLayou
   consumer_sync();
 }
 
-template <int KIND>
+template <int KIND, int TG>
 LK_DEVICE void consume(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, int i0, int i1, int c) {
   int u = i0 / p.S, s = i0 - u * p.S;
   int it = i0, n = 0, buf = 0;
@@ -866,13 +918,13 @@ LK_DEVICE void consume(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
     const int len = waited ? unit_len(p, b) : p.stable_len;
     const int csk = lk_chunk_bytes(g.rbk);
     if (KIND == 0 || g.ngv == 1) {
-      if (csk == 16) run_unit_nm<KIND, 16, true>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
-      else if (csk == 8) run_unit_nm<KIND, 8, true>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
-      else run_unit_nm<KIND, 4, true>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      if (csk == 16) run_unit_nm<KIND, 16, true, TG>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      else if (csk == 8) run_unit_nm<KIND, 8, true, TG>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      else run_unit_nm<KIND, 4, true, TG>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
     } else if constexpr (KIND == 1) {
-      if (csk == 16) run_unit_nm<KIND, 16, false>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
-      else if (csk == 8) run_unit_nm<KIND, 8, false>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
-      else run_unit_nm<KIND, 4, false>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      if (csk == 16) run_unit_nm<KIND, 16, false, TG>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      else if (csk == 8) run_unit_nm<KIND, 8, false, TG>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      else run_unit_nm<KIND, 4, false, TG>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
     }
     finish_unit<KIND>(p, smem, L, g, b, h, u, it, seg_end, i0, c, n);
     it = seg_end;
@@ -883,7 +935,7 @@ LK_DEVICE void consume(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
   if (!waited) lk_grid_dep_wait();  // this grid never completes before the previous one
 }
 
-template <int KIND>
+template <int KIND, int TG>
 __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const SmemLayout L = smem_layout(p);
@@ -913,7 +965,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const __grid_c
     if (threadIdx.x == kConsumerThreads) produce<KIND>(p, smem, L, i0, i1);
     return;
   }
-  consume<KIND>(p, smem, L, i0, i1, c);
+  consume<KIND, TG>(p, smem, L, i0, i1, c);
   if (threadIdx.x == 0 && *bars_of(smem, L).abort_flag) lk_dev_fail(LK_DEV_TIMEOUT_PIPE);
 }
 
@@ -926,34 +978,38 @@ namespace lk {
 namespace {
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
+using DecodeKernel = void (*)(DecodeParams);
+DecodeKernel decode_kernel(int kind, int tg) {
+  if (kind == 0) return tg == 2 ? decode_attn_kernel<0, 2> : decode_attn_kernel<0, 1>;
+  return tg == 2 ? decode_attn_kernel<1, 2> : decode_attn_kernel<1, 1>;
+}
+
 // Resident CTAs per SM of the decode kernel for `smem` bytes of shared memory
-// (cached per device, kind and size; the query costs a few microseconds).
-int decode_occupancy(int kind, int smem) {
+// (cached per device, kernel and size; the query costs a few microseconds).
+int decode_occupancy(int kind, int tg, int smem) {
   static std::mutex mu;
   static std::map<std::tuple<int, int, int>, int> cache;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 1;
-  const auto key = std::make_tuple(dev, kind, smem);
+  const auto key = std::make_tuple(dev, kind * 4 + tg, smem);
   std::lock_guard<std::mutex> lock(mu);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
   int occ = 0;
-  cudaError_t e = kind == 0
-                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_attn_kernel<0>, kThreads, smem)
-                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_attn_kernel<1>, kThreads, smem);
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel(kind, tg), kThreads, smem);
   if (e != cudaSuccess || occ < 1) occ = 1;
   cache[key] = occ;
   return occ;
 }
-int decode_stages(int max_len) { return std::max(1, (max_len + kStageT - 1) / kStageT); }
+int decode_stages(int max_len, int st = kStageMin) { return std::max(1, (max_len + st - 1) / st); }
 // CTAs of the split (never more than items).  n_split > 0 asks for about
 // n_split pieces per (b, h) unit.  Automatic (n_split = 0), `cap` = CTAs that
 // fit on the GPU at once: with fewer units than that, each unit is cut into
 // the same number k = cap / units of pieces, so that no CTA straddles two
 // units (a straddling CTA pays a second q absorption and its pieces a merge);
 // with more units, `cap` CTAs share all items evenly (stream-K).
-int64_t decode_ctas(int units, int max_len, int n_split, int64_t cap) {
-  const int64_t W = (int64_t)units * decode_stages(max_len);
+int64_t decode_ctas(int units, int max_len, int n_split, int64_t cap, int st = kStageMin) {
+  const int64_t W = (int64_t)units * decode_stages(max_len, st);
   if (n_split > 0) return std::min(W, (int64_t)units * n_split);
   if (units >= cap) return std::min(W, cap);
   return std::min(W, (int64_t)units * (cap / units));
@@ -1030,42 +1086,49 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   const int rbk_max = a.kind == 0 ? rk_max : rk_max / 2;
   const int rbv_max = a.kind == 0 ? rv_max : rv_max / 2;
   const int ssz = a.kind == 0 ? 4 : 2;
-  p.st_kc = round_up(kStageT * rbk_max, 128);
-  p.st_vc = round_up(kStageT * rbv_max, 128);
-  p.st_ks = round_up(kStageT * ngk_max * ssz, 128);
-  p.st_vs = round_up(kStageT * ngv_max * ssz, 128);
   p.q_size = a.q_bf16 ? 2 : 4;
   p.b_size = a.b_bf16 ? 2 : 4;
   p.st_q = round_up(a.head_dim * p.q_size, 128);
   p.st_bk = round_up(rk_max * a.head_dim * p.b_size, 128);
   p.st_bv = round_up(rv_max * a.head_dim * p.b_size, 128);
-  p.st_fr = ngv_max > 1 ? kCW * ngv_max * 32 * 8 : 0;  // per-warp V fragments of each scale group
-  // as many stages as fit while two CTAs share an SM (about 64 KB of copies in
-  // flight per SM keeps HBM busy), between 2 and kMaxStages
-  {
+  // two token groups per warp (448-token stages: more independent work per
+  // warp) when two such stages of the widest head fit in ~110 KB beside the
+  // fixed regions, so that two CTAs still share an SM; else one (224 tokens)
+  int tg = 2;
+  for (;; tg = 1) {
+    p.ST = 32 * tg * kCW;
+    p.st_kc = round_up(p.ST * rbk_max, 128);
+    p.st_vc = round_up(p.ST * rbv_max, 128);
+    p.st_ks = round_up(p.ST * ngk_max * ssz, 128);
+    p.st_vs = round_up(p.ST * ngv_max * ssz, 128);
+    p.st_fr = ngv_max > 1 ? kCW * ngv_max * 2 * 32 * 8 : 0;  // per-warp V fragments: scale group x token group
     p.nstages = 0;
     const int stage = p.st_kc + p.st_vc + p.st_ks + p.st_vs;
     const int room = 110 * 1024 - smem_bytes_for(p);  // smem_bytes_for counts 0 stages here
-    p.nstages = std::max(2, std::min(kMaxStages, room / std::max(stage, 1)));
+    if (tg == 1 || room >= 2 * stage) {
+      // as many stages as fit (about 64 KB of copies in flight per SM keeps
+      // HBM busy), between 2 and kMaxStages
+      p.nstages = std::max(2, std::min(kMaxStages, room / std::max(stage, 1)));
+      break;
+    }
   }
   const int units = a.batch * a.n_heads;
-  p.S = decode_stages(a.max_len);
+  p.S = decode_stages(a.max_len, p.ST);
   const int64_t W = (int64_t)units * p.S;
   // a ring deeper than the stages a CTA streams only costs shared memory (and
   // keeps the kernel off SMs the previous kernel still occupies): size it for
   // the grid a full GPU would take
   {
-    const int64_t g_full = decode_ctas(units, a.max_len, a.n_split, std::min(2 * a.num_sms, kAutoCtaBound));
+    const int64_t g_full = decode_ctas(units, a.max_len, a.n_split, std::min(2 * a.num_sms, kAutoCtaBound), p.ST);
     const int64_t per_cta = (W + g_full - 1) / std::max<int64_t>(1, g_full) + 1;
     p.nstages = (int)std::max<int64_t>(2, std::min<int64_t>(p.nstages, per_cta));
   }
   const int smem = smem_bytes_for(p);
-  cudaError_t e = a.kind == 0
-                      ? cudaFuncSetAttribute(decode_attn_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
-                      : cudaFuncSetAttribute(decode_attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const DecodeKernel kernel = decode_kernel(a.kind, tg);
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int resident = decode_occupancy(a.kind, smem) * a.num_sms;
-  const int64_t G = decode_ctas(units, a.max_len, a.n_split, std::min(resident, kAutoCtaBound));
+  const int resident = decode_occupancy(a.kind, tg, smem) * a.num_sms;
+  const int64_t G = decode_ctas(units, a.max_len, a.n_split, std::min(resident, kAutoCtaBound), p.ST);
   if (W > INT32_MAX || G < 1) return cudaErrorInvalidValue;
   p.W = (int)W;
   p.G = (int)G;
@@ -1087,7 +1150,7 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = a.kind == 0 ? cudaLaunchKernelEx(&cfg, decode_attn_kernel<0>, p) : cudaLaunchKernelEx(&cfg, decode_attn_kernel<1>, p);
+  e = cudaLaunchKernelEx(&cfg, kernel, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
