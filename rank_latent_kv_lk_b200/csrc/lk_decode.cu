@@ -183,10 +183,22 @@ struct Chunk<4> {
   }
 };
 
+// A non-negative finite fp16 value as fp32, exactly, without a conversion
+// instruction: its bits shifted into fp32 position read as the value times
+// 2^-112 (normal or subnormal alike), so one multiply by 2^112 restores it.
+LK_DEVICE float f16_nonneg_to_f32(uint32_t h) { return __uint_as_float(h << 13) * 0x1p112f; }
+
 LK_DEVICE float load_scale(const uint8_t* base, int i, int kind) {
   return kind == 0 ? reinterpret_cast<const float*>(base)[i]
-                   : lk_f16_to_f32(reinterpret_cast<const uint16_t*>(base)[i]);
+                   : f16_nonneg_to_f32(reinterpret_cast<const uint16_t*>(base)[i]);
 }
+
+// Exact int -> float for |a| < 2^22 on the integer and FMA pipes: a added to
+// the bit pattern of 1.5 * 2^23 is that float plus a, so one subtraction
+// leaves a.  (The conversion instruction shares the pipe with exp2.)
+constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr int kMagicBits = 0x4B400000;
+LK_DEVICE float i2f_small(int a) { return __fsub_rn(__int_as_float(a + kMagicBits), kMagic); }
 
 LK_DEVICE float ld_f(const uint8_t* base, int i, int is_bf16) {
   return is_bf16 ? lk_bf16_to_f32(reinterpret_cast<const uint16_t*>(base)[i])
@@ -213,17 +225,23 @@ constexpr float kInv254cu = 1.0f / (254.0f * 254.0f * 254.0f);
 // Four int8 terms t_i of x in [0, 127]: x = t0 + t1/254 + t2/254^2 + t3/254^3
 // up to 127/254^4 (each remainder lies in [-1/2, 1/2], so |t_i| <= 127),
 // packed little-endian into one word (byte i = t_i).
+// Each rounding is x + 1.5 * 2^23 (round half to even, |x| < 2^22): the sum's
+// low byte is already the two's-complement int8 of the rounded value, and
+// subtracting the constant again gives it as a float.  No conversion
+// instruction is needed (those share a pipe with exp2).
+// (Explicitly rounded operations: a product contracted into the rounding
+// add would round the exact product instead of the stored one.)
 LK_DEVICE uint32_t expand_weight(float x) {
   x = fminf(x, 127.0f);
-  const float t0 = rintf(x);
-  x = (x - t0) * 254.0f;
-  const float t1 = rintf(x);
-  x = (x - t1) * 254.0f;
-  const float t2 = rintf(x);
-  x = (x - t2) * 254.0f;
-  const float t3 = rintf(x);
-  const uint32_t lo = __byte_perm((uint32_t)(int)t0, (uint32_t)(int)t1, 0x0040u);
-  const uint32_t hi = __byte_perm((uint32_t)(int)t2, (uint32_t)(int)t3, 0x0040u);
+  const float m0 = __fadd_rn(x, kMagic);
+  x = __fmul_rn(__fsub_rn(x, __fsub_rn(m0, kMagic)), 254.0f);
+  const float m1 = __fadd_rn(x, kMagic);
+  x = __fmul_rn(__fsub_rn(x, __fsub_rn(m1, kMagic)), 254.0f);
+  const float m2 = __fadd_rn(x, kMagic);
+  x = __fmul_rn(__fsub_rn(x, __fsub_rn(m2, kMagic)), 254.0f);
+  const float m3 = __fadd_rn(x, kMagic);
+  const uint32_t lo = __byte_perm(__float_as_uint(m0), __float_as_uint(m1), 0x0040u);
+  const uint32_t hi = __byte_perm(__float_as_uint(m2), __float_as_uint(m3), 0x0040u);
   return __byte_perm(lo, hi, 0x5410u);
 }
 
@@ -322,8 +340,9 @@ LK_DEVICE void token_score2(const uint8_t* kc, const uint8_t* ks, const HeadGeom
         }
       }
     }
-    const float xa = fmaf((float)a2, kInv254sq, fmaf((float)a1, kInv254, (float)a0));
-    const float xb = fmaf((float)b2, kInv254sq, fmaf((float)b1, kInv254, (float)b0));
+    // |a_i| <= 64 * 127 * 127 < 2^22
+    const float xa = fmaf(i2f_small(a2), kInv254sq, fmaf(i2f_small(a1), kInv254, i2f_small(a0)));
+    const float xb = fmaf(i2f_small(b2), kInv254sq, fmaf(i2f_small(b1), kInv254, i2f_small(b0)));
     sa = reinterpret_cast<const float*>(ks)[tl] * (qa * xa);
     if constexpr (TG == 2) sb = reinterpret_cast<const float*>(ks)[tb] * (qa * xb);
   } else {
@@ -348,10 +367,10 @@ LK_DEVICE void token_score2(const uint8_t* kc, const uint8_t* ks, const HeadGeom
         for (int wi = 0; wi < WPC; ++wi) {
           if (wleft == 0) {  // flush the finished group (uniform branch)
             const float sg_a = load_scale(ks, tl * g.ngk + cur_g, 1);
-            s_a = fmaf(sg_a, qa * fmaf((float)a2, kInv254sq, fmaf((float)a1, kInv254, (float)a0)), s_a);
+            s_a = fmaf(sg_a, qa * fmaf(i2f_small(a2), kInv254sq, fmaf(i2f_small(a1), kInv254, i2f_small(a0))), s_a);
             if constexpr (TG == 2) {
               const float sg_b = load_scale(ks, tb * g.ngk + cur_g, 1);
-              s_b = fmaf(sg_b, qa * fmaf((float)b2, kInv254sq, fmaf((float)b1, kInv254, (float)b0)), s_b);
+              s_b = fmaf(sg_b, qa * fmaf(i2f_small(b2), kInv254sq, fmaf(i2f_small(b1), kInv254, i2f_small(b0))), s_b);
             }
             a0 = a1 = a2 = b0 = b1 = b2 = 0;
             ++cur_g;
@@ -370,9 +389,12 @@ LK_DEVICE void token_score2(const uint8_t* kc, const uint8_t* ks, const HeadGeom
         }
       }
     }
-    sa = fmaf(load_scale(ks, tl * g.ngk + cur_g, 1), qa * fmaf((float)a2, kInv254sq, fmaf((float)a1, kInv254, (float)a0)), s_a);
+    // per group |a_i| <= 64 * 7 * 127 < 2^22
+    sa = fmaf(load_scale(ks, tl * g.ngk + cur_g, 1),
+              qa * fmaf(i2f_small(a2), kInv254sq, fmaf(i2f_small(a1), kInv254, i2f_small(a0))), s_a);
     if constexpr (TG == 2)
-      sb = fmaf(load_scale(ks, tb * g.ngk + cur_g, 1), qa * fmaf((float)b2, kInv254sq, fmaf((float)b1, kInv254, (float)b0)), s_b);
+      sb = fmaf(load_scale(ks, tb * g.ngk + cur_g, 1),
+                qa * fmaf(i2f_small(b2), kInv254sq, fmaf(i2f_small(b1), kInv254, i2f_small(b0))), s_b);
   }
 }
 
@@ -626,7 +648,10 @@ LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
   };
 
   int tl_end = len - s0 * ST - tl;  // token (s0 + j) * ST + tl is valid iff j * ST < tl_end
-  for (int j = 0; j < s1 - s0; ++j) {
+  // after an expired wait (error path) later units skip their stages; within
+  // a unit the flag is consulted only when a wait expires
+  const int nst = *B.abort_flag ? 0 : s1 - s0;
+  for (int j = 0; j < nst; ++j) {
     if (!waited && (s0 + j + 1) * ST > p.stable_len) {  // past the stable prefix: the append's output
       lk_grid_dep_wait();
       waited = true;
@@ -634,9 +659,10 @@ LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
       tl_end = len - s0 * ST - tl;
     }
     if ((s0 + j) * ST >= len) break;  // no copies were issued for the unit's later stages
-    if (*B.abort_flag) break;
-    if (!lk_mbar_wait_bounded(&B.full[buf], phase, LK_WAIT_LIMIT_NS)) *B.abort_flag = 1;
-    if (*B.abort_flag) break;
+    if (!lk_mbar_wait_bounded(&B.full[buf], phase, LK_WAIT_LIMIT_NS)) {
+      *B.abort_flag = 1;
+      break;
+    }
     const uint8_t* st = smem + buf * L.stage_bytes;
     const uint8_t* vs = st + L.off_vs;
     const bool va = j * ST < tl_end, vb = TG == 2 && j * ST + 32 < tl_end;
