@@ -28,8 +28,6 @@ cudaError_t launch_gemm_f(const void* A, int lda, const void* B, int ldb, float*
 namespace {
 
 constexpr int kGemvThreads = 256;
-constexpr int kColsPerWarp = 4;
-constexpr int kColsPerCta = kColsPerWarp * (kGemvThreads / 32);  // 32
 constexpr int kGemvMaxRows = 8;  // more rows: the tensor-core GEMM, then the quantise-and-append pass
 
 template <int XT> struct XTraits;
@@ -469,7 +467,6 @@ int cluster_slice(int E, int xtype) {
   return round_up((E + kClusterE - 1) / kClusterE, ve);
 }
 
-int x_ve(int xtype) { return xtype == lk::X_F32 ? 4 : (xtype == lk::X_BF16 ? 8 : 16); }
 int x_size(int xtype) { return xtype == lk::X_F32 ? 4 : (xtype == lk::X_BF16 ? 2 : 1); }
 
 constexpr int kPrefillRowChunk = 8192;
