@@ -213,25 +213,34 @@ class DecodeState:
         return self.A.numel() * self.A.element_size() + w.batch * w.embed_dim * 2 + codes
 
 
-def kernel_source_hash():
+# sources each profiled kernel is built from (its traffic figure stays valid
+# while these are unchanged)
+KERNEL_SOURCES = {
+    "decode_attn_kernel": ["lk_decode.cu", "lk_common.cuh", "lk_internal.h"],
+    "proj_cluster_kernel": ["lk_project.cu", "lk_common.cuh", "lk_quant.cuh", "lk_internal.h"],
+}
+
+
+def kernel_source_hash(kernel):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "rank_latent_kv_lk_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    with open(os.path.join(ROOT, "include", "lk.h"), "rb") as f:
+        h.update(b"lk.h" + f.read())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(kernel, workload):
-    """DRAM bytes per launch from a committed ncu capture, if the kernels have not changed since."""
+    """DRAM bytes per launch from a committed ncu capture, if the kernel's sources have not changed since."""
     try:
         with open(PROFILE_TRAFFIC) as f:
             for line in f:
                 parts = line.split()
                 if not parts or parts[0].startswith("#"):
                     continue
-                if parts[0] == f"{kernel}@{workload}" and parts[2] == kernel_source_hash():
+                if parts[0] == f"{kernel}@{workload}" and parts[2] == kernel_source_hash(kernel):
                     return int(parts[1])
     except OSError:
         pass
