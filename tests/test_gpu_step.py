@@ -1,8 +1,10 @@
 """The decode step entry point (append, then attention launched so that it
 overlaps the append's tail) against the two calls made one after the other,
-on identical caches: same appended codes and scales, same seq_len, same
-output bits -- for one and several rows, ragged lengths and ranks, int4
-caches and int8 (W8A8) inputs."""
+on identical caches: same appended codes and scales, same seq_len, and the
+same output within the fp32 parity bound (1e-5 of the output RMS; the step
+may split the attention over a different grid, which changes only the
+rounding of the merge) -- for one and several rows, ragged lengths and
+ranks, int4 caches and int8 (W8A8) inputs."""
 import dataclasses
 import math
 
@@ -13,6 +15,11 @@ from rank_latent_kv_lk_b200 import synth
 from rank_latent_kv_lk_b200.configs import WORKLOADS
 
 pytestmark = pytest.mark.gpu
+
+
+def _same_output(out1, out2):
+    rms = float(out2.double().pow(2).mean().sqrt())
+    return float((out1 - out2).abs().max()) <= 1e-5 * rms
 
 
 def _state(lk, w, ctx, device, shorten, extra=32):
@@ -35,6 +42,7 @@ def _state(lk, w, ctx, device, shorten, extra=32):
 CASES = [
     # (workload, batch, context, per-row shortening)
     (2, 1, 700, [0]),                                   # bf16, one row
+    (2, 1, 4096, [0]),                                  # full context: the step's grid differs
     (1, 1, 256, [0]),                                   # fp32 activations and factors
     (4, 8, 300, [0, 17, 5, 40, 1, 0, 33, 16]),          # ragged ranks and lengths, 8 rows
     (3, 4, 500, [3, 0, 11, 7]),                         # int4 groups of 24, 4 rows
@@ -65,7 +73,7 @@ def test_step_matches_separate_calls(wl, batch, ctx, shorten):
         assert seq.tolist() == seq2.tolist() == lens
         assert torch.equal(ck.codes, ck2.codes) and torch.equal(cv.codes, cv2.codes)
         assert torch.equal(ck.scales, ck2.scales) and torch.equal(cv.scales, cv2.scales)
-        assert torch.equal(out1, out2), f"step {step}: outputs differ"
+        assert _same_output(out1, out2), f"step {step}: outputs differ"
         assert torch.isfinite(out1).all() and float(out1.abs().max()) > 0
 
 
@@ -108,7 +116,7 @@ def test_step_w8a8_inputs_match_separate_calls():
         assert seq.tolist() == seq2.tolist() == lens
         assert torch.equal(ck.codes, ck2.codes) and torch.equal(cv.codes, cv2.codes)
         assert torch.equal(ck.scales, ck2.scales) and torch.equal(cv.scales, cv2.scales)
-        assert torch.equal(out1, out2)
+        assert _same_output(out1, out2)
         assert math.isfinite(float(out1.abs().max()))
 
 
@@ -133,7 +141,7 @@ def test_step_many_calls_leave_workspace_clean():
             torch.cuda.synchronize()
             lk.device_status()
             assert a[2].tolist() == b[2].tolist() == lens
-            assert torch.equal(out1, out2)
+            assert _same_output(out1, out2)
             assert torch.equal(a[0].codes, b[0].codes) and torch.equal(a[1].codes, b[1].codes)
     ws = lk.api.workspaces.get("project", 0, dev)
     assert int(ws[:256].count_nonzero()) == 0
