@@ -120,3 +120,53 @@ def test_layer_full_size():
     """B=32, E=4096, 32 heads x 128, r=32, context 4096, hybrid FFN 11008 (25% dense, rank 512)."""
     w = configs.WORKLOADS[5]
     run_layer(w, T_ctx=w.context, seed=32)
+
+
+def _layer_state(w, T_ctx, seed):
+    rk, rv = [w.rank] * w.n_heads, [w.rank] * w.n_heads
+    wts = synth.layer_weights_w8a8(w, rk, rv)
+    capacity = (T_ctx + 1 + 15) // 16 * 16
+    layer = W8A8DecoderLayer(wts, w.n_heads, w.head_dim, rk, rv, w.batch, capacity, w.ffn_inter)
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    for c in (layer.cache_k, layer.cache_v):
+        c.codes.copy_(torch.randint(0, 256, c.codes.shape, dtype=torch.uint8, device="cuda", generator=g))
+        c.scales.copy_(torch.rand(c.scales.shape, device="cuda", generator=g) * 0.02 + 0.01)
+    return layer
+
+
+@pytest.mark.parametrize("batch,T_ctx", [(4, 40), (32, 4096)])
+def test_layer_step_replayed_from_a_cuda_graph(batch, T_ctx):
+    """One layer step captured in a CUDA graph and replayed (as bench.py
+    --layer times it) writes what the eager step writes: the same output
+    bits, the same appended latents and the same seq_len, on every replay."""
+    w = configs.WORKLOADS[5]
+    if batch != w.batch:
+        w = dataclasses.replace(w, batch=batch, embed_dim=256, n_heads=4, head_dim=64, rank=16, ffn_inter=512,
+                                ffn_rank=64)
+    eager, graphed = _layer_state(w, T_ctx, 41), _layer_state(w, T_ctx, 41)
+    x = torch.randn(w.batch, w.embed_dim, generator=torch.Generator().manual_seed(42)).to(torch.bfloat16).cuda()
+    seq_e = torch.full((w.batch,), T_ctx, dtype=torch.int32, device="cuda")
+    out_e = eager.step(x, seq_e, [T_ctx] * w.batch).clone()
+    seq_g = torch.full((w.batch,), T_ctx, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):  # warm-up: workspaces allocated outside the capture
+        graphed.step(x, seq_g, [T_ctx] * w.batch)
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    seq_g.fill_(T_ctx)
+    with torch.cuda.graph(graph):
+        out_g = graphed.step(x, seq_g, [T_ctx] * w.batch)
+    for _ in range(3):
+        seq_g.fill_(T_ctx)
+        graph.replay()
+        torch.cuda.synchronize()
+        _lk().device_status()
+        assert seq_g.tolist() == seq_e.tolist() == [T_ctx + 1] * w.batch
+        assert torch.equal(out_g, out_e)
+        assert torch.equal(graphed.cache_k.codes, eager.cache_k.codes)
+        assert torch.equal(graphed.cache_v.codes, eager.cache_v.codes)
+        assert torch.equal(graphed.cache_k.scales, eager.cache_k.scales)
+    del graph
