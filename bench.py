@@ -19,6 +19,7 @@ host cores, same workload and metric.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -55,6 +56,9 @@ def parse_args(argv=None):
     ap.add_argument("--attn-only", action="store_true",
                     help="time the latent decode attention alone on one layer of the workload, "
                          "its cache filled with seeded random codes (no prefill)")
+    ap.add_argument("--dense-compare", action="store_true",
+                    help="time one layer's latent attention against dense bf16 attention over materialised "
+                         "K/V of the same shapes (library SDPA), workloads 2-5")
     return ap.parse_args(argv)
 
 
@@ -686,6 +690,74 @@ def run_layer(args):
     return 0
 
 
+def run_dense_compare(args):
+    """Context for the pages' decode speedups (measured against flash decoding
+    over dense K/V): per workload, one layer's latent attention against dense
+    bf16 attention over materialised K and V of the same shapes
+    ([B, heads, T, H], PyTorch scaled_dot_product_attention -- a library
+    comparator, not part of this path).  L2 flushed before every launch."""
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    import rank_latent_kv_lk_b200 as lk
+    from rank_latent_kv_lk_b200 import synth
+    from rank_latent_kv_lk_b200.configs import WORKLOADS
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+        torch.cuda._sleep(int(5e7))
+        for e in ev:
+            flush.fill_(1)
+            e[0].record()
+            fn()
+            e[1].record()
+        torch.cuda.synchronize()
+        return statistics.median(e[0].elapsed_time(e[1]) * 1e3 for e in ev)
+
+    lines = []
+    for key in (2, 3, 4, 5):
+        w = WORKLOADS[key]
+        rk, rv = synth.ranks(w)
+        rk, rv = rk[0], rv[0]
+        _, BK, BV = synth.factors(dataclasses.replace(w, act="bf16"), 0, rk, rv)
+        BK, BV = BK.to(device), BV.to(device)
+        T = w.context + 1
+        g = torch.Generator(device=device)
+        g.manual_seed(synth.seed_for(w, synth.CONTEXT))
+        ck = lk.LatentCache(w.batch, rk, w.capacity, w.kind, w.group, device)
+        cv = lk.LatentCache(w.batch, rv, w.capacity, w.kind, w.group, device, role="v")
+        for c in (ck, cv):
+            c.codes.copy_(torch.randint(0, 256, c.codes.shape, dtype=torch.uint8, device=device, generator=g))
+            c.scales.copy_((torch.rand(c.scales.shape, device=device, generator=g) * 0.02 + 0.01).to(c.scales.dtype))
+        q = torch.randn(w.batch, w.n_heads, w.head_dim, generator=g, device=device).to(torch.bfloat16)
+        seq = torch.full((w.batch,), T, dtype=torch.int32, device=device)
+        out = torch.empty(w.batch, w.n_heads, w.head_dim, dtype=torch.bfloat16, device=device)
+        latent_us = timed(lambda: lk.latent_decode_attn(ck, cv, q, BK, BV, seq, T, out=out), args.steps)
+        del ck, cv
+        K = torch.randn(w.batch, w.n_heads, T, w.head_dim, generator=g, device=device).to(torch.bfloat16)
+        V = torch.randn(w.batch, w.n_heads, T, w.head_dim, generator=g, device=device).to(torch.bfloat16)
+        q4 = q.unsqueeze(2)
+        dense_us = timed(lambda: torch.nn.functional.scaled_dot_product_attention(q4, K, V), args.steps)
+        dense_bytes = 2 * K.numel() * K.element_size()
+        del K, V
+        torch.cuda.empty_cache()
+        lines.append({"workload": w.name, "layer": 0, "batch": w.batch, "tokens": T,
+                      "latent_attn_us": latent_us, "dense_sdpa_us": dense_us,
+                      "dense_kv_bytes": dense_bytes, "dense_gbs": dense_bytes / (dense_us * 1e-6) / 1e9,
+                      "speedup_vs_dense": dense_us / latent_us})
+    if rank == 0:
+        print(json.dumps({"mode": "dense-compare", "steps": args.steps,
+                          "note": "dense side: torch scaled_dot_product_attention over bf16 K/V of the same "
+                                  "shapes (library kernel), the pages' flash-decoding comparison point",
+                          "l2": "flushed before every launch (256 MiB write, untimed)",
+                          "results": lines}), flush=True)
+    return 0
+
+
 def _finish(world):
     if world > 1 and torch.distributed.is_initialized():
         torch.distributed.destroy_process_group()
@@ -701,6 +773,8 @@ def main(argv=None):
         return run_attn_only(args)
     if args.layer:
         return run_layer(args)
+    if args.dense_compare:
+        return run_dense_compare(args)
     return run_ours(args)
 
 
