@@ -56,6 +56,9 @@ def parse_args(argv=None):
     ap.add_argument("--attn-only", action="store_true",
                     help="time the latent decode attention alone on one layer of the workload, "
                          "its cache filled with seeded random codes (no prefill)")
+    ap.add_argument("--all-layers", action="store_true",
+                    help="time one decode step across every layer of a multi-layer workload "
+                         "(--workload 4: 32 layers), caches filled with seeded random codes")
     ap.add_argument("--dense-compare", action="store_true",
                     help="time one layer's latent attention against dense bf16 attention over materialised "
                          "K/V of the same shapes (library SDPA), workloads 2-5")
@@ -690,6 +693,98 @@ def run_layer(args):
     return 0
 
 
+def run_all_layers(args):
+    """One decode step across every layer of a multi-layer workload (workload
+    4: 32 layers, ragged ranks, B = 8, T = 16384 + 1): per layer, the new
+    token's latent projection, quantisation and append, then the latent
+    attention, through lk_latent_decode_step.  The caches hold seeded random
+    codes (no prefill); x and q per layer are seeded draws.  The working set
+    (10.7 GB of latents and factors) is far larger than L2, so no flush is
+    needed; every timed step starts from the same context (seq_len reset,
+    untimed)."""
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    import rank_latent_kv_lk_b200 as lk
+    from rank_latent_kv_lk_b200 import synth
+    from rank_latent_kv_lk_b200.configs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    rks, rvs = synth.ranks(w)
+    g = torch.Generator(device=device)
+    g.manual_seed(synth.seed_for(w, synth.CONTEXT))
+    layers = []
+    for l in range(w.n_layers):
+        A, BK, BV = synth.factors(w, l, rks[l], rvs[l])
+        ck = lk.LatentCache(w.batch, rks[l], w.capacity, w.kind, w.group, device)
+        cv = lk.LatentCache(w.batch, rvs[l], w.capacity, w.kind, w.group, device, role="v")
+        for c in (ck, cv):
+            c.codes.copy_(torch.randint(0, 256, c.codes.shape, dtype=torch.uint8, device=device, generator=g))
+            c.scales.copy_((torch.rand(c.scales.shape, device=device, generator=g) * 0.02 + 0.01).to(c.scales.dtype))
+        x = torch.randn(w.batch, w.embed_dim, generator=g, device=device).to(A.dtype)
+        q = torch.randn(w.batch, w.n_heads, w.head_dim, generator=g, device=device).to(A.dtype)
+        out = torch.empty(w.batch, w.n_heads, w.head_dim, dtype=A.dtype, device=device)
+        seq = torch.full((w.batch,), w.context, dtype=torch.int32, device=device)
+        layers.append((ck, cv, A.to(device), BK.to(device), BV.to(device), x, q, out, seq))
+    lens0 = [w.context] * w.batch
+
+    def step():
+        for ck, cv, A, BK, BV, x, q, out, seq in layers:
+            lk.latent_decode_step(ck, cv, x, A, seq, lens0, q, BK, BV, out=out)
+
+    def reset():
+        for layer in layers:
+            layer[8].fill_(w.context)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+        reset()
+    torch.cuda.synchronize()
+    K = args.steps
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(2e8))
+    with ClockSampler(local) as clocks:
+        for i in range(K):
+            reset()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    lk.device_status()
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), world, device)
+    us = total_ms / K * 1e3
+    T = w.context + 1
+    rb = lambda r: r if w.kind == "i8" else r // 2
+    sb = lambda r: 4 if w.kind == "i8" else 2 * (-(-r // min(w.group, r)))
+    nbytes = 0
+    for l in range(w.n_layers):
+        per_tok = sum(rb(r) + sb(r) for r in rks[l]) + sum(rb(r) + sb(r) for r in rvs[l])
+        n_tot = sum(rks[l]) + sum(rvs[l])
+        nbytes += w.batch * T * per_tok + n_tot * w.embed_dim * 2 + n_tot * w.head_dim * 2
+    gbs = nbytes / (us * 1e-6) / 1e9
+    hbm, peak_kind = peaks()
+    if rank == 0:
+        print(json.dumps({
+            "mode": "all-layers", "metric": "decode tokens/s (one step across all layers)",
+            "value": w.batch * world / (us * 1e-6), "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "us_per_step": us, "higher_is_better": True, "scaling": "weak",
+            "dtype": "int8/f32" if w.kind == "i8" else "int4/f32",
+            "data": "synthetic (seeded random latent codes and scales, seeded factors, x and q)",
+            "config": {"workload": w.name, "layers": w.n_layers, "batch": w.batch, "tokens": T,
+                       "l2": "not flushed: the working set is far larger than L2",
+                       "launches": f"{2 * w.n_layers} per step (projection + attention per layer)"},
+            "algorithmic_bytes_per_step": nbytes,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "peak_kind": peak_kind},
+            "gpu_launches": 2 * w.n_layers * K, "clocks": clocks.summary()}), flush=True)
+    _finish(world)
+    return 0
+
+
 def run_dense_compare(args):
     """Context for the pages' decode speedups (measured against flash decoding
     over dense K/V): per workload, one layer's latent attention against dense
@@ -775,6 +870,8 @@ def main(argv=None):
         return run_layer(args)
     if args.dense_compare:
         return run_dense_compare(args)
+    if args.all_layers:
+        return run_all_layers(args)
     return run_ours(args)
 
 
