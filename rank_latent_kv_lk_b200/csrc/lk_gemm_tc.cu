@@ -25,11 +25,14 @@
 namespace {
 
 constexpr int kBM = 128, kBN = 128, kBK = 64;
-constexpr int kStages = 4;
+constexpr int kStages = 4;    // int8 kernel ring depth
+// bf16 kernel: 3 stages (≈100 KB) so that two CTAs share an SM and one's
+// epilogue (TMEM -> global) overlaps the other's MMAs
+constexpr int kStagesBf = 3;
 constexpr int kTileBytes = kBM * kBK * 2;  // 16 KB; the B tile has the same size (kBN == kBM)
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 128;  // fp32 accumulator: 128 lanes x 128 columns
-constexpr int kSmemBytes = 2 * kStages * kTileBytes + 1024 /* barriers */ + 1024 /* alignment */;
+constexpr int kSmemBytes = 2 * kStagesBf * kTileBytes + 1024 /* barriers */ + 1024 /* alignment */;
 
 // Shared-memory matrix descriptor of a K-major tile with the 128-byte swizzle
 // (rows of 128 bytes, 8-row groups 1024 bytes apart): start address >> 4,
@@ -92,17 +95,17 @@ LK_DEVICE void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                         float* __restrict__ C, int ldc, int M, int N, int K) {
   extern __shared__ uint8_t smem_raw[];
   // the 128-byte swizzle repeats every 1024 bytes: tiles start 1024-aligned
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* tiles_a = smem;
-  uint8_t* tiles_b = smem + kStages * kTileBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + 2 * kStages * kTileBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* done = empty + kStages;
+  uint8_t* tiles_b = smem + kStagesBf * kTileBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + 2 * kStagesBf * kTileBytes);
+  uint64_t* empty = full + kStagesBf;
+  uint64_t* done = empty + kStagesBf;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -111,7 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nk = (K + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStagesBf; ++s) {
       lk_mbar_init(&full[s], 1);
       lk_mbar_init(&empty[s], 1);
     }
@@ -134,9 +137,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ================= producer: TMA loads of the A and B tiles
       int issued = 0;
       for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % kStages;
-        if (kb >= kStages &&
-            !lk_mbar_wait_bounded(&empty[s], (uint32_t)(((kb / kStages) - 1) & 1), LK_WAIT_LIMIT_NS)) {
+        const int s = kb % kStagesBf;
+        if (kb >= kStagesBf &&
+            !lk_mbar_wait_bounded(&empty[s], (uint32_t)(((kb / kStagesBf) - 1) & 1), LK_WAIT_LIMIT_NS)) {
           *abort_flag = 1;
           break;
         }
@@ -147,16 +150,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued = kb + 1;
       }
       // every load this CTA started has landed before it may finish
-      for (int kb = max(0, issued - kStages); kb < issued; ++kb)
-        if (!lk_mbar_wait_bounded(&full[kb % kStages], (uint32_t)((kb / kStages) & 1), LK_WAIT_LIMIT_NS))
+      for (int kb = max(0, issued - kStagesBf); kb < issued; ++kb)
+        if (!lk_mbar_wait_bounded(&full[kb % kStagesBf], (uint32_t)((kb / kStagesBf) & 1), LK_WAIT_LIMIT_NS))
           lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ================= MMA issue: the accumulator lives in TMEM
       for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % kStages;
-        if (!lk_mbar_wait_bounded(&full[s], (uint32_t)((kb / kStages) & 1), LK_WAIT_LIMIT_NS)) *abort_flag = 1;
+        const int s = kb % kStagesBf;
+        if (!lk_mbar_wait_bounded(&full[s], (uint32_t)((kb / kStagesBf) & 1), LK_WAIT_LIMIT_NS)) *abort_flag = 1;
         if (*abort_flag) break;
         tc_fence_after();
         const uint64_t adesc = sw128_desc(lk_smem_addr(tiles_a + s * kTileBytes));
