@@ -180,12 +180,15 @@ LK_DEVICE void append_values(const FinalizeParams& p, int grow, int j, float v0,
   }
 }
 
-// Prefill epilogue: one warp per (row, head); the last CTA advances seq_len.
+// Prefill epilogue: a warp per (row, head) item, the warps striding over all
+// items (a grid of a few CTAs per SM, so that the closing ticket below is a
+// few thousand atomics on one word, not one per 4 items); the last CTA
+// advances seq_len.
 __global__ void __launch_bounds__(128) proj_finalize_kernel(const __grid_constant__ FinalizeParams p) {
   lk_grid_dep_launch();  // a decode launched next may start its set-up now
   const int n_heads_tot = p.k.n_heads + p.v.n_heads;
-  const int64_t item = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
-  if (item < (int64_t)p.rows * n_heads_tot) {
+  const int64_t items = (int64_t)p.rows * n_heads_tot;
+  for (int64_t item = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5); item < items; item += (int64_t)gridDim.x * 4) {
     const int lrow = (int)(item / n_heads_tot);
     append_head(p, lrow, p.row0 + lrow, (int)(item % n_heads_tot));
   }
@@ -619,7 +622,8 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
     f.rows = nr;
     f.do_update = (r0 + nr == rows);
     const int64_t items = (int64_t)nr * heads_tot;
-    proj_finalize_kernel<<<(unsigned)((items + 3) / 4), 128, 0, stream>>>(f);
+    const int64_t grid = std::min<int64_t>((items + 3) / 4, (int64_t)std::max(1, a.num_sms) * 16);
+    proj_finalize_kernel<<<(unsigned)grid, 128, 0, stream>>>(f);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
