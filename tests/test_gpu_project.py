@@ -118,11 +118,13 @@ def test_ragged_ranks_append():
     assert h.check() <= 40
 
 
-@pytest.mark.parametrize("B", [1, 8, 9, 32])
+@pytest.mark.parametrize("B", [1, 8, 9, 16, 32, 64, 65])
 def test_decode_rows_gemv(B):
     w = configs.WORKLOADS[2]
     h = _float_case(w, B, 1, 1, [32] * 32, [32] * 32, seed=15 + B)
-    assert h.check() <= 20
+    # codes off by one only inside the rounding band (check() raises
+    # otherwise); their count grows with the rows: about 20 per 32 rows
+    assert h.check() <= 20 * max(1, -(-B // 32))
 
 
 def _w8a8_case(B, n_prefill, n_decode, seed):
