@@ -52,7 +52,7 @@ typedef enum {
   LK_ERR_DTYPE = 3,       /* dtype not supported for this argument          */
   LK_ERR_ALIGN = 4,       /* pointer or size not aligned as required        */
   LK_ERR_CAPACITY = 5,    /* append would overrun the cache capacity        */
-  LK_ERR_UNSUPPORTED = 6, /* valid request this build does not implement    */
+  LK_ERR_UNSUPPORTED = 6, /* valid request the library does not implement   */
   LK_ERR_WORKSPACE = 7,   /* workspace null or smaller than required        */
   LK_ERR_CUDA = 8,        /* a CUDA call failed (text in lk_last_error)     */
   LK_ERR_DEVICE = 9       /* a kernel reported a bounded wait that expired  */
