@@ -35,6 +35,16 @@ MUTANTS = {
  "svd_no_sigma": ("return U[:, :r] * sig[None, :r], Vt[:r, :]", "return U[:, :r], Vt[:r, :]"),
  "w8a8_sa_order": ("* np.asarray(a_scale, np.float16).astype(np.float32)[None, :]).astype(np.float32)\n    return v", "* np.asarray(a_scale, np.float16).astype(np.float32)[::-1][None, :]).astype(np.float32)\n    return v"),
  "i4_group_index": ("idx = np.arange(r) // group", "idx = np.arange(r) % (-(-r // group))"),
+ "layer_swiglu_swap": ("act = swiglu(gate, upv).astype(np.float32)", "act = swiglu(upv, gate).astype(np.float32)"),
+ "layer_ffn_fed_h1": ("h2 = rmsnorm(x2, eps).astype(np.float32)", "h2 = h1"),
+ "layer_attn_quant_before_store": (
+     "attn = round_bf16(attn.reshape(Bsz, n_h * H))\n    aq, sa = quantize_rows_i8(attn.astype(np.float32))",
+     "aq, sa = quantize_rows_i8(attn.reshape(Bsz, n_h * H).astype(np.float32))\n"
+     "    attn = round_bf16(attn.reshape(Bsz, n_h * H))"),
+ "layer_no_attn_residual": ("layer[\"s_O\"], residual=x))", "layer[\"s_O\"], residual=None))"),
+ "layer_ffn_residual_x": ("d[\"s_V\"], residual=x2)", "d[\"s_V\"], residual=x)"),
+ "layer_q_from_x": ("q = round_bf16(_linear_dense_w8a8(xq, sx, layer[\"W_Q\"], layer[\"s_Q\"]))",
+                    "q = round_bf16(_linear_dense_w8a8(*quantize_rows_i8(x.astype(np.float32)), layer[\"W_Q\"], layer[\"s_Q\"]))"),
 }
 
 

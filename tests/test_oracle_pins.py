@@ -453,3 +453,50 @@ def test_decoder_layer_zero_branches_is_identity():
     np.testing.assert_array_equal(out, x)
     assert ck.length(0) == 1 and cv.length(1) == 1
     assert np.all(np.abs(inter["attn"]) > 0)
+
+
+def test_decoder_layer_tiny_worked():
+    """A whole layer step on a hand-worked example (tests/golden/decoder_layer_tiny.json).
+
+    E = 4, one head with H = 2 and r_K = r_V = 1, one cached token, a 2-channel
+    hybrid FFN.  Every stored intermediate is compared exactly (int8 codes,
+    float32 scales, bf16 tensors); the float64 layer output to 1e-12 relative.
+    The values fix which tensor feeds which stage: SwiGLU(gate, up) and not
+    (up, gate), the FFN fed RMSNorm(x2) and not h1, the attention output
+    stored as bf16 before it is quantised, both residuals."""
+    gj = _gold("decoder_layer_tiny.json")
+    inp, exp = gj["inputs"], gj["expected"]
+    f16 = lambda a: np.asarray(a, np.float16)
+    i8 = lambda a: np.asarray(a, np.int8)
+
+    def hyb(w):
+        return dict(dense_idx=np.asarray(w["dense_idx"]), lr_idx=np.asarray(w["lr_idx"]), W_D=i8(w["W_D"]),
+                    s_D=f16(w["s_D"]), U=i8(w["U"]), s_U=f16(w["s_U"]), V=i8(w["V"]), s_V=f16(w["s_V"]))
+
+    layer = dict(n_heads=1, head_dim=2, ranks_k=[1], ranks_v=[1],
+                 W_Q=i8(inp["W_Q"]), s_Q=f16(inp["s_Q"]), W_O=i8(inp["W_O"]), s_O=f16(inp["s_O"]),
+                 A=i8(inp["A"]), s_A=f16(inp["s_A"]),
+                 B_K=[np.asarray(inp["B_K"], np.float64)], B_V=[np.asarray(inp["B_V"], np.float64)],
+                 gate=hyb(inp["gate"]), up=hyb(inp["up"]), down=hyb(inp["down"]))
+    ck, cv = O.LatentCache(1, [1], "i8", 32), O.LatentCache(1, [1], "i8", 32)
+    tok = inp["cached_token"]
+    ck.append(0, [(i8([[tok["k_code"]]]), np.asarray([tok["k_scale"]], np.float32))])
+    cv.append(0, [(i8([[tok["v_code"]]]), np.asarray([tok["v_scale"]], np.float32))])
+    out, inter = O.decoder_layer_w8a8(np.asarray(inp["x"], np.float64), layer, ck, cv, eps=0.0)
+
+    hx = lambda a: np.vectorize(float.fromhex)(np.asarray(a, dtype=object)).astype(np.float64)
+    for key in ("xq", "aq", "hq", "mq"):
+        np.testing.assert_array_equal(np.asarray(inter[key], np.int64), np.asarray(exp[key], np.int64), err_msg=key)
+    for key in ("sx", "sa", "sh", "sm"):
+        got = np.asarray(inter[key], np.float32)
+        np.testing.assert_array_equal(got.view(np.uint32), hx(exp[key]).astype(np.float32).view(np.uint32),
+                                      err_msg=key)
+    np.testing.assert_array_equal(np.asarray(inter["q"], np.float64), np.asarray(exp["q"], np.float64))
+    for key in ("latent", "attn", "x2", "gate", "up"):
+        np.testing.assert_array_equal(np.asarray(inter[key], np.float64), hx(exp[key]), err_msg=key)
+    np.testing.assert_allclose(out, hx(exp["out"]), rtol=1e-12, atol=0)
+    # the new token was appended behind the cached one with the quantiser's codes and scales
+    assert ck.length(0) == 2 and cv.length(0) == 2
+    for cache, (code, scale) in ((ck, exp["k_new"]), (cv, exp["v_new"])):
+        assert int(cache.codes[0][0][1, 0]) == code
+        assert np.float32(cache.scales[0][0][1]).view(np.uint32) == np.float32(float.fromhex(scale)).view(np.uint32)
