@@ -215,8 +215,11 @@ size_t lk_latent_decode_workspace_bytes(const lk_latent_cache* k_cache,
  *  - All calls share the one array: calls that overlap on the GPU (other
  *    streams, other host threads) race on it.  Serialise them.
  *  - The arrival counters in the array start at zero when the library loads
- *    and every completed call leaves them zero; a call whose B * n_heads
- *    differs from the device's previous call first clears them on `stream`.
+ *    and every completed call leaves them zero.  A call first clears them on
+ *    `stream` when its B * n_heads differs from the device's last accepted
+ *    call, when the last call failed, and always while `stream` is being
+ *    captured (a replay may follow direct calls of any shape).  A rejected
+ *    call launches nothing and leaves the array as it was.
  */
 #define LK_DECODE_NOALLOC_SCRATCH_BYTES (4u << 20)
 lk_status lk_latent_decode_attn_noalloc(const lk_latent_cache* k_cache, const lk_latent_cache* v_cache,
@@ -323,6 +326,12 @@ lk_status lk_device_status(int32_t reset);
 const char* lk_status_string(lk_status status);
 const char* lk_last_error(void);
 int32_t lk_version(void);
+
+/* Number of kernels this library has enqueued in this process so far, over
+ * all devices, streams and host threads (memsets not counted).  The
+ * difference across a region of calls is how many of the library's kernels
+ * that region launched (no counterpart on the pages: instrumentation). */
+uint64_t lk_kernel_launches(void);
 
 #ifdef __cplusplus
 }

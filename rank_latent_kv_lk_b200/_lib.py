@@ -79,6 +79,7 @@ def _load():
     WP = C.POINTER(LowrankWeightDesc)
     sig = {
         "lk_version": (I32, []),
+        "lk_kernel_launches": (C.c_uint64, []),
         "lk_last_error": (C.c_char_p, []),
         "lk_status_string": (C.c_char_p, [C.c_int]),
         "lk_latent_cache_bytes": (C.c_int, [CP, C.POINTER(SZ), C.POINTER(SZ)]),

@@ -230,3 +230,8 @@ def swiglu_quant_i8(gate, up, stream=None):
 def device_status(reset=True):
     """Synchronise and raise if a kernel reported an expired bounded wait."""
     check(lib.lk_device_status(1 if reset else 0))
+
+
+def kernel_launches():
+    """Kernels the library has enqueued in this process so far (lk_kernel_launches)."""
+    return int(lib.lk_kernel_launches())

@@ -4,7 +4,17 @@
 #include <cstdio>
 #include <cstring>
 
+#include <atomic>
+
 #include "lk_internal.h"
+
+namespace lk {
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}
+void count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+unsigned long long launches_value() { return g_launches.load(std::memory_order_relaxed); }
+}  // namespace lk
 
 cudaError_t lk_quant_status_word(unsigned int* value, int reset);
 cudaError_t lk_project_status_word(unsigned int* value, int reset);
@@ -90,6 +100,8 @@ lk_status set_error(lk_status s, const char* msg) {
 extern "C" {
 
 int32_t lk_version(void) { return 1; }
+
+uint64_t lk_kernel_launches(void) { return lk::launches_value(); }
 
 const char* lk_last_error(void) { return g_last_error; }
 

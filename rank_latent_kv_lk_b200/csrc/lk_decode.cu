@@ -1186,6 +1186,7 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, kernel, p);
   if (e != cudaSuccess) return e;
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -1230,40 +1231,48 @@ extern "C" lk_status lk_latent_decode_attn_noalloc(const lk_latent_cache* k, con
     snprintf(msg, sizeof(msg), "lk_latent_decode_attn_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
     return lk::set_error(LK_ERR_CUDA, msg);
   }
-  void* scratch = nullptr;
-  bool clear = false;
-  const int units = k->batch * k->n_heads;
-  {
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-      // once per device, with that device current
-      void* p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_decode_noalloc_scratch);
-      if (e != cudaSuccess || !p) {
-        snprintf(msg, sizeof(msg), "lk_latent_decode_attn_noalloc: cudaGetSymbolAddress: %s",
-                 cudaGetErrorString(e));
-        return lk::set_error(LK_ERR_CUDA, msg);
-      }
-      g_noalloc_ptr[dev] = p;
-    }
-    scratch = g_noalloc_ptr[dev];
-    // the partials of a call with another B * n_heads may cover this call's
-    // counters: clear them first (every completed call leaves them zero)
-    clear = g_noalloc_units[dev] != units;
-    g_noalloc_units[dev] = units;
-  }
   int rv_max = 0;
   for (int h = 0; h < v->n_heads; ++h) rv_max = std::max(rv_max, (int)v->ranks[h]);
-  const size_t need = lk::decode_workspace_bytes(k->batch * k->n_heads, rv_max, max_seq_len, n_split);
+  const int units = k->batch * k->n_heads;
+  const size_t need = lk::decode_workspace_bytes(units, rv_max, max_seq_len, n_split);
   if (need > LK_DECODE_NOALLOC_SCRATCH_BYTES) {
+    // rejected before any state changes: the next call sees the array as the
+    // last accepted call left it
     snprintf(msg, sizeof(msg),
              "lk_latent_decode_attn_noalloc: needs %zu bytes of scratch, the static array holds %u; "
              "lower n_split or use lk_latent_decode_attn with a workspace",
              need, (unsigned)LK_DECODE_NOALLOC_SCRATCH_BYTES);
     return lk::set_error(LK_ERR_WORKSPACE, msg);
   }
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(cs, &capture);
+  if (e != cudaSuccess) {
+    snprintf(msg, sizeof(msg), "lk_latent_decode_attn_noalloc: cudaStreamIsCapturing: %s", cudaGetErrorString(e));
+    return lk::set_error(LK_ERR_CUDA, msg);
+  }
+  // One lock over the whole call: the recorded shape must describe what the
+  // stream will find in the array, so no other host thread may interleave.
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    // once per device, with that device current
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+      snprintf(msg, sizeof(msg), "lk_latent_decode_attn_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+      return lk::set_error(LK_ERR_CUDA, msg);
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  void* scratch = g_noalloc_ptr[dev];
+  // The partials of a call with another B * n_heads may cover this call's
+  // arrival counters: clear them first (every completed call leaves its own
+  // counters zero).  While the stream is being captured the clear is always
+  // recorded, because a replay may follow direct calls of any shape.
+  const bool clear = g_noalloc_units[dev] != units || capture != cudaStreamCaptureStatusNone;
+  g_noalloc_units[dev] = 0;  // unknown until this call has been enqueued
   if (clear) {
-    e = cudaMemsetAsync(scratch, 0, (size_t)(units * 4 + 255) / 256 * 256, reinterpret_cast<cudaStream_t>(stream));
+    e = cudaMemsetAsync(scratch, 0, (size_t)(units * 4 + 255) / 256 * 256, cs);
     if (e != cudaSuccess) {
       snprintf(msg, sizeof(msg), "lk_latent_decode_attn_noalloc: clearing counters: %s", cudaGetErrorString(e));
       return lk::set_error(LK_ERR_CUDA, msg);
@@ -1272,6 +1281,7 @@ extern "C" lk_status lk_latent_decode_attn_noalloc(const lk_latent_cache* k, con
   const lk_status st = lk_latent_decode_attn(k, v, q, q_dtype, B_K, B_V, b_dtype, head_dim, seq_len, max_seq_len,
                                              softmax_scale, out, out_dtype, n_split, scratch,
                                              LK_DECODE_NOALLOC_SCRATCH_BYTES, stream);
-  if (st != LK_OK) return st;
+  if (st != LK_OK) return st;  // the recorded shape stays 0: the next call clears
+  g_noalloc_units[dev] = units;
   return LK_OK;
 }

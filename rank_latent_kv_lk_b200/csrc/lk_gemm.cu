@@ -106,6 +106,7 @@ cudaError_t launch_gemm_f(const void* A, int lda, const void* B, int ldb, float*
   dim3 grid((N + kBN - 1) / kBN, (M + kBM - 1) / kBM);
   if (bf16) gemm_f_kernel<true><<<grid, kThreads, 0, stream>>>(A, lda, B, ldb, C, ldc, M, N, K);
   else gemm_f_kernel<false><<<grid, kThreads, 0, stream>>>(A, lda, B, ldb, C, ldc, M, N, K);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -388,6 +388,7 @@ cudaError_t launch_gemm_bf16_tc(const void* A, int lda, const void* B, int ldb, 
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + kBM - 1) / kBM));
   gemm_bf16_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(map_a, map_b, C, ldc, M, N, K);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -399,6 +400,7 @@ cudaError_t launch_i8_nt(const CUtensorMap& mw, const CUtensorMap& mx, int32_t* 
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)((N + 127) / 128), (unsigned)((M + NT - 1) / NT), (unsigned)splits);
   gemm_i8_tc_kernel<NT><<<grid, kThreads, smem, stream>>>(mw, mx, C, ldc, M, N, K, kbps);
+  count_launch();
   return cudaGetLastError();
 }
 

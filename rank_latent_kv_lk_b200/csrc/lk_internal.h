@@ -12,6 +12,10 @@
 
 namespace lk {
 
+// Kernels this library has launched in the process (every launch site calls
+// count_launch once per kernel it enqueues; read through lk_kernel_launches).
+void count_launch(unsigned n = 1);
+
 // ---------------------------------------------------------------- decode
 struct DecodeLaunch {
   const void* codes_k;

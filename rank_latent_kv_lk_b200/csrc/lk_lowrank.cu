@@ -123,6 +123,7 @@ cudaError_t launch_lowrank_linear(const LowrankLaunch& a, cudaStream_t stream) {
     int8_t* xd = reinterpret_cast<int8_t*>(ws + L.xd);
     const int ld = pad16(a.n_dense);
     gather_cols_kernel<<<dim3((ld + 255) / 256, a.m), 256, 0, stream>>>(a.x_q, a.k_in, a.dense_idx, a.n_dense, ld, xd);
+    count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     accD = reinterpret_cast<int32_t*>(ws + L.accD);
     e = launch_gemm_i8(xd, ld, a.W_D, a.n_dense, accD, a.n_out, a.m, a.n_out, a.n_dense, stream);
@@ -132,11 +133,13 @@ cudaError_t launch_lowrank_linear(const LowrankLaunch& a, cudaStream_t stream) {
     int8_t* xg = reinterpret_cast<int8_t*>(ws + L.xg);
     const int ld = pad16(n_lr);
     gather_cols_kernel<<<dim3((ld + 255) / 256, a.m), 256, 0, stream>>>(a.x_q, a.k_in, a.lr_idx, n_lr, ld, xg);
+    count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     int32_t* accU = reinterpret_cast<int32_t*>(ws + L.accU);
     e = launch_gemm_i8(xg, ld, a.U, n_lr, accU, a.rank, a.m, a.rank, n_lr, stream);
     if (e != cudaSuccess) return e;
     requant_kernel<<<a.m, 256, 0, stream>>>(accU, a.rank, a.x_scale, a.s_U, t_q, ld_tq, s_t);
+    count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     accV = reinterpret_cast<int32_t*>(ws + L.accV);
     e = launch_gemm_i8(t_q, ld_tq, a.V, a.rank, accV, a.n_out, a.m, a.n_out, a.rank, stream);
@@ -145,6 +148,7 @@ cudaError_t launch_lowrank_linear(const LowrankLaunch& a, cudaStream_t stream) {
   const dim3 egrid((unsigned)std::min((a.n_out + 255) / 256, 64), (unsigned)a.m);
   lowrank_epilogue_kernel<<<egrid, 256, 0, stream>>>(accD, accV, a.x_scale, s_t, a.s_D, a.s_V, a.residual, a.m,
                                                      a.n_out, a.y, a.y_bf16);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -573,6 +573,7 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
                              (int)smem);                                                             \
     if (e != cudaSuccess) return e;                                                                   \
     e = cudaLaunchKernelEx(&cfg, proj_cluster_kernel<XTV, MTV, STV>, d);                             \
+    if (e == cudaSuccess) count_launch();                                                             \
   } while (0)
 #define LK_PROJ_LAUNCH(XTV, MTV)                         \
   do {                                                   \
@@ -624,6 +625,7 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
     const int64_t items = (int64_t)nr * heads_tot;
     const int64_t grid = std::min<int64_t>((items + 3) / 4, (int64_t)std::max(1, a.num_sms) * 16);
     proj_finalize_kernel<<<(unsigned)grid, 128, 0, stream>>>(f);
+    count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;

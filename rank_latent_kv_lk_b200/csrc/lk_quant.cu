@@ -135,6 +135,7 @@ cudaError_t launch_quantize_latent(const float* v, int m, int r, int kind, int g
                                    void* scales, cudaStream_t stream) {
   if (m == 0) return cudaSuccess;
   const int warps = 4;
+  count_launch();
   quantize_latent_kernel<<<(m + warps - 1) / warps, warps * 32, 0, stream>>>(
       v, m, r, kind, group, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales));
   return cudaGetLastError();
@@ -148,10 +149,12 @@ cudaError_t launch_rowquant(int mode, const void* x, const void* x2, int x_bf16,
   if (x_bf16) {
     e = cudaFuncSetAttribute(rowquant_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    count_launch();
     rowquant_kernel<true><<<m, kRowThreads, smem, stream>>>(mode, x, x2, k, eps, x_q, x_scale);
   } else {
     e = cudaFuncSetAttribute(rowquant_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    count_launch();
     rowquant_kernel<false><<<m, kRowThreads, smem, stream>>>(mode, x, x2, k, eps, x_q, x_scale);
   }
   return cudaGetLastError();
