@@ -1,20 +1,22 @@
 #!/usr/bin/env python3
 """Decode-step benchmark of the per-head latent-KV path on B200.
 
-One step = one autoregressive decode step of the attention layer of the
-LLaVA-7B-like workload (E=4096, 32 heads x H=128, rank 32 int8 latents, batch 1,
-4096-token context, 128 decode steps): latent projection + quantise + append
-of the new token and latent flash-decode attention, through
-lk_latent_decode_step (the two kernels, the attention launch overlapping the
-append).  Inputs are resident in HBM before timing; L2 is
-flushed (a 256 MiB write) before every step; each step is timed with CUDA
+Default line: one autoregressive decode step of the LASER-style ragged-rank
+workload across all of its layers (32 layers x 32 heads x H = 128, ranks
+r_h in {8, 16, 32, 48, 64} per (layer, head), K and V drawn independently,
+int8 latents, batch 8, 16384 cached tokens + the new one): per layer the new
+token's latent projection + quantise + append and the latent flash-decode
+attention, through lk_latent_decode_step.  The 10.7 GB working set lives in
+HBM before timing and is far larger than L2.  Each step is timed with CUDA
 events on the launching stream, the max over ranks is taken, and rank 0
 prints one JSON line.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 2]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 4]
 
---impl reference times the CPU oracle (float64, K and V materialised) on the
-host cores, same workload and metric.
+--workload 1..3 time the single-layer appending workloads instead (L2
+flushed before every step); --impl reference times the CPU oracle (float64,
+K and V materialised) on the host cores, same workload and metric, on a
+bounded sample of each step.
 """
 from __future__ import annotations
 
@@ -44,10 +46,10 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.txt")
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--workload", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--layer", action="store_true",
@@ -57,8 +59,9 @@ def parse_args(argv=None):
                     help="time the latent decode attention alone on one layer of the workload, "
                          "its cache filled with seeded random codes (no prefill)")
     ap.add_argument("--all-layers", action="store_true",
-                    help="time one decode step across every layer of a multi-layer workload "
-                         "(--workload 4: 32 layers), caches filled with seeded random codes")
+                    help="kept for old command lines: multi-layer workloads always time every layer")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the extra single-layer B = 1 measurement in the default line")
     ap.add_argument("--dense-compare", action="store_true",
                     help="time one layer's latent attention against dense bf16 attention over materialised "
                          "K/V of the same shapes (library SDPA), workloads 2-5")
@@ -106,13 +109,15 @@ _REASONS = {
 class ClockSampler:
     """Samples SM clock and throttle reasons every few ms while running (read-only NVML)."""
 
-    def __init__(self, device_index, period_s=0.005):
+    def __init__(self, device_index, period_s=0.005, enabled=True):
         self.period = period_s
         self.samples = []
         self.reasons = 0
         self.max_mhz = None
         self._stop = threading.Event()
         self._h = None
+        if not enabled:
+            return
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -265,8 +270,16 @@ def peaks():
 
 # ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
 
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 def oracle_session(w):
-    """Oracle state after the (untimed) context prefill; returns a step function."""
+    """Oracle state of a single-layer appending workload after its (untimed)
+    context prefill; returns a step function (one decode step of the workload)."""
     import oracle as O
     from rank_latent_kv_lk_b200 import synth
     rk, rv = synth.ranks(w)
@@ -299,16 +312,108 @@ def oracle_session(w):
     return step
 
 
-def blas_threads():
+class OracleLayerSample:
+    """Bounded samples of one decode step of a multi-layer workload for the CPU
+    oracle.  A full step (every layer, every (b, h) over T tokens, K and V
+    materialised in float64) takes the oracle many minutes, so a sample is one
+    (layer, b, h) unit: that layer's projection of the new tokens (its share
+    per unit), then the unit's quantise + append and its attention over the
+    cache, whose T - 1 context codes and scales are seeded random draws like
+    the device bench's.  A step's time is a unit's time times the units of
+    all layers."""
+
+    def __init__(self, w):
+        import oracle as O
+        from rank_latent_kv_lk_b200 import synth
+        self.O, self.w = O, w
+        self.rks, self.rvs = synth.ranks(w)
+        self.T = w.context + 1
+        self.units = w.n_layers * w.batch * w.n_heads
+        self._synth = synth
+        self._layer = None
+
+    def _load_layer(self, l):
+        if self._layer is not None and self._layer[0] == l:
+            return self._layer
+        w, synth = self.w, self._synth
+        A, BK, BV = synth.factors(w, l, self.rks[l], self.rvs[l])
+        A64 = synth.as_numpy(A).T.astype(np.float64)
+        BK, BV = synth.as_numpy(BK).astype(np.float64), synth.as_numpy(BV).astype(np.float64)
+        x = synth.as_numpy(synth.decode_tokens(w, l)[0])
+        q = synth.as_numpy(synth.queries(w, l)[0])
+        self._layer = (l, A64, BK, BV, x, q)
+        return self._layer
+
+    def unit(self, i):
+        """Oracle work of unit i (cycling over (layer, b, h)).  Returns the
+        seconds the oracle took; drawing the unit's random context codes is
+        not timed."""
+        O, w = self.O, self.w
+        u = i % self.units
+        l, rest = divmod(u, w.batch * w.n_heads)
+        b, h = divmod(rest, w.n_heads)
+        l, A64, BK, BV, x, q = self._load_layer(l)
+        rk, rv = self.rks[l], self.rvs[l]
+        nk = sum(rk)
+        rng = np.random.default_rng(1000003 * (l + 1) + 1009 * b + h)
+        ck, cv = O.LatentCache(1, [rk[h]], w.kind, w.group), O.LatentCache(1, [rv[h]], w.kind, w.group)
+        ctx = []
+        for r in (rk[h], rv[h]):
+            codes = rng.integers(-127, 128, (self.T - 1, r), dtype=np.int64).astype(np.int8)
+            scales = (rng.random(self.T - 1) * 0.02 + 0.01).astype(np.float32)
+            ctx.append((codes, scales))
+        t0 = time.perf_counter()
+        ck.append(0, [ctx[0]])
+        cv.append(0, [ctx[1]])
+        # this unit's share of the layer's projection: the new token's latent of head h (K and V)
+        ok, ov = sum(rk[:h]), nk + sum(rv[:h])
+        vk = O.latent_project_float(x[b:b + 1], A64[:, ok:ok + rk[h]])
+        vv = O.latent_project_float(x[b:b + 1], A64[:, ov:ov + rv[h]])
+        ck.append(0, O.quantize_latents(vk, [rk[h]], w.kind, w.group))
+        cv.append(0, O.quantize_latents(vv, [rv[h]], w.kind, w.group))
+        offk, offv = sum(rk[:h]), sum(rv[:h])
+        O.latent_attention(q[b:b + 1, h:h + 1], ck, cv, [BK[offk:offk + rk[h]]],
+                           [BV[offv:offv + rv[h]]], 1.0 / math.sqrt(w.head_dim))
+        return time.perf_counter() - t0
+
+    def sample_text(self, n):
+        w = self.w
+        return (f"{n} (layer, b, h) units of the {w.n_layers}-layer step, each: its share of the layer's "
+                f"projection of the new token, quantise + append, and float64 attention with K and V "
+                f"materialised over {self.T} tokens (drawing the unit's random context codes untimed); "
+                f"step time = mean unit time x {self.units} units")
+
+
+def _timed_units(sample, budget_s, max_units=None):
+    """Oracle seconds over units until about budget_s of wall time has passed."""
+    t0 = time.perf_counter()
+    n, dt = 0, 0.0
+    while True:
+        dt += sample.unit(n)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s or (max_units and n >= max_units):
+            return n, dt
+
+
+def cpu_baseline(w, budget_s=12.0):
+    """The oracle on the host cores: all the cores this process may use, and one thread."""
+    cores = host_cores()
     try:
         import threadpoolctl
-        info = threadpoolctl.threadpool_info()
-        return max([i.get("num_threads", 1) for i in info] or [1])
-    except Exception:
-        return os.cpu_count() or 1
-
-
-def cpu_baseline(w, budget_s=15.0):
+    except ImportError:
+        threadpoolctl = None
+    if w.n_layers > 1:
+        sample = OracleLayerSample(w)
+        sample.unit(0)  # warm-up (first layer load)
+        n, dt = _timed_units(sample, budget_s)
+        value = w.batch / (dt / n * sample.units)
+        single = None
+        if threadpoolctl is not None:
+            with threadpoolctl.threadpool_limits(1):
+                n1, dt1 = _timed_units(sample, budget_s / 2)
+            single = w.batch / (dt1 / n1 * sample.units)
+        return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "single_thread_value": single, "sample": sample.sample_text(n)}
     step = oracle_session(w)
     t0 = time.perf_counter()
     step(0)
@@ -318,95 +423,317 @@ def cpu_baseline(w, budget_s=15.0):
     for i in range(1, n + 1):
         step(i)
     dt = time.perf_counter() - t0
-    return {"value": w.batch * n / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+    single = None
+    if threadpoolctl is not None:
+        with threadpoolctl.threadpool_limits(1):
+            t0 = time.perf_counter()
+            m = max(1, n // 2)
+            for i in range(n + 1, n + 1 + m):
+                step(i)
+            single = w.batch * m / (time.perf_counter() - t0)
+    return {"value": w.batch * n / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "single_thread_value": single,
             "sample": f"{n} decode steps of the workload after its context prefill (prefill untimed; "
                       f"float64, K and V materialised)"}
 
 
 # ---------------------------------------------------------------- arms
 
+def workload_dtype(w):
+    codes = "int8" if w.kind == "i8" else "int4"
+    acts = {"f32": "f32", "bf16": "bf16", "i8": "int8"}[w.act]
+    return f"{codes} latents, {acts} activations and factors, f32 accumulate"
+
+
+def workload_data(w):
+    if w.n_layers > 1:
+        return ("synthetic (seeded): random int8 latent codes and positive scales in every cache (no prefill), "
+                "factors A ~ N(0, 1/E) and B ~ N(0, 1/r) in bf16, x and q ~ N(0, 1) per layer")
+    extra = f", first {w.image_tokens} context tokens sigma {w.image_sigma}" if w.image_tokens else ""
+    if w.outlier_frac:
+        extra += f", {w.outlier_frac:.0%} of x channels x{w.outlier_scale:g}"
+    return f"synthetic (seeded): x ~ N(0, 1){extra}, prefilled through the library; q ~ N(0, 1) per step"
+
+
 def run_reference(args):
+    """The CPU oracle as the reference arm: same workload, metric and unit; each
+    step is a bounded sample of a decode step (a unit of it for multi-layer
+    workloads), its time scaled to the whole step."""
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
     from rank_latent_kv_lk_b200.configs import WORKLOADS
     w = WORKLOADS[args.workload]
-    step = oracle_session(w)
-    for i in range(args.warmup):
-        step(i)
-    t0 = time.perf_counter()
-    for i in range(args.warmup, args.warmup + args.steps):
-        step(i)
-    dt = time.perf_counter() - t0
-    value = w.batch * args.steps / dt
-    cores = blas_threads()
+    if w.n_layers > 1:
+        sample = OracleLayerSample(w)
+        for i in range(args.warmup):
+            sample.unit(i)
+        dt = sum(sample.unit(i) for i in range(args.warmup, args.warmup + args.steps))
+        step_s = dt / args.steps * sample.units
+        value = w.batch / step_s
+        text = sample.sample_text(args.steps) + f", after {args.warmup} warm-up units"
+        config = {"workload": w.name, "layers": w.n_layers, "batch": w.batch, "tokens": w.context + 1}
+    else:
+        step = oracle_session(w)
+        for i in range(args.warmup):
+            step(i)
+        t0 = time.perf_counter()
+        for i in range(args.warmup, args.warmup + args.steps):
+            step(i)
+        dt = time.perf_counter() - t0
+        step_s = dt / args.steps
+        value = w.batch / step_s
+        text = (f"{args.steps} timed oracle decode steps after {args.warmup} warm-up steps and an untimed "
+                "context prefill")
+        config = {"workload": w.name, "batch": w.batch, "context": w.context}
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic (seeded)",
-            "config": {"workload": w.name, "batch": w.batch, "context": w.context},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": f"{args.steps} timed oracle decode steps after {args.warmup} warm-up "
-                                       "steps and an untimed context prefill"},
+            "data": workload_data(w), "config": config,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+                             "sample": text},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
 def run_ours(args):
+    from rank_latent_kv_lk_b200.configs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if w.n_layers > 1:
+        return run_multilayer(args, w)
+    return run_single(args, w)
+
+
+class MultiLayerState:
+    """Device state of a multi-layer workload: per layer the K and V latent
+    caches (seeded random codes and positive scales: their contents do not
+    change the work), the factors, the new token x and the query q."""
+
+    def __init__(self, w, device):
+        import rank_latent_kv_lk_b200 as lk
+        from rank_latent_kv_lk_b200 import synth
+        self.lk, self.w = lk, w
+        self.rks, self.rvs = synth.ranks(w)
+        L = w.n_layers
+        g = torch.Generator(device=device)
+        g.manual_seed(synth.seed_for(w, synth.CONTEXT))
+        self.layers = []
+        for l in range(L):
+            A, BK, BV = synth.factors(w, l, self.rks[l], self.rvs[l])
+            ck = lk.LatentCache(w.batch, self.rks[l], w.capacity, w.kind, w.group, device)
+            cv = lk.LatentCache(w.batch, self.rvs[l], w.capacity, w.kind, w.group, device, role="v")
+            for c in (ck, cv):
+                c.codes.copy_(torch.randint(0, 256, c.codes.shape, dtype=torch.uint8, device=device, generator=g))
+                sc = torch.rand(c.scales.shape, device=device, generator=g) * 0.02 + 0.01
+                c.scales.copy_(sc.to(c.scales.dtype))
+            self.layers.append((ck, cv, A.to(device), BK.to(device), BV.to(device)))
+        self.x = torch.stack([synth.decode_tokens(w, l)[0] for l in range(L)]).to(device)   # [L, B, E]
+        self.q = torch.stack([synth.queries(w, l)[0] for l in range(L)]).to(device)         # [L, B, nh, H]
+        self.out = torch.empty(L, w.batch, w.n_heads, w.head_dim, dtype=self.q.dtype, device=device)
+        self.seq = torch.full((L, w.batch), w.context, dtype=torch.int32, device=device)
+        self.lens0 = [w.context] * w.batch
+        torch.cuda.synchronize()
+
+    def reset(self):
+        self.seq.fill_(self.w.context)
+
+    def step(self, x=None, q=None, out=None):
+        x = self.x if x is None else x
+        q = self.q if q is None else q
+        out = self.out if out is None else out
+        for l, (ck, cv, A, BK, BV) in enumerate(self.layers):
+            self.lk.latent_decode_step(ck, cv, x[l], A, self.seq[l], self.lens0, q[l], BK, BV, out=out[l])
+
+    def attn_bytes(self, l):
+        """Algorithmic bytes of one attention launch of layer l (cache of T tokens, factors, q, out)."""
+        w = self.w
+        T = w.context + 1
+        rb = lambda r: r if w.kind == "i8" else r // 2
+        sb = lambda r: 4 if w.kind == "i8" else 2 * (-(-r // min(w.group, r)))
+        per_tok = sum(rb(r) + sb(r) for r in self.rks[l]) + sum(rb(r) + sb(r) for r in self.rvs[l])
+        factors = (sum(self.rks[l]) + sum(self.rvs[l])) * w.head_dim * 2
+        return w.batch * T * per_tok + factors + 2 * w.batch * w.n_heads * w.head_dim * 2
+
+    def proj_bytes(self, l):
+        w = self.w
+        rb = lambda r: r if w.kind == "i8" else r // 2
+        n_tot = sum(self.rks[l]) + sum(self.rvs[l])
+        codes = w.batch * (sum(rb(r) for r in self.rks[l]) + sum(rb(r) for r in self.rvs[l]))
+        return n_tot * w.embed_dim * 2 + w.batch * w.embed_dim * 2 + codes
+
+
+def run_multilayer(args, w):
+    """The headline: one decode step across every layer of the workload."""
     rank, world, local = dist_env()
     if not torch.cuda.is_available():
         raise RuntimeError("bench.py needs a CUDA device")
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     init_dist(world, "nccl")
-    from rank_latent_kv_lk_b200.configs import WORKLOADS
-    w = WORKLOADS[args.workload]
+    st = MultiLayerState(w, device)
+    lk = st.lk
+    stream = torch.cuda.current_stream()
+    L = w.n_layers
+    for _ in range(max(3, args.warmup)):
+        st.step()
+        st.reset()
+    torch.cuda.synchronize()
+    lk.device_status()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(2e8))  # let the host queue run ahead of the device
+    n0 = lk.kernel_launches()
+    with ClockSampler(local) as clocks:
+        for i in range(K):
+            st.reset()
+            ev[i][0].record(stream)
+            st.step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    launches = lk.kernel_launches() - n0
+    barrier(world)
+    lk.device_status()
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), world, device)
+    value = w.batch * K * world / (total_ms / 1e3)
+
+    # per-kernel durations: a second pass with events between the two kernels
+    # of every layer (for the roofline; the events stop the overlap of the two)
+    KP = min(K, 10)
+    kev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(L)] for _ in range(KP)]
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(1e8))
+    for i in range(KP):
+        st.reset()
+        for l, (ck, cv, A, BK, BV) in enumerate(st.layers):
+            kev[i][l][0].record(stream)
+            lk.latent_project_append(ck, cv, st.x[l], A, st.seq[l], st.lens0)
+            kev[i][l][1].record(stream)
+            lk.latent_decode_attn(ck, cv, st.q[l], BK, BV, st.seq[l], w.context + 1, out=st.out[l])
+            kev[i][l][2].record(stream)
+    torch.cuda.synchronize()
+    attn_s = sum(kev[i][l][1].elapsed_time(kev[i][l][2]) for i in range(KP) for l in range(L)) / 1e3
+    proj_s = sum(kev[i][l][0].elapsed_time(kev[i][l][1]) for i in range(KP) for l in range(L)) / 1e3
+    attn_bytes = KP * sum(st.attn_bytes(l) for l in range(L))
+    proj_bytes = KP * sum(st.proj_bytes(l) for l in range(L))
+    attn_gbs = attn_bytes / attn_s / 1e9
+    proj_gbs = proj_bytes / proj_s / 1e9
+
+    # e2e: every layer's x and q copied host -> device from pinned memory and
+    # every layer's output copied back, inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        nx = st.x.numel() * st.x.element_size()
+        nq = st.q.numel() * st.q.element_size()
+        hbuf = torch.empty(nx + nq, dtype=torch.uint8).pin_memory()
+        hbuf[:nx].copy_(st.x.reshape(-1).view(torch.uint8).cpu())
+        hbuf[nx:].copy_(st.q.reshape(-1).view(torch.uint8).cpu())
+        dbuf = torch.empty(nx + nq, dtype=torch.uint8, device=device)
+        xd = dbuf[:nx].view(st.x.dtype).view(st.x.shape)
+        qd = dbuf[nx:].view(st.q.dtype).view(st.q.shape)
+        oh = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+        e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        barrier(world)
+        torch.cuda.synchronize()
+        torch.cuda._sleep(int(1e8))
+        for i in range(K):
+            st.reset()
+            e_ev[i][0].record(stream)
+            dbuf.copy_(hbuf, non_blocking=True)
+            st.step(x=xd, q=qd)
+            oh.copy_(st.out, non_blocking=True)
+            e_ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e_ev), world, device)
+        e2e = {"value": w.batch * K * world / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": nx + nq,
+               "d2h_bytes_per_step": oh.numel() * oh.element_size(),
+               "path": "rank_latent_kv_lk_b200.latent_decode_step per layer (C ABI), inputs from pinned host "
+                       "memory, outputs back to pinned host memory"}
+    extra = None
+    if not args.no_extra:
+        from rank_latent_kv_lk_b200.configs import WORKLOADS
+        del st
+        torch.cuda.empty_cache()
+        extra = measure_single(args, WORKLOADS[2], device, world, clocks_too=False, K=max(K, 128))
+
+    if rank != 0:
+        _finish(world)
+        return 0
+    hbm, peak_kind = peaks()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": workload_dtype(w), "data": workload_data(w),
+        "config": {"workload": w.name, "layers": L, "batch": w.batch, "tokens": w.context + 1,
+                   "l2": "not flushed: the 10.7 GB working set is far larger than L2 (126 MB)",
+                   "timing": "CUDA events at step boundaries on the launching stream; max over ranks; "
+                             "per-kernel times from a second pass with events between the kernels",
+                   "parallelism": f"replicas x{world} (independent decode problems, no collective)"},
+        "roofline": {"kernel": "decode_attn_kernel", "bound": "hbm", "achieved": attn_gbs, "peak": hbm,
+                     "unit": "GB/s", "frac": attn_gbs / hbm, "peak_kind": peak_kind,
+                     "frac_of_8tbs": attn_gbs / 8000.0,
+                     "algorithmic_bytes_per_launch": attn_bytes / (KP * L),
+                     "us_per_launch": attn_s / (KP * L) * 1e6,
+                     "traffic": profiled_traffic("decode_attn_kernel", w.key)},
+        "latent_project": {"achieved_gbs": proj_gbs, "us_per_call": proj_s / (KP * L) * 1e6,
+                           "algorithmic_bytes_per_call": proj_bytes / (KP * L)},
+        "step_algorithmic_gbs": (attn_bytes + proj_bytes) / KP / (total_ms / K / 1e3) / 1e9,
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if extra:
+        line["llava7b_b1_step"] = extra
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+    _finish(world)
+    return 0
+
+
+def measure_single(args, w, device, world, clocks_too=True, K=None):
+    """Appending decode steps of a single-layer workload (L2 flushed before
+    every step); returns the measurements as a dict."""
     st = DecodeState(w, device)
+    lk = st.lk
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
-
-    def flush_l2():
-        flush.fill_(1)
-
-    # warm-up (untimed)
     for i in range(max(3, args.warmup)):
         st.rewind_if_full()
         st.step(i)
     torch.cuda.synchronize()
-
-    K = args.steps
+    K = K or args.steps
     # timed region: events at step boundaries only (an event between the two
     # kernels would stop the attention launch from overlapping the projection)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    lens_at = []
     barrier(world)
     torch.cuda.synchronize()
-    torch.cuda._sleep(int(1e8))  # let the host queue run ahead of the device
-    with ClockSampler(local) as clocks:
+    torch.cuda._sleep(int(1e8))
+    n0 = lk.kernel_launches()
+    with ClockSampler(device.index, enabled=clocks_too) as clocks:
         for i in range(K):
             st.rewind_if_full()
-            flush_l2()
+            flush.fill_(1)
             ev[i][0].record(stream)
             st.step(i)
             ev[i][1].record(stream)
-            lens_at.append(st.lens)
         torch.cuda.synchronize()
+    launches = lk.kernel_launches() - n0
     barrier(world)
-    st.lk.device_status()
-    step_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
-    total_ms = max_over_ranks(sum(step_ms), world, device)
-    value = w.batch * K * world / (total_ms / 1e3)
-
-    # per-kernel durations: a second pass of K steps with an event between the
-    # kernels (for the roofline of each kernel; not the step time)
+    lk.device_status()
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), world, device)
     kev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     klens = []
     torch.cuda.synchronize()
     torch.cuda._sleep(int(1e8))
     for i in range(K):
         st.rewind_if_full()
-        flush_l2()
+        flush.fill_(1)
         kev[i][0].record(stream)
         st.project(i)
         kev[i][1].record(stream)
@@ -414,14 +741,11 @@ def run_ours(args):
         kev[i][2].record(stream)
         klens.append(st.lens)
     torch.cuda.synchronize()
-    proj_ms = [kev[i][0].elapsed_time(kev[i][1]) for i in range(K)]
-    attn_ms = [kev[i][1].elapsed_time(kev[i][2]) for i in range(K)]
-
-    # e2e: host buffers through the C ABI, copies inside the timed region
+    proj_s = statistics.mean(kev[i][0].elapsed_time(kev[i][1]) for i in range(K)) / 1e3
+    attn_s = statistics.mean(kev[i][1].elapsed_time(kev[i][2]) for i in range(K)) / 1e3
+    attn_bytes = statistics.mean(st.attn_bytes(n) for n in klens)
     e2e = None
     if not args.no_e2e:
-        # each step's x and q sit side by side in one pinned host buffer, so
-        # one host->device copy brings both (device views of one buffer)
         xs, qs = st.x_dec[0], st.q[0]
         nx = xs.numel() * xs.element_size()
         nq = qs.numel() * qs.element_size()
@@ -439,7 +763,7 @@ def run_ours(args):
         for i in range(K):
             j = i % w.steps
             st.rewind_if_full()
-            flush_l2()
+            flush.fill_(1)
             e_ev[i][0].record(stream)
             dbuf.copy_(hbuf[j], non_blocking=True)
             st.step(i, x=xd, q=qd)
@@ -447,49 +771,60 @@ def run_ours(args):
             e_ev[i][1].record(stream)
         torch.cuda.synchronize()
         barrier(world)
-        e_ms = max_over_ranks(sum(e_ev[i][0].elapsed_time(e_ev[i][1]) for i in range(K)), world, device)
-        e2e = {"value": w.batch * K * world / (e_ms / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": nx + nq,
+        e_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e_ev), world, device)
+        e2e = {"value": w.batch * K * world / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": nx + nq,
                "d2h_bytes_per_step": oh.numel() * oh.element_size()}
+    res = {"workload": w.name, "value": w.batch * K * world / (total_ms / 1e3), "unit": UNIT, "steps": K,
+           "ms_per_step": total_ms / K, "l2": "flushed before every step (256 MiB write, untimed)",
+           "gpu_launches": launches,
+           "attn_us_per_launch": attn_s * 1e6, "attn_gbs": attn_bytes / attn_s / 1e9,
+           "attn_algorithmic_bytes_per_launch": attn_bytes,
+           "proj_us_per_call": proj_s * 1e6, "proj_gbs": st.proj_bytes() / proj_s / 1e9,
+           "proj_algorithmic_bytes_per_call": st.proj_bytes()}
+    if e2e:
+        res["e2e"] = e2e
+    if clocks_too:
+        res["clocks"] = clocks.summary()
+    del st
+    torch.cuda.empty_cache()
+    return res
 
+
+def run_single(args, w):
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    r = measure_single(args, w, device, world)
     if rank != 0:
         _finish(world)
         return 0
     hbm, peak_kind = peaks()
-    attn_avg_s = statistics.mean(attn_ms) / 1e3
-    proj_avg_s = statistics.mean(proj_ms) / 1e3
-    attn_bytes = statistics.mean(st.attn_bytes(L) for L in klens)
-    proj_bytes = st.proj_bytes()
-    attn_gbs = attn_bytes / attn_avg_s / 1e9
-    proj_gbs = proj_bytes / proj_avg_s / 1e9
-    dominant = "latent_decode_attn" if attn_avg_s >= proj_avg_s else "latent_project_append"
-    if dominant == "latent_decode_attn":
-        ach, traffic = attn_gbs, profiled_traffic("decode_attn_kernel", w.key)
-    else:
-        ach, traffic = proj_gbs, profiled_traffic("proj_cluster_kernel", w.key)
+    dominant = "decode_attn_kernel" if r["attn_us_per_launch"] >= r["proj_us_per_call"] else "proj_cluster_kernel"
+    ach = r["attn_gbs"] if dominant == "decode_attn_kernel" else r["proj_gbs"]
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int8/f32", "data": "synthetic (seeded, shapes of the LLaVA-7B-like workload)",
+        "metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": r["steps"],
+        "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": workload_dtype(w), "data": workload_data(w),
         "config": {"workload": w.name, "batch": w.batch, "context": w.context, "decode_steps": w.steps,
-                   "storage": f"{w.kind} latents + per-token scales, bf16 factors and activations",
-                   "l2": "flushed before every step (256 MiB write, untimed)",
+                   "l2": r["l2"],
                    "timing": "CUDA events at step boundaries on the launching stream; max over ranks; "
                              "per-kernel times from a second pass of the same steps with an event between "
                              "the kernels",
                    "parallelism": f"replicas x{world} (independent decode problems, no collective)"},
         "roofline": {"kernel": dominant, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
-                     "frac": ach / hbm, "peak_kind": peak_kind, "traffic": traffic},
-        "latent_attn": {"achieved_gbs": attn_gbs, "frac_of_measured_hbm": attn_gbs / hbm,
-                        "frac_of_8tbs": attn_gbs / 8000.0, "us_per_launch": attn_avg_s * 1e6,
-                        "algorithmic_bytes_per_launch": attn_bytes},
-        "latent_project": {"achieved_gbs": proj_gbs, "us_per_call": proj_avg_s * 1e6,
-                           "algorithmic_bytes_per_call": proj_bytes},
-        "gpu_launches": K * 2,  # proj_cluster_kernel + decode_attn_kernel per step
-        "clocks": clocks.summary(),
+                     "frac": ach / hbm, "peak_kind": peak_kind, "frac_of_8tbs": ach / 8000.0,
+                     "traffic": profiled_traffic(dominant, w.key)},
+        "latent_attn": {"achieved_gbs": r["attn_gbs"], "us_per_launch": r["attn_us_per_launch"],
+                        "algorithmic_bytes_per_launch": r["attn_algorithmic_bytes_per_launch"]},
+        "latent_project": {"achieved_gbs": r["proj_gbs"], "us_per_call": r["proj_us_per_call"],
+                           "algorithmic_bytes_per_call": r["proj_algorithmic_bytes_per_call"]},
+        "gpu_launches": r["gpu_launches"], "clocks": r.get("clocks"),
     }
-    if e2e:
-        line["e2e"] = e2e
+    if "e2e" in r:
+        line["e2e"] = r["e2e"]
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
@@ -693,98 +1028,6 @@ def run_layer(args):
     return 0
 
 
-def run_all_layers(args):
-    """One decode step across every layer of a multi-layer workload (workload
-    4: 32 layers, ragged ranks, B = 8, T = 16384 + 1): per layer, the new
-    token's latent projection, quantisation and append, then the latent
-    attention, through lk_latent_decode_step.  The caches hold seeded random
-    codes (no prefill); x and q per layer are seeded draws.  The working set
-    (10.7 GB of latents and factors) is far larger than L2, so no flush is
-    needed; every timed step starts from the same context (seq_len reset,
-    untimed)."""
-    rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    init_dist(world, "nccl")
-    import rank_latent_kv_lk_b200 as lk
-    from rank_latent_kv_lk_b200 import synth
-    from rank_latent_kv_lk_b200.configs import WORKLOADS
-    w = WORKLOADS[args.workload]
-    rks, rvs = synth.ranks(w)
-    g = torch.Generator(device=device)
-    g.manual_seed(synth.seed_for(w, synth.CONTEXT))
-    layers = []
-    for l in range(w.n_layers):
-        A, BK, BV = synth.factors(w, l, rks[l], rvs[l])
-        ck = lk.LatentCache(w.batch, rks[l], w.capacity, w.kind, w.group, device)
-        cv = lk.LatentCache(w.batch, rvs[l], w.capacity, w.kind, w.group, device, role="v")
-        for c in (ck, cv):
-            c.codes.copy_(torch.randint(0, 256, c.codes.shape, dtype=torch.uint8, device=device, generator=g))
-            c.scales.copy_((torch.rand(c.scales.shape, device=device, generator=g) * 0.02 + 0.01).to(c.scales.dtype))
-        x = torch.randn(w.batch, w.embed_dim, generator=g, device=device).to(A.dtype)
-        q = torch.randn(w.batch, w.n_heads, w.head_dim, generator=g, device=device).to(A.dtype)
-        out = torch.empty(w.batch, w.n_heads, w.head_dim, dtype=A.dtype, device=device)
-        seq = torch.full((w.batch,), w.context, dtype=torch.int32, device=device)
-        layers.append((ck, cv, A.to(device), BK.to(device), BV.to(device), x, q, out, seq))
-    lens0 = [w.context] * w.batch
-
-    def step():
-        for ck, cv, A, BK, BV, x, q, out, seq in layers:
-            lk.latent_decode_step(ck, cv, x, A, seq, lens0, q, BK, BV, out=out)
-
-    def reset():
-        for layer in layers:
-            layer[8].fill_(w.context)
-
-    for _ in range(max(3, args.warmup)):
-        step()
-        reset()
-    torch.cuda.synchronize()
-    K = args.steps
-    stream = torch.cuda.current_stream()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    barrier(world)
-    torch.cuda.synchronize()
-    torch.cuda._sleep(int(2e8))
-    with ClockSampler(local) as clocks:
-        for i in range(K):
-            reset()
-            ev[i][0].record(stream)
-            step()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    lk.device_status()
-    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), world, device)
-    us = total_ms / K * 1e3
-    T = w.context + 1
-    rb = lambda r: r if w.kind == "i8" else r // 2
-    sb = lambda r: 4 if w.kind == "i8" else 2 * (-(-r // min(w.group, r)))
-    nbytes = 0
-    for l in range(w.n_layers):
-        per_tok = sum(rb(r) + sb(r) for r in rks[l]) + sum(rb(r) + sb(r) for r in rvs[l])
-        n_tot = sum(rks[l]) + sum(rvs[l])
-        nbytes += w.batch * T * per_tok + n_tot * w.embed_dim * 2 + n_tot * w.head_dim * 2
-    gbs = nbytes / (us * 1e-6) / 1e9
-    hbm, peak_kind = peaks()
-    if rank == 0:
-        print(json.dumps({
-            "mode": "all-layers", "metric": "decode tokens/s (one step across all layers)",
-            "value": w.batch * world / (us * 1e-6), "unit": "tokens/s", "n_gpus": world, "steps": K,
-            "warmup": args.warmup, "us_per_step": us, "higher_is_better": True, "scaling": "weak",
-            "dtype": "int8/f32" if w.kind == "i8" else "int4/f32",
-            "data": "synthetic (seeded random latent codes and scales, seeded factors, x and q)",
-            "config": {"workload": w.name, "layers": w.n_layers, "batch": w.batch, "tokens": T,
-                       "l2": "not flushed: the working set is far larger than L2",
-                       "launches": f"{2 * w.n_layers} per step (projection + attention per layer)"},
-            "algorithmic_bytes_per_step": nbytes,
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                         "peak_kind": peak_kind},
-            "gpu_launches": 2 * w.n_layers * K, "clocks": clocks.summary()}), flush=True)
-    _finish(world)
-    return 0
-
-
 def run_dense_compare(args):
     """Context for the pages' decode speedups (measured against flash decoding
     over dense K/V): per workload, one layer's latent attention against dense
@@ -870,8 +1113,6 @@ def main(argv=None):
         return run_layer(args)
     if args.dense_compare:
         return run_dense_compare(args)
-    if args.all_layers:
-        return run_all_layers(args)
     return run_ours(args)
 
 

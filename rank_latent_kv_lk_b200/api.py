@@ -88,6 +88,13 @@ class LatentCache:
         """Logical code rows and scales of the first lens[b] tokens (host copies)."""
         return self.geom.unpack(self.codes.cpu().numpy(), self.scales.cpu().numpy(), lens)
 
+    def read_unit(self, b, h, T):
+        """Code rows [T, rb_h] and scales of the first T tokens of one (b, h) (host copies)."""
+        off, n = self.geom.code_plane(b, h)
+        soff, sn = self.geom.scale_plane(b, h)
+        return self.geom.unpack_unit(self.codes[off:off + n].cpu().numpy(),
+                                     self.scales[soff:soff + sn].cpu().numpy(), h, T)
+
 
 def latent_project_append(k_cache, v_cache, x, A, seq_len, seq_len_host, x_scale=None, a_scale=None,
                           stream=None):

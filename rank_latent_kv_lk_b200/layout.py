@@ -167,3 +167,15 @@ class CacheGeometry:
             rows.append(rr)
             sc.append(ss)
         return rows, sc
+
+    def unpack_unit(self, plane, scale_plane, h, T):
+        """Code rows [T, rb_h] and scales of one (b, h) from that plane's bytes
+        (``plane``: the capacity * rb_h code bytes; ``scale_plane``: its
+        capacity * ng_h scales)."""
+        plane = np.asarray(plane, np.uint8)
+        if self.role == "k":
+            rows = plane[tile_index(T, self.rb[h])]
+        else:
+            rows = rows_from_v_plane(plane, T, self.rb[h], self.kind)
+        s = np.asarray(scale_plane).view(self.scale_dtype)[:T * self.ng[h]].reshape(T, self.ng[h])
+        return rows, (s[:, 0].copy() if self.kind == "i8" else s.copy())

@@ -24,3 +24,15 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Report how much of the band rule's slack the GPU tests actually used."""
+    helpers = sys.modules.get("tests.helpers")
+    if helpers is None or not helpers.BAND_STATS["codes"]:
+        return
+    s = helpers.BAND_STATS
+    terminalreporter.write_line(
+        f"band rule: {s['codes']} codes compared, {s['flips']} flipped by one at a tie "
+        f"(largest distance of a flip from the tie {s['max_flip_tie_distance']:.2e}, allowed 2e-3); "
+        f"largest relative scale deviation {s['max_scale_rel']:.2e} (allowed 1e-4)")
