@@ -63,8 +63,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the extra single-layer B = 1 measurement in the default line")
     ap.add_argument("--dense-compare", action="store_true",
-                    help="time one layer's latent attention against dense bf16 attention over materialised "
-                         "K/V of the same shapes (library SDPA), workloads 2-5")
+                    help="time one layer's latent attention against this library's dense bf16 flash-decoding "
+                         "over materialised K/V and the naive rebuild-then-attend path, workloads 2-5")
     return ap.parse_args(argv)
 
 
@@ -1029,11 +1029,15 @@ def run_layer(args):
 
 
 def run_dense_compare(args):
-    """Context for the pages' decode speedups (measured against flash decoding
-    over dense K/V): per workload, one layer's latent attention against dense
-    bf16 attention over materialised K and V of the same shapes
-    ([B, heads, T, H], PyTorch scaled_dot_product_attention -- a library
-    comparator, not part of this path).  L2 flushed before every launch."""
+    """The decode speed-up the pages report (latent attention vs flash decoding
+    over dense K/V; the naive path that rebuilds K and V through memory), per
+    workload, one layer, on this library's own kernels:
+      latent : lk_latent_decode_attn over the latent cache;
+      dense  : lk_dense_decode_attn over bf16 K and V of the same shapes;
+      naive  : lk_latent_reconstruct_kv (K and V rebuilt into memory) followed
+               by lk_dense_decode_attn;
+    and, for context, torch's scaled_dot_product_attention (a library kernel)
+    over the same dense K and V.  L2 flushed before every launch."""
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
@@ -1056,6 +1060,7 @@ def run_dense_compare(args):
         torch.cuda.synchronize()
         return statistics.median(e[0].elapsed_time(e[1]) * 1e3 for e in ev)
 
+    hbm, peak_kind = peaks()
     lines = []
     for key in (2, 3, 4, 5):
         w = WORKLOADS[key]
@@ -1075,24 +1080,32 @@ def run_dense_compare(args):
         seq = torch.full((w.batch,), T, dtype=torch.int32, device=device)
         out = torch.empty(w.batch, w.n_heads, w.head_dim, dtype=torch.bfloat16, device=device)
         latent_us = timed(lambda: lk.latent_decode_attn(ck, cv, q, BK, BV, seq, T, out=out), args.steps)
+        Kd = torch.empty(w.batch, w.n_heads, w.capacity, w.head_dim, dtype=torch.bfloat16, device=device)
+        Vd = torch.empty_like(Kd)
+        naive_us = timed(lambda: (lk.reconstruct_kv(ck, cv, BK, BV, seq, T, w.head_dim, Kd, Vd),
+                                  lk.dense_decode_attn(q, Kd, Vd, seq, T, out=out)), args.steps)
+        recon_us = timed(lambda: lk.reconstruct_kv(ck, cv, BK, BV, seq, T, w.head_dim, Kd, Vd), args.steps)
         del ck, cv
-        K = torch.randn(w.batch, w.n_heads, T, w.head_dim, generator=g, device=device).to(torch.bfloat16)
-        V = torch.randn(w.batch, w.n_heads, T, w.head_dim, generator=g, device=device).to(torch.bfloat16)
+        Kd.copy_(torch.randn(Kd.shape, generator=g, device=device).to(torch.bfloat16))
+        Vd.copy_(torch.randn(Vd.shape, generator=g, device=device).to(torch.bfloat16))
+        dense_us = timed(lambda: lk.dense_decode_attn(q, Kd, Vd, seq, T, out=out), args.steps)
+        Ks, Vs = Kd[:, :, :T], Vd[:, :, :T]
         q4 = q.unsqueeze(2)
-        dense_us = timed(lambda: torch.nn.functional.scaled_dot_product_attention(q4, K, V), args.steps)
-        dense_bytes = 2 * K.numel() * K.element_size()
-        del K, V
+        sdpa_us = timed(lambda: torch.nn.functional.scaled_dot_product_attention(q4, Ks, Vs), args.steps)
+        dense_bytes = 2 * w.batch * w.n_heads * T * w.head_dim * 2
+        del Kd, Vd, Ks, Vs
         torch.cuda.empty_cache()
         lines.append({"workload": w.name, "layer": 0, "batch": w.batch, "tokens": T,
-                      "latent_attn_us": latent_us, "dense_sdpa_us": dense_us,
+                      "latent_attn_us": latent_us, "dense_us": dense_us, "naive_us": naive_us,
+                      "naive_reconstruct_us": recon_us, "library_sdpa_us": sdpa_us,
                       "dense_kv_bytes": dense_bytes, "dense_gbs": dense_bytes / (dense_us * 1e-6) / 1e9,
-                      "speedup_vs_dense": dense_us / latent_us})
+                      "dense_frac_of_measured_hbm": dense_bytes / (dense_us * 1e-6) / 1e9 / hbm,
+                      "speedup_vs_dense": dense_us / latent_us, "speedup_vs_naive": naive_us / latent_us})
     if rank == 0:
         print(json.dumps({"mode": "dense-compare", "steps": args.steps,
-                          "note": "dense side: torch scaled_dot_product_attention over bf16 K/V of the same "
-                                  "shapes (library kernel), the pages' flash-decoding comparison point",
+                          "note": "latent, dense and naive on this library's kernels; torch SDPA for context",
                           "l2": "flushed before every launch (256 MiB write, untimed)",
-                          "results": lines}), flush=True)
+                          "peak_gbs": hbm, "peak_kind": peak_kind, "results": lines}), flush=True)
     return 0
 
 

@@ -253,6 +253,39 @@ lk_status lk_latent_decode_step(const lk_latent_cache* k_cache, const lk_latent_
                                 size_t decode_workspace_bytes, lk_stream_t stream);
 
 /*
+ * Dense bf16 flash-decoding over materialised K and V: the baseline the
+ * pages measure their decode speed-ups against (WSVD technical summary §4:
+ * speed-up over flash decoding; LASER results).  For every batch row b and
+ * head h, out = softmax(q K^T * softmax_scale) V over positions
+ * [0, seq_len[b]), split over the tokens like lk_latent_decode_attn.
+ * q: bf16 [B, n_heads, head_dim]; K, V: bf16 [B, n_heads, capacity,
+ * head_dim] (one row per position); head_dim a multiple of 8 up to 256;
+ * q, K, V 16-byte aligned.  out: [B, n_heads, head_dim] LK_F32 or LK_BF16.
+ * workspace: lk_dense_decode_workspace_bytes(...) bytes, 256-B aligned, its
+ * first round_up(4 * B * n_heads, 256) bytes zero at entry (left zero).
+ */
+lk_status lk_dense_decode_attn(const void* q, const void* K, const void* V, int32_t batch, int32_t n_heads,
+                               int32_t head_dim, int32_t capacity, const int32_t* seq_len,
+                               int32_t max_seq_len, float softmax_scale, void* out, lk_dtype out_dtype,
+                               void* workspace, size_t workspace_bytes, lk_stream_t stream);
+size_t lk_dense_decode_workspace_bytes(int32_t batch, int32_t n_heads, int32_t head_dim, int32_t max_seq_len);
+
+/*
+ * The naive low-rank path the WSVD page contrasts with its fused kernel
+ * (technical summary §1: rebuilding K and V from the factors through
+ * memory costs more than it saves): for positions [0, seq_len[b]),
+ *   K_out[b, h, t, :] = dequant(c_K[b, h, t]) B_K^h,  V_out likewise,
+ * stored bf16 [B, n_heads, capacity, head_dim] (rows past seq_len[b] are not
+ * written).  Caches, B_K / B_V and their layouts as for lk_latent_decode_attn.
+ * Attending the result with lk_dense_decode_attn gives the same output as
+ * lk_latent_decode_attn up to the bf16 rounding of K and V.
+ */
+lk_status lk_latent_reconstruct_kv(const lk_latent_cache* k_cache, const lk_latent_cache* v_cache,
+                                   const void* B_K, const void* B_V, lk_dtype b_dtype, int32_t head_dim,
+                                   const int32_t* seq_len, int32_t max_seq_len, void* K_out, void* V_out,
+                                   lk_stream_t stream);
+
+/*
  * LASER hybrid dense + low-rank linear, W8A8 (LASER technical summary §3:
  * selected input channels go through SVD factors, the rest stay dense; both
  * branches RTN-quantised).
@@ -318,6 +351,25 @@ lk_status lk_rmsnorm_quant_i8(const void* x, lk_dtype x_dtype, int32_t m, int32_
  * per-row int8 quantisation of h.  gate, up: [m, n] LK_F32 or LK_BF16. */
 lk_status lk_swiglu_quant_i8(const void* gate, const void* up, lk_dtype dtype, int32_t m,
                              int32_t n, int8_t* h_q, float* h_scale, lk_stream_t stream);
+
+/*
+ * Test hook for the failure path (no counterpart on the pages): the decode
+ * attention of lk_latent_decode_attn (same arguments and validation), with its
+ * copy producer told to stop before work item `stall_item` (>= 0; items are
+ * (b, h) units times stages of 224 or 448 tokens) as if that copy never
+ * arrived, and every pipeline wait bounded by `wait_us` microseconds instead
+ * of the default 2 s.  The waits behind the missing copy expire, the kernel
+ * lets every copy it did start land (allowing 2 s for each) and returns;
+ * `out` then holds no meaningful values, the workspace counters are left
+ * zero, and lk_device_status() reports LK_ERR_DEVICE.  No other entry point
+ * reaches this path.
+ */
+lk_status lk_debug_decode_attn_stall(const lk_latent_cache* k_cache, const lk_latent_cache* v_cache,
+                                     const void* q, lk_dtype q_dtype, const void* B_K, const void* B_V,
+                                     lk_dtype b_dtype, int32_t head_dim, const int32_t* seq_len,
+                                     int32_t max_seq_len, float softmax_scale, void* out, lk_dtype out_dtype,
+                                     int32_t n_split, void* workspace, size_t workspace_bytes,
+                                     int32_t stall_item, uint32_t wait_us, lk_stream_t stream);
 
 /* Synchronises the device, then reports (and with reset != 0 clears) the
  * error word kernels set when a bounded wait expires: LK_OK or LK_ERR_DEVICE. */

@@ -8,7 +8,7 @@ import importlib
 
 _API = ("LatentCache", "LowrankWeight", "device_status", "latent_decode_attn", "latent_decode_step",
         "latent_project_append", "lowrank_linear", "quantize_latent", "quantize_rows_i8", "rmsnorm_quant_i8",
-        "swiglu_quant_i8", "workspaces", "kernel_launches")
+        "swiglu_quant_i8", "workspaces", "kernel_launches", "dense_decode_attn", "reconstruct_kv")
 
 
 def __getattr__(name):

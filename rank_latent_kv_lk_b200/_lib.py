@@ -90,8 +90,13 @@ def _load():
         "lk_latent_decode_workspace_bytes": (SZ, [CP, CP, I32, I32]),
         "lk_latent_decode_attn_noalloc": (C.c_int, [CP, CP, P, C.c_int, P, P, C.c_int, I32, P, I32, C.c_float, P,
                                                     C.c_int, I32, P]),
+        "lk_debug_decode_attn_stall": (C.c_int, [CP, CP, P, C.c_int, P, P, C.c_int, I32, P, I32, C.c_float, P,
+                                                 C.c_int, I32, P, SZ, I32, C.c_uint32, P]),
         "lk_latent_decode_step": (C.c_int, [CP, CP, P, C.c_int, P, P, C.c_int, P, I32, P, P, P, C.c_int, P, P,
                                             C.c_int, I32, C.c_float, P, C.c_int, I32, P, SZ, P, SZ, P]),
+        "lk_dense_decode_attn": (C.c_int, [P, P, P, I32, I32, I32, I32, P, I32, C.c_float, P, C.c_int, P, SZ, P]),
+        "lk_dense_decode_workspace_bytes": (SZ, [I32, I32, I32, I32]),
+        "lk_latent_reconstruct_kv": (C.c_int, [CP, CP, P, P, C.c_int, I32, P, I32, P, P, P]),
         "lk_lowrank_linear": (C.c_int, [WP, P, P, I32, P, P, C.c_int, P, P, P, SZ, P]),
         "lk_lowrank_workspace_bytes": (SZ, [WP, I32]),
         "lk_quantize_latent": (C.c_int, [P, I32, I32, C.c_int, I32, P, P, P]),

@@ -168,6 +168,34 @@ def latent_decode_step(k_cache, v_cache, x, A, seq_len, seq_len_host, q, B_K, B_
     return out
 
 
+def dense_decode_attn(q, K, V, seq_len, max_seq_len, softmax_scale=None, out=None, out_dtype=None, stream=None):
+    """Dense bf16 flash-decoding over materialised K, V [B, heads, capacity, H] (comparison point)."""
+    B, nh, cap, H = K.shape
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(H)
+    if out is None:
+        out = torch.empty((B, nh, H), dtype=out_dtype or q.dtype, device=q.device)
+    need = lib.lk_dense_decode_workspace_bytes(B, nh, H, int(max_seq_len))
+    ws = workspaces.get(("dense", B * nh), need, q.device)
+    check(lib.lk_dense_decode_attn(_ptr(q), _ptr(K), _ptr(V), B, nh, H, cap, _ptr(seq_len), int(max_seq_len),
+                                   float(softmax_scale), _ptr(out), _dtype_code(out), _ptr(ws), ws.numel(),
+                                   _stream(stream)))
+    return out
+
+
+def reconstruct_kv(k_cache, v_cache, B_K, B_V, seq_len, max_seq_len, head_dim, K_out=None, V_out=None, stream=None):
+    """The naive path: K, V rebuilt from the latent cache into bf16 [B, heads, capacity, H]."""
+    shape = (k_cache.batch, len(k_cache.ranks), k_cache.capacity, head_dim)
+    if K_out is None:
+        K_out = torch.zeros(shape, dtype=torch.bfloat16, device=B_K.device)
+    if V_out is None:
+        V_out = torch.zeros(shape, dtype=torch.bfloat16, device=B_K.device)
+    check(lib.lk_latent_reconstruct_kv(k_cache.desc(), v_cache.desc(), _ptr(B_K), _ptr(B_V), _dtype_code(B_K),
+                                       head_dim, _ptr(seq_len), int(max_seq_len), _ptr(K_out), _ptr(V_out),
+                                       _stream(stream)))
+    return K_out, V_out
+
+
 class LowrankWeight:
     """Device weights of one LASER hybrid linear (int8, fp16 scales)."""
 

@@ -223,7 +223,8 @@ lk_status decode_attn_impl(const lk_latent_cache* k, const lk_latent_cache* v, c
                            const void* B_K, const void* B_V, lk_dtype b_dtype, int32_t head_dim,
                            const int32_t* seq_len, int32_t max_seq_len, float softmax_scale, void* out,
                            lk_dtype out_dtype, int32_t n_split, void* workspace, size_t workspace_bytes,
-                           lk_stream_t stream, bool launch, int early_inputs, int stable_len) {
+                           lk_stream_t stream, bool launch, int early_inputs, int stable_len,
+                           int stall_item = -1, uint64_t wait_ns = 0) {
   lk_status s;
   if ((s = check_cache(k, "k_cache", true)) != LK_OK) return s;
   if ((s = check_cache(v, "v_cache", true)) != LK_OK) return s;
@@ -277,6 +278,8 @@ lk_status decode_attn_impl(const lk_latent_cache* k, const lk_latent_cache* v, c
   a.softmax_scale = softmax_scale;
   a.early_inputs = early_inputs;
   a.stable_len = stable_len;
+  a.stall_item = stall_item;
+  a.wait_ns = wait_ns;
   if (!launch) return LK_OK;
   cudaError_t e = lk::launch_decode_attn(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "lk_latent_decode_attn");
@@ -291,6 +294,18 @@ lk_status lk_latent_decode_attn(const lk_latent_cache* k, const lk_latent_cache*
                                 void* workspace, size_t workspace_bytes, lk_stream_t stream) {
   return decode_attn_impl(k, v, q, q_dtype, B_K, B_V, b_dtype, head_dim, seq_len, max_seq_len, softmax_scale, out,
                           out_dtype, n_split, workspace, workspace_bytes, stream, true, 0, 0);
+}
+
+lk_status lk_debug_decode_attn_stall(const lk_latent_cache* k, const lk_latent_cache* v, const void* q,
+                                     lk_dtype q_dtype, const void* B_K, const void* B_V, lk_dtype b_dtype,
+                                     int32_t head_dim, const int32_t* seq_len, int32_t max_seq_len,
+                                     float softmax_scale, void* out, lk_dtype out_dtype, int32_t n_split,
+                                     void* workspace, size_t workspace_bytes, int32_t stall_item, uint32_t wait_us,
+                                     lk_stream_t stream) {
+  if (stall_item < 0 || wait_us == 0) return fail(LK_ERR_INVALID_ARG, "stall_item must be >= 0 and wait_us > 0");
+  return decode_attn_impl(k, v, q, q_dtype, B_K, B_V, b_dtype, head_dim, seq_len, max_seq_len, softmax_scale, out,
+                          out_dtype, n_split, workspace, workspace_bytes, stream, true, 0, 0, stall_item,
+                          (uint64_t)wait_us * 1000u);
 }
 
 lk_status lk_latent_decode_step(const lk_latent_cache* k, const lk_latent_cache* v, const void* x, lk_dtype x_dtype,
@@ -317,6 +332,91 @@ lk_status lk_latent_decode_step(const lk_latent_cache* k, const lk_latent_cache*
   if (s != LK_OK) return s;
   return decode_attn_impl(k, v, q, q_dtype, B_K, B_V, b_dtype, head_dim, seq_len, max_len, softmax_scale, out,
                           out_dtype, n_split, decode_workspace, decode_workspace_bytes, stream, true, 1, stable_len);
+}
+
+size_t lk_dense_decode_workspace_bytes(int32_t batch, int32_t n_heads, int32_t head_dim, int32_t max_seq_len) {
+  if (batch < 1 || n_heads < 1 || head_dim < 8 || max_seq_len < 0) return 0;
+  return lk::dense_workspace_bytes(batch * n_heads, head_dim, max_seq_len, num_sms());
+}
+
+lk_status lk_dense_decode_attn(const void* q, const void* K, const void* V, int32_t batch, int32_t n_heads,
+                               int32_t head_dim, int32_t capacity, const int32_t* seq_len, int32_t max_seq_len,
+                               float softmax_scale, void* out, lk_dtype out_dtype, void* workspace,
+                               size_t workspace_bytes, lk_stream_t stream) {
+  if (!q || !K || !V || !seq_len || !out) return fail(LK_ERR_INVALID_ARG, "null q, K, V, seq_len or out");
+  if (batch < 1 || n_heads < 1 || capacity < 1) return fail(LK_ERR_SHAPE, "batch, n_heads and capacity must be >= 1");
+  if (head_dim < 8 || head_dim > LK_MAX_HEAD_DIM || head_dim % 8 != 0)
+    return fail(LK_ERR_SHAPE, "head_dim %d must be a multiple of 8 in [8, %d]", head_dim, LK_MAX_HEAD_DIM);
+  if (max_seq_len < 0 || max_seq_len > capacity)
+    return fail(LK_ERR_SHAPE, "max_seq_len %d outside [0, capacity]", max_seq_len);
+  if (out_dtype != LK_F32 && out_dtype != LK_BF16) return fail(LK_ERR_DTYPE, "out dtype must be LK_F32 or LK_BF16");
+  if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16)) return fail(LK_ERR_ALIGN, "q, K and V must be 16-byte aligned");
+  if (!(softmax_scale == softmax_scale)) return fail(LK_ERR_INVALID_ARG, "softmax_scale is NaN");
+  const size_t need = lk_dense_decode_workspace_bytes(batch, n_heads, head_dim, max_seq_len);
+  if (!workspace || workspace_bytes < need)
+    return fail(LK_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
+  if (!aligned(workspace, 256)) return fail(LK_ERR_ALIGN, "workspace must be 256-byte aligned");
+  lk::DenseLaunch a{};
+  a.q = q;
+  a.K = K;
+  a.V = V;
+  a.seq_len = seq_len;
+  a.out = out;
+  a.workspace = workspace;
+  a.batch = batch;
+  a.n_heads = n_heads;
+  a.head_dim = head_dim;
+  a.capacity = capacity;
+  a.max_len = max_seq_len;
+  a.out_bf16 = out_dtype == LK_BF16;
+  a.num_sms = num_sms();
+  a.softmax_scale = softmax_scale;
+  if (max_seq_len == 0 && batch * n_heads == 0) return LK_OK;
+  cudaError_t e = lk::launch_dense_decode(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lk_dense_decode_attn");
+  return LK_OK;
+}
+
+lk_status lk_latent_reconstruct_kv(const lk_latent_cache* k, const lk_latent_cache* v, const void* B_K,
+                                   const void* B_V, lk_dtype b_dtype, int32_t head_dim, const int32_t* seq_len,
+                                   int32_t max_seq_len, void* K_out, void* V_out, lk_stream_t stream) {
+  lk_status s;
+  if ((s = check_cache(k, "k_cache", true)) != LK_OK) return s;
+  if ((s = check_cache(v, "v_cache", true)) != LK_OK) return s;
+  if (k->batch != v->batch || k->n_heads != v->n_heads || k->capacity != v->capacity)
+    return fail(LK_ERR_SHAPE, "k and v caches differ in batch, heads or capacity");
+  if (k->code_dtype != v->code_dtype) return fail(LK_ERR_UNSUPPORTED, "k and v caches differ in code dtype");
+  if (!B_K || !B_V || !seq_len || !K_out || !V_out) return fail(LK_ERR_INVALID_ARG, "null B_K, B_V, seq_len or outputs");
+  if (b_dtype != LK_F32 && b_dtype != LK_BF16) return fail(LK_ERR_DTYPE, "B dtype must be LK_F32 or LK_BF16");
+  if (head_dim < 8 || head_dim > LK_MAX_HEAD_DIM || head_dim % 8 != 0)
+    return fail(LK_ERR_SHAPE, "head_dim %d must be a multiple of 8 in [8, %d]", head_dim, LK_MAX_HEAD_DIM);
+  if (max_seq_len < 0 || max_seq_len > k->capacity)
+    return fail(LK_ERR_SHAPE, "max_seq_len %d outside [0, capacity]", max_seq_len);
+  if (!aligned(K_out, 16) || !aligned(V_out, 16)) return fail(LK_ERR_ALIGN, "K_out and V_out must be 16-byte aligned");
+  lk::ReconLaunch a{};
+  a.codes[0] = k->codes;
+  a.codes[1] = v->codes;
+  a.scales[0] = k->scales;
+  a.scales[1] = v->scales;
+  a.B[0] = B_K;
+  a.B[1] = B_V;
+  a.out[0] = K_out;
+  a.out[1] = V_out;
+  a.ranks[0] = k->ranks;
+  a.ranks[1] = v->ranks;
+  a.group[0] = k->group;
+  a.group[1] = v->group;
+  a.seq_len = seq_len;
+  a.kind = k->code_dtype == LK_I8 ? 0 : 1;
+  a.batch = k->batch;
+  a.n_heads = k->n_heads;
+  a.head_dim = head_dim;
+  a.capacity = k->capacity;
+  a.max_len = max_seq_len;
+  a.b_bf16 = b_dtype == LK_BF16;
+  cudaError_t e = lk::launch_reconstruct_kv(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lk_latent_reconstruct_kv");
+  return LK_OK;
 }
 
 size_t lk_lowrank_workspace_bytes(const lk_lowrank_weight* w, int32_t m) {
@@ -424,12 +524,13 @@ lk_status lk_swiglu_quant_i8(const void* gate, const void* up, lk_dtype dtype, i
 lk_status lk_device_status(int32_t reset) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "lk_device_status");
-  unsigned int words[4] = {0, 0, 0, 0};
-  cudaError_t (*fns[5])(unsigned int*, int) = {lk_decode_status_word, lk_quant_status_word,
-                                                lk_project_status_word, lk_lowrank_status_word,
-                                                lk_gemm_tc_status_word};
+  cudaError_t (*fns[])(unsigned int*, int) = {lk_decode_status_word, lk_quant_status_word,
+                                               lk_project_status_word, lk_lowrank_status_word,
+                                               lk_gemm_tc_status_word};
+  constexpr int kWords = (int)(sizeof(fns) / sizeof(fns[0]));
+  unsigned int words[kWords] = {};
   unsigned int any = 0;
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < kWords; ++i) {
     e = fns[i](&words[i], reset);
     if (e != cudaSuccess) return cuda_fail(e, "lk_device_status");
     any |= words[i];

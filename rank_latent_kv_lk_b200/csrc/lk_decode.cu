@@ -84,6 +84,8 @@ struct DecodeParams {
   int q_bf16, b_bf16, out_bf16;
   int early_inputs;  // q, B_K, B_V are read before waiting for the previous kernel on the stream
   int stable_len;    // with early_inputs: cache positions below it are final before the kernel starts
+  uint64_t wait_ns;  // limit of the pipeline waits (draining copies after an error always allows 2 s)
+  int stall_item;    // test hook: the producer stops before this (unit, stage) item (-1: never)
   int max_len;
   int ST;  // tokens per stage: 32 * TG * kCW
   int S;   // stages per unit: ceil(max_len / ST)
@@ -413,7 +415,7 @@ struct SmemLayout {
 };
 
 constexpr int kSmemFixed = kMaxR * 4 + 3 * kMaxR + kCW * (2 + kMaxR) * 4 + (2 + kMaxR) * 4 +
-                           (2 * kMaxStages + 4) * 8 + 16;
+                           (2 * kMaxStages + 4) * 8 + 32;
 
 LK_DEVICE SmemLayout smem_layout(const DecodeParams& p) {
   SmemLayout L;
@@ -449,6 +451,7 @@ struct Bars {
   volatile int* abort_flag;
   int* ticket_flag;
   float* qa;
+  int* bv_issued;  // this unit's B_V copy was started (it must land before the CTA may end)
 };
 
 LK_DEVICE Bars bars_of(uint8_t* smem, const SmemLayout& L) {
@@ -461,6 +464,7 @@ LK_DEVICE Bars bars_of(uint8_t* smem, const SmemLayout& L) {
   B.abort_flag = reinterpret_cast<volatile int*>(smem + L.off_misc);
   B.ticket_flag = reinterpret_cast<int*>(smem + L.off_misc) + 1;
   B.qa = reinterpret_cast<float*>(smem + L.off_misc) + 2;
+  B.bv_issued = reinterpret_cast<int*>(smem + L.off_misc) + 3;
   return B;
 }
 
@@ -482,7 +486,7 @@ LK_DEVICE void produce(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
     const int s_end = min(p.S, s + (i1 - it));
     const int b = u / p.n_heads, h = u - b * p.n_heads;
     const HeadGeom g = unit_geometry<KIND>(p, b, h);
-    if (ok && nunit > 0 && !lk_mbar_wait_bounded(B.fempty, (uint32_t)((nunit - 1) & 1), LK_WAIT_LIMIT_NS)) {
+    if (ok && nunit > 0 && !lk_mbar_wait_bounded(B.fempty, (uint32_t)((nunit - 1) & 1), p.wait_ns)) {
       *B.abort_flag = 1;
       ok = false;
     }
@@ -508,12 +512,12 @@ LK_DEVICE void produce(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
         end = min((int64_t)((len + 15) & ~15), (int64_t)p.capacity);
       }
       if (t0 >= len) break;  // this and the unit's later stages hold no tokens
-      if (*B.abort_flag) {
+      if (*B.abort_flag || u * p.S + ss == p.stall_item) {  // (the test hook stops here, copies unissued)
         ok = false;
         break;
       }
       const int buf = k % NS;
-      if (k >= NS && !lk_mbar_wait_bounded(&B.empty[buf], (uint32_t)(((k / NS) - 1) & 1), LK_WAIT_LIMIT_NS)) {
+      if (k >= NS && !lk_mbar_wait_bounded(&B.empty[buf], (uint32_t)(((k / NS) - 1) & 1), p.wait_ns)) {
         *B.abort_flag = 1;
         ok = false;
         break;
@@ -552,14 +556,17 @@ LK_DEVICE void absorb_q(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
   const int H = p.head_dim;
   float* qt_s = reinterpret_cast<float*>(smem + L.off_qt);
   int8_t* qterm = reinterpret_cast<int8_t*>(smem + L.off_qterm);
-  if (threadIdx.x == 0 && !*B.abort_flag) {
+  if (threadIdx.x == 0) {
     // B_V^h is read when the unit ends; the previous unit's output is done
     // (the slot is free) and its copy was waited for
-    const uint32_t bvb = g.rv * H * p.b_size;
-    lk_mbar_arrive_expect_tx(B.vbar, bvb);
-    lk_bulk_g2s(smem + L.off_bv, static_cast<const uint8_t*>(p.BV) + g.bv_off * p.b_size, bvb, B.vbar);
+    *B.bv_issued = !*B.abort_flag;
+    if (*B.bv_issued) {
+      const uint32_t bvb = g.rv * H * p.b_size;
+      lk_mbar_arrive_expect_tx(B.vbar, bvb);
+      lk_bulk_g2s(smem + L.off_bv, static_cast<const uint8_t*>(p.BV) + g.bv_off * p.b_size, bvb, B.vbar);
+    }
   }
-  if (!*B.abort_flag && !lk_mbar_wait_bounded(B.fbar, (uint32_t)(n & 1), LK_WAIT_LIMIT_NS)) *B.abort_flag = 1;
+  if (!*B.abort_flag && !lk_mbar_wait_bounded(B.fbar, (uint32_t)(n & 1), p.wait_ns)) *B.abort_flag = 1;
   if (!*B.abort_flag) {
     const uint8_t* qs = smem + L.off_q;
     const uint8_t* bks = smem + L.off_bk;
@@ -659,7 +666,7 @@ LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
       tl_end = len - s0 * ST - tl;
     }
     if ((s0 + j) * ST >= len) break;  // no copies were issued for the unit's later stages
-    if (!lk_mbar_wait_bounded(&B.full[buf], phase, LK_WAIT_LIMIT_NS)) {
+    if (!lk_mbar_wait_bounded(&B.full[buf], phase, p.wait_ns)) {
       *B.abort_flag = 1;
       break;
     }
@@ -839,8 +846,16 @@ LK_DEVICE void finish_unit(const DecodeParams& p, uint8_t* smem, const SmemLayou
   float* wst = reinterpret_cast<float*>(smem + L.off_wst);
   float* cta = reinterpret_cast<float*>(smem + L.off_cta);
   // this unit's B_V copy has landed long ago; waiting here also keeps the next
-  // unit's copy from starting while this one is in flight
-  if (!*B.abort_flag && !lk_mbar_wait_bounded(B.vbar, (uint32_t)(n & 1), LK_WAIT_LIMIT_NS)) *B.abort_flag = 1;
+  // unit's copy from starting while this one is in flight, and a copy that
+  // was started is waited for even after an error (it must land before the
+  // CTA may end)
+  if (*B.bv_issued) {
+    const bool was_aborted = *B.abort_flag != 0;
+    if (!lk_mbar_wait_bounded(B.vbar, (uint32_t)(n & 1), was_aborted ? LK_WAIT_LIMIT_NS : p.wait_ns)) {
+      *B.abort_flag = 1;
+      if (was_aborted) lk_dev_fail(LK_DEV_TIMEOUT_DRAIN);
+    }
+  }
   const bool aborted = consumer_sync_or(*B.abort_flag != 0);  // every warp's state is written
   float M = -INFINITY;
 #pragma unroll
@@ -1053,6 +1068,8 @@ size_t decode_workspace_bytes(int units, int rv_max, int max_len, int n_split) {
 
 cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
   DecodeParams p{};
+  p.wait_ns = a.wait_ns ? a.wait_ns : LK_WAIT_LIMIT_NS;
+  p.stall_item = a.stall_item;
   p.codes_k = static_cast<const uint8_t*>(a.codes_k);
   p.codes_v = static_cast<const uint8_t*>(a.codes_v);
   p.scales_k = static_cast<const uint8_t*>(a.scales_k);

@@ -38,12 +38,41 @@ struct DecodeLaunch {
   int early_inputs;  // read q, B_K, B_V before waiting for the previous kernel (decode step entry point)
   int stable_len;    // with early_inputs: positions below it are final before the kernel starts
   float softmax_scale;
+  uint64_t wait_ns = 0;  // bound of the pipeline waits (0: the library's default)
+  int stall_item = -1;   // test hook: the copy producer stops before this item
 };
 // Workspace of a decode call: arrival counters for the units plus two partial
 // slots per CTA; n_split > 0 asks for about n_split pieces per unit, 0 for a
 // grid that fills the GPU (at most 1024 CTAs).
 size_t decode_workspace_bytes(int units, int rv_max, int max_len, int n_split);
 cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream);
+
+
+// ---------------------------------------------------------------- dense comparison points
+struct DenseLaunch {
+  const void* q;  // bf16 [B, n_heads, H]
+  const void* K;  // bf16 [B, n_heads, capacity, H]
+  const void* V;
+  const int32_t* seq_len;
+  void* out;
+  void* workspace;
+  int batch, n_heads, head_dim, capacity, max_len, out_bf16, num_sms;
+  float softmax_scale;
+};
+size_t dense_workspace_bytes(int units, int head_dim, int max_len, int num_sms);
+cudaError_t launch_dense_decode(const DenseLaunch& a, cudaStream_t stream);
+
+struct ReconLaunch {
+  const void* codes[2];      // K cache, V cache
+  const void* scales[2];
+  const void* B[2];          // B_K, B_V packed per head
+  void* out[2];              // bf16 [B, n_heads, capacity, H]
+  const int32_t* ranks[2];   // host
+  int group[2];
+  const int32_t* seq_len;
+  int kind, batch, n_heads, head_dim, capacity, max_len, b_bf16;
+};
+cudaError_t launch_reconstruct_kv(const ReconLaunch& a, cudaStream_t stream);
 
 // ---------------------------------------------------------------- projection
 enum XType { X_F32 = 0, X_BF16 = 1, X_I8 = 2 };

@@ -9,10 +9,11 @@
 //      the int8 dequantisation scales when the inputs are int8, quantise the
 //      r_h values (absmax, RNE) and write codes + scale at position
 //      seq_len[b] + t in the token-tiled cache layout.
-// Decode (<= 32 rows) runs both phases in ONE launch: a cluster of CTAs per
-// head splits E, and the cluster's rank 0 sums the partials over distributed
-// shared memory and appends; the last head to finish advances seq_len.  Prefill runs the tiled GEMM per
-// row chunk, then an epilogue launch.
+// Decode (at most kGemvMaxRows = 8 token rows) runs both phases in ONE
+// launch: a cluster of CTAs per head splits E, and the cluster's rank 0 sums
+// the partials over distributed shared memory and appends; the last head to
+// finish advances seq_len.  More rows (prefill, or a decode batch above 8)
+// run the tensor-core GEMM, then the quantise-and-append launch.
 #include "lk_common.cuh"
 #include "lk_internal.h"
 #include "lk_quant.cuh"
@@ -211,9 +212,18 @@ __global__ void __launch_bounds__(128) proj_finalize_kernel(const __grid_constan
 // cluster's rank 0 sums the kClusterE partials over distributed shared memory,
 // quantises and appends.  No partials leave the SMs and nobody waits on a
 // global counter; the last head to finish advances seq_len (atomic ticket).
-constexpr int kClusterE = 4;
-constexpr int kProjNC = 2;  // latent columns a warp works on at once
-constexpr int kProjU = 4;   // 16-byte chunks per lane per column in flight
+//
+// Inside a CTA the head's columns are cut into tiles of 8; a warp takes one
+// tile over a contiguous range of the slice (the 8 warps spread over the
+// tiles, several warps per tile when the head has fewer than 8 tiles).
+// Lane 4 c + k takes column c of the tile and every fourth 16-byte chunk of
+// the range starting at k: the four lanes of a column read 64 consecutive
+// bytes of its weight row per load, each weight is read once from memory,
+// and the rows of x (converted once to fp32 in shared memory) are broadcast
+// loads.  The four lanes' sums meet by two shuffles, the warps of a tile in
+// shared memory in a fixed order (the result does not depend on timing).
+constexpr int kClusterE = 8;  // CTAs per head (portable cluster size): each reduces 1/8 of E
+constexpr int kProjWarps = kGemvThreads / 32;
 
 struct ClusterProjParams {
   FinalizeParams f;
@@ -221,14 +231,10 @@ struct ClusterProjParams {
   const void* A;
   int M, E, slice;
   int32_t* done_cnt;
-  int off_A, off_x, off_bar;  // staged variant: shared-memory offsets of the A and x slices and the barrier
+  int off_x, off_red;  // shared-memory offsets: x slice (fp32, or int8 for int8 inputs), warp partials
 };
 
-// ST (staged, M <= 8): the CTA's whole slice of A (r rows x slice) and of x
-// is brought into shared memory by bulk copies issued at once, so all of the
-// CTA's bytes are in flight together; the dot products then read shared
-// memory.  Otherwise each warp streams its A rows from global memory.
-template <int XT, int MT, bool ST>
+template <int XT, int MT>
 __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid_constant__ ClusterProjParams p) {
   lk_grid_dep_launch();  // a decode launched next may start its set-up now
   using T = typename XTraits<XT>::T;
@@ -252,178 +258,124 @@ __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid
   // a peer's shared memory may be written only once that CTA runs: arrive now,
   // wait just before the first remote write
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-  bool joined = false;
-  auto join = [&]() {
-    if (!joined) {
-      asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-      joined = true;
-    }
-  };
-  const T* x = static_cast<const T*>(p.x);  // read through L1: every warp of the CTA uses the same slice
+  const T* x = static_cast<const T*>(p.x);
   const T* A = static_cast<const T*>(p.A);
-
-  if constexpr (ST) {
-    // rows in groups of 8 (x with group 0), one barrier each, so the first
-    // rows are worked on while the later ones are still arriving
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + p.off_bar);
-    const T* As = reinterpret_cast<const T*>(smem_raw + p.off_A);
-    const T* xs = reinterpret_cast<const T*>(smem_raw + p.off_x);
-    const int ngroups = (r + 7) / 8;
-    if (threadIdx.x == 0) {
-      for (int gi = 0; gi < ngroups; ++gi) lk_mbar_init(&bar[gi], 1);
-      lk_fence_mbar_init();
+  // x slice into shared memory: fp32 for float inputs, the int8 codes as they are
+  float* xf = reinterpret_cast<float*>(smem_raw + p.off_x);
+  int8_t* xi = reinterpret_cast<int8_t*>(smem_raw + p.off_x);
+  for (int i = threadIdx.x; i < M * chunks; i += kGemvThreads) {
+    const int m = i / chunks, cc = i - m * chunks;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + (int64_t)m * p.E + e0 + cc * VE));
+    if constexpr (INT) {
+      *reinterpret_cast<uint4*>(xi + (size_t)m * p.slice + cc * VE) = v;
+    } else {
+      float vf[VE];
+      expand16<XT>(v, vf);
+      float4* dst = reinterpret_cast<float4*>(xf + (size_t)m * p.slice + cc * VE);
+#pragma unroll
+      for (int k = 0; k < VE / 4; ++k) dst[k] = make_float4(vf[4 * k], vf[4 * k + 1], vf[4 * k + 2], vf[4 * k + 3]);
     }
-    __syncthreads();
-    if (threadIdx.x == 0 && elen > 0) {
-      const uint32_t rowb = (uint32_t)(elen * sizeof(T));
-      for (int gi = 0; gi < ngroups; ++gi) {
-        const int n0 = 8 * gi, n1 = min(r, n0 + 8);
-        lk_mbar_arrive_expect_tx(&bar[gi], (uint32_t)(n1 - n0 + (gi == 0 ? M : 0)) * rowb);
-        if (gi == 0)
-          for (int m = 0; m < M; ++m)
-            lk_bulk_g2s(smem_raw + p.off_x + (size_t)m * p.slice * sizeof(T), x + (int64_t)m * p.E + e0, rowb, &bar[0]);
-        for (int n = n0; n < n1; ++n)
-          lk_bulk_g2s(smem_raw + p.off_A + (size_t)n * p.slice * sizeof(T), A + (int64_t)(col0 + n) * p.E + e0, rowb,
-                      &bar[gi]);
-      }
-    }
-    bool ok = true;
-    int waited = 0;  // groups this thread has seen land
-    for (int n = warp; n < r; n += kGemvThreads / 32) {
-      for (; ok && elen > 0 && waited <= n / 8; ++waited) {
-        if (!lk_mbar_wait_bounded(&bar[waited], 0, LK_WAIT_LIMIT_NS)) {
-          ok = false;
-          if (lane == 0) lk_dev_fail(LK_DEV_TIMEOUT_PIPE);
-        }
-      }
-      float facc[MT];
-      int iacc[MT];
+  }
+  __syncthreads();
+  // warps -> (column tile, range of the slice)
+  const int ntiles = (r + 7) / 8;
+  const int wpt = ntiles >= kProjWarps ? 1 : kProjWarps / ntiles;  // warps per tile
+  const int tile = warp / wpt, sub = warp - tile * wpt;
+  const int c = lane >> 2, kp = lane & 3;
+  const int n = 8 * tile + c;  // column of this lane
+  const bool live = tile < ntiles && n < r;
+  float facc[MT];
+  int iacc[MT];
 #pragma unroll
-      for (int i = 0; i < MT; ++i) { facc[i] = 0.0f; iacc[i] = 0; }
-      for (int cc = lane; ok && cc < chunks; cc += 32) {
-        const uint4 wv = *reinterpret_cast<const uint4*>(As + (size_t)n * p.slice + cc * VE);
-        float wf[VE];
-        if (!INT) expand16<XT>(wv, wf);
+  for (int i = 0; i < MT; ++i) { facc[i] = 0.0f; iacc[i] = 0; }
+  if (tile < ntiles) {
+    const int per = (chunks + wpt - 1) / wpt;
+    const int k0 = sub * per, k1 = min(chunks, k0 + per);
+    const T* arow = A + (int64_t)(col0 + (live ? n : 0)) * p.E + e0;
+    constexpr int U = 8;  // loads in flight per lane
+    for (int kc0 = k0 + kp; kc0 < k1; kc0 += 4 * U) {
+      uint4 wv[U];
 #pragma unroll
-        for (int i = 0; i < MT; ++i) {
-          if (i < M) {
-            const uint4 xv4 = *reinterpret_cast<const uint4*>(xs + (size_t)i * p.slice + cc * VE);
-            if (INT) {
-              int a = iacc[i];
-              a = __dp4a((int)xv4.x, (int)wv.x, a);
-              a = __dp4a((int)xv4.y, (int)wv.y, a);
-              a = __dp4a((int)xv4.z, (int)wv.z, a);
-              a = __dp4a((int)xv4.w, (int)wv.w, a);
-              iacc[i] = a;
-            } else {
-              float xf[VE];
-              expand16<XT>(xv4, xf);
-              float a = facc[i];
-#pragma unroll
-              for (int k = 0; k < VE; ++k) a = fmaf(xf[k], wf[k], a);
-              facc[i] = a;
-            }
-          }
-        }
+      for (int u = 0; u < U; ++u) {
+        const int kc = kc0 + 4 * u;
+        wv[u] = (live && kc < k1) ? __ldg(reinterpret_cast<const uint4*>(arow + kc * VE)) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int i = 0; i < MT; ++i) {
-        uint32_t val;
-        if (INT) {
-          int a = iacc[i];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-          val = (uint32_t)a;
-        } else {
-          val = __float_as_uint(lk_warp_sum(facc[i]));
-        }
-        if (i < M) {
-          join();
-          if (lane == 0) mine[n * M + i] = val;
-        }
-      }
-    }
-    // copies of groups no warp waited for (r not a multiple of the warps' stride)
-    // have landed before the CTA may finish
-    for (int gi = waited; ok && elen > 0 && gi < ngroups; ++gi)
-      if (!lk_mbar_wait_bounded(&bar[gi], 0, LK_WAIT_LIMIT_NS)) ok = false;
-  } else
-  for (int cb = warp * kProjNC; cb < r; cb += (kGemvThreads / 32) * kProjNC) {
-    for (int m0 = 0; m0 < M; m0 += MT) {
-      const int mt = min(MT, M - m0);
-      float facc[kProjNC][MT];
-      int iacc[kProjNC][MT];
-#pragma unroll
-      for (int jj = 0; jj < kProjNC; ++jj)
-#pragma unroll
-        for (int i = 0; i < MT; ++i) { facc[jj][i] = 0.0f; iacc[jj][i] = 0; }
-      for (int u0 = 0; u0 < chunks; u0 += 32 * kProjU) {
-        uint4 wv[kProjNC][kProjU];
-#pragma unroll
-        for (int jj = 0; jj < kProjNC; ++jj)
-#pragma unroll
-          for (int u = 0; u < kProjU; ++u) {
-            const int cc = u0 + lane + 32 * u, cl = cb + jj;
-            wv[jj][u] = (cc < chunks && cl < r)
-                            ? __ldg(reinterpret_cast<const uint4*>(A + (int64_t)(col0 + cl) * p.E + e0 + cc * VE))
-                            : make_uint4(0, 0, 0, 0);
-          }
-#pragma unroll
-        for (int u = 0; u < kProjU; ++u) {
-          const int cc = u0 + lane + 32 * u;
-          if (cc < chunks) {
+      for (int u = 0; u < U; ++u) {
+        const int kc = kc0 + 4 * u;
+        if (kc < k1) {
+          if constexpr (INT) {
 #pragma unroll
             for (int i = 0; i < MT; ++i) {
-              if (i < mt) {
-                const uint4 xv4 = __ldg(reinterpret_cast<const uint4*>(x + (int64_t)(m0 + i) * p.E + e0 + cc * VE));
-                if (INT) {
+              if (i < M) {
+                const uint4 xv = *reinterpret_cast<const uint4*>(xi + (size_t)i * p.slice + kc * VE);
+                int a2 = iacc[i];
+                a2 = __dp4a((int)xv.x, (int)wv[u].x, a2);
+                a2 = __dp4a((int)xv.y, (int)wv[u].y, a2);
+                a2 = __dp4a((int)xv.z, (int)wv[u].z, a2);
+                a2 = __dp4a((int)xv.w, (int)wv[u].w, a2);
+                iacc[i] = a2;
+              }
+            }
+          } else {
+            float wf[VE];
+            expand16<XT>(wv[u], wf);
 #pragma unroll
-                  for (int jj = 0; jj < kProjNC; ++jj) {
-                    int a = iacc[jj][i];
-                    a = __dp4a((int)xv4.x, (int)wv[jj][u].x, a);
-                    a = __dp4a((int)xv4.y, (int)wv[jj][u].y, a);
-                    a = __dp4a((int)xv4.z, (int)wv[jj][u].z, a);
-                    a = __dp4a((int)xv4.w, (int)wv[jj][u].w, a);
-                    iacc[jj][i] = a;
-                  }
-                } else {
-                  float xf[VE];
-                  expand16<XT>(xv4, xf);
+            for (int i = 0; i < MT; ++i) {
+              if (i < M) {
+                const float4* xr = reinterpret_cast<const float4*>(xf + (size_t)i * p.slice + kc * VE);
+                float a2 = facc[i];
 #pragma unroll
-                  for (int jj = 0; jj < kProjNC; ++jj) {
-                    float wf[VE];
-                    expand16<XT>(wv[jj][u], wf);
-                    float a = facc[jj][i];
-#pragma unroll
-                    for (int k = 0; k < VE; ++k) a = fmaf(xf[k], wf[k], a);
-                    facc[jj][i] = a;
-                  }
+                for (int k = 0; k < VE / 4; ++k) {
+                  const float4 xv = xr[k];
+                  a2 = fmaf(xv.x, wf[4 * k], a2);
+                  a2 = fmaf(xv.y, wf[4 * k + 1], a2);
+                  a2 = fmaf(xv.z, wf[4 * k + 2], a2);
+                  a2 = fmaf(xv.w, wf[4 * k + 3], a2);
                 }
+                facc[i] = a2;
               }
             }
           }
         }
       }
-#pragma unroll
-      for (int jj = 0; jj < kProjNC; ++jj) {
-#pragma unroll
-        for (int i = 0; i < MT; ++i) {
-          uint32_t val;
-          if (INT) {
-            int a = iacc[jj][i];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-            val = (uint32_t)a;
-          } else {
-            val = __float_as_uint(lk_warp_sum(facc[jj][i]));
-          }
-          join();
-          if (lane == 0 && i < mt && cb + jj < r) mine[(cb + jj) * M + m0 + i] = val;
-        }
-      }
     }
   }
-  join();  // (warps without columns)
+  // the four lanes of a column (k phases 0..3), then the warps of a tile
+  uint32_t* red = reinterpret_cast<uint32_t*>(smem_raw + p.off_red);  // [warp][8 columns][MT]
+#pragma unroll
+  for (int i = 0; i < MT; ++i) {
+    uint32_t val;
+    if (INT) {
+      int a2 = iacc[i];
+      a2 += __shfl_xor_sync(0xffffffffu, a2, 1);
+      a2 += __shfl_xor_sync(0xffffffffu, a2, 2);
+      val = (uint32_t)a2;
+    } else {
+      float a2 = facc[i];
+      a2 += __shfl_xor_sync(0xffffffffu, a2, 1);
+      a2 += __shfl_xor_sync(0xffffffffu, a2, 2);
+      val = __float_as_uint(a2);
+    }
+    if (kp == 0) red[(warp * 8 + c) * MT + i] = val;
+  }
+  __syncthreads();
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // every peer runs: its shared memory may be written
+  for (int idx = threadIdx.x; idx < r * M; idx += kGemvThreads) {
+    const int nn = idx / M, m = idx - nn * M;
+    const int t = nn / 8, cc = nn - 8 * t;
+    uint32_t val;
+    if (INT) {
+      int a2 = 0;
+      for (int s2 = 0; s2 < wpt; ++s2) a2 += (int)red[((t * wpt + s2) * 8 + cc) * MT + m];
+      val = (uint32_t)a2;
+    } else {
+      float a2 = 0.0f;
+      for (int s2 = 0; s2 < wpt; ++s2) a2 += __uint_as_float(red[((t * wpt + s2) * 8 + cc) * MT + m]);
+      val = __float_as_uint(a2);
+    }
+    mine[nn * M + m] = val;
+  }
   cluster.sync();  // every CTA's partials are in rank 0's shared memory
   if (rank != 0) return;
   {
@@ -434,12 +386,12 @@ __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid
         const int d = lane + 32 * q2;
         float val = 0.0f;
         if (d < r) {
-          const int n = col0 + d;
+          const int nn = col0 + d;
           if (INT) {
             int acc = 0;
 #pragma unroll
             for (int q = 0; q < kClusterE; ++q) acc += (int)part[((size_t)q * LK_MAX_RANK + d) * M + m];
-            val = __fmul_rn(__fmul_rn((float)acc, f.x_scale[m]), lk_f16_to_f32(f.a_scale[n]));
+            val = __fmul_rn(__fmul_rn((float)acc, f.x_scale[m]), lk_f16_to_f32(f.a_scale[nn]));
           } else {
 #pragma unroll
             for (int q = 0; q < kClusterE; ++q) val += __uint_as_float(part[((size_t)q * LK_MAX_RANK + d) * M + m]);
@@ -544,16 +496,11 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
     d.E = a.embed_dim;
     d.slice = cluster_slice(a.embed_dim, a.xtype);
     d.done_cnt = static_cast<int32_t*>(a.workspace);
-    size_t smem = (size_t)kClusterE * LK_MAX_RANK * rows * 4;
-    // staged variant: A rows of the widest head and the x rows, one slice each
-    int r_max = 0;
-    for (int j = 0; j < heads_tot; ++j) r_max = std::max(r_max, (int)f.rank[j]);
-    const size_t slice_b = (size_t)d.slice * x_size(a.xtype);
-    d.off_A = round_up((int)smem, 128);
-    d.off_x = d.off_A + round_up((int)(r_max * slice_b), 128);
-    d.off_bar = d.off_x + round_up((int)(rows * slice_b), 16);
-    const bool staged = rows <= 8 && (size_t)d.off_bar + 8 * 8 <= 200 * 1024;
-    if (staged) smem = (size_t)d.off_bar + 8 * 8;  // up to 8 row groups (r <= 64)
+    const size_t xelem = a.xtype == X_I8 ? 1 : 4;  // x slice in shared memory: int8 or fp32
+    d.off_x = round_up(kClusterE * LK_MAX_RANK * rows * 4, 128);
+    d.off_red = d.off_x + round_up((int)(rows * d.slice * xelem), 128);
+    const int mt = rows <= 1 ? 1 : (rows <= 2 ? 2 : (rows <= 4 ? 4 : 8));
+    const size_t smem = (size_t)d.off_red + (size_t)kProjWarps * 8 * mt * 4;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kClusterE, heads_tot, 1);
     cfg.blockDim = dim3(kGemvThreads, 1, 1);
@@ -566,19 +513,13 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const int mt = rows <= 1 ? 1 : (rows <= 2 ? 2 : (rows <= 4 ? 4 : 8));
-#define LK_PROJ_LAUNCH2(XTV, MTV, STV)                                                                   \
+#define LK_PROJ_LAUNCH(XTV, MTV)                                                                        \
   do {                                                                                                \
-    e = cudaFuncSetAttribute(proj_cluster_kernel<XTV, MTV, STV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+    e = cudaFuncSetAttribute(proj_cluster_kernel<XTV, MTV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              (int)smem);                                                             \
     if (e != cudaSuccess) return e;                                                                   \
-    e = cudaLaunchKernelEx(&cfg, proj_cluster_kernel<XTV, MTV, STV>, d);                             \
+    e = cudaLaunchKernelEx(&cfg, proj_cluster_kernel<XTV, MTV>, d);                                  \
     if (e == cudaSuccess) count_launch();                                                             \
-  } while (0)
-#define LK_PROJ_LAUNCH(XTV, MTV)                         \
-  do {                                                   \
-    if (staged) LK_PROJ_LAUNCH2(XTV, MTV, true);         \
-    else LK_PROJ_LAUNCH2(XTV, MTV, false);               \
   } while (0)
 #define LK_PROJ_MT(XTV)                          \
   do {                                           \
@@ -592,7 +533,6 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
     else LK_PROJ_MT(X_I8);
 #undef LK_PROJ_MT
 #undef LK_PROJ_LAUNCH
-#undef LK_PROJ_LAUNCH2
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }

@@ -35,4 +35,5 @@ def pytest_terminal_summary(terminalreporter):
     terminalreporter.write_line(
         f"band rule: {s['codes']} codes compared, {s['flips']} flipped by one at a tie "
         f"(largest distance of a flip from the tie {s['max_flip_tie_distance']:.2e}, allowed 2e-3); "
-        f"largest relative scale deviation {s['max_scale_rel']:.2e} (allowed 1e-4)")
+        f"largest relative int8 scale deviation {s['max_scale_rel']:.2e} (allowed 1e-4); "
+        f"largest int4 fp16 scale difference {s['max_scale_fp16_ulps']:.0f} fp16 ulp (allowed 1)")
