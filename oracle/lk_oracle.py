@@ -53,6 +53,7 @@ __all__ = [
     "attention_materialized", "attention_absorbed", "latent_attention",
     "linear_w8a8_hybrid", "quantize_rows_i8", "rmsnorm", "swiglu",
     "per_head_svd", "round_bf16", "LatentCache", "decoder_layer_w8a8",
+    "hadamard", "latent_rotation", "rotate_latents", "rmsnorm_hadamard",
 ]
 
 FP16_MAX = 65504.0
@@ -365,6 +366,58 @@ def round_bf16(x):
     nan = np.isnan(x32)
     out = rounded.astype(np.uint32).view(np.float32).astype(np.float64)
     return np.where(nan, np.nan, out)
+
+
+# ---------------------------------------------------------------------------
+# Outlier-smoothing rotations (WSVD page §2C: S1 on the activations and S2 on
+# the latent, both orthogonal, applied before RTN; LASER page §3: a rotation
+# between the SVD factors before quantisation).  Orthogonal maps do not change
+# what is computed -- x A = (x S1)(S1^T A), c B = (c S2)(S2^T B) -- only which
+# values get quantised.  Readings: S1 is the normalised Walsh-Hadamard matrix
+# of the activation width (a power of two); S2 is block diagonal, each block
+# the normalised Walsh-Hadamard matrix of order n = the largest power of two
+# dividing r (at most 64).
+# ---------------------------------------------------------------------------
+
+def hadamard(n):
+    """Normalised Walsh-Hadamard matrix of order n (a power of two), by
+    Sylvester's doubling: H_1 = [1], H_2m = [[H_m, H_m], [H_m, -H_m]], then
+    divided by sqrt(n).  Symmetric and orthogonal."""
+    assert n >= 1 and (n & (n - 1)) == 0
+    h = np.ones((1, 1))
+    while h.shape[0] < n:
+        h = np.block([[h, h], [h, -h]])
+    return h / math.sqrt(n)
+
+
+def latent_rotation(r):
+    """S2 for an r-dim latent: block diagonal with blocks hadamard(n), n the
+    largest power of two dividing r, capped at 64."""
+    n = 1
+    while r % (2 * n) == 0 and 2 * n <= 64:
+        n *= 2
+    s2 = np.zeros((r, r))
+    for b0 in range(0, r, n):
+        s2[b0:b0 + n, b0:b0 + n] = hadamard(n)
+    return s2
+
+
+def rotate_latents(v, ranks):
+    """Each head's latent v^h (consecutive blocks of v [..., sum ranks]) times
+    its S2, in float64, rounded once to float32 (what gets quantised)."""
+    v = np.asarray(v, np.float64)
+    out = np.empty_like(v)
+    off = 0
+    for r in ranks:
+        out[..., off:off + r] = v[..., off:off + r] @ latent_rotation(r)
+        off += r
+    return out.astype(np.float32)
+
+
+def rmsnorm_hadamard(x, eps=1e-5):
+    """S1 after the pre-norm: RMSNorm(x) times hadamard(k), k = the row width."""
+    x = rmsnorm(x, eps)
+    return x @ hadamard(x.shape[-1])
 
 
 # ---------------------------------------------------------------------------

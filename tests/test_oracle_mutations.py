@@ -43,6 +43,10 @@ MUTANTS = {
      "    attn = round_bf16(attn.reshape(Bsz, n_h * H))"),
  "layer_no_attn_residual": ("layer[\"s_O\"], residual=x))", "layer[\"s_O\"], residual=None))"),
  "layer_ffn_residual_x": ("d[\"s_V\"], residual=x2)", "d[\"s_V\"], residual=x)"),
+ "hadamard_unnormalised": ("    return h / math.sqrt(n)", "    return h"),
+ "rotation_block_cap_32": ("    while r % (2 * n) == 0 and 2 * n <= 64:", "    while r % (2 * n) == 0 and 2 * n <= 32:"),
+ "rotate_latents_skips_head": ("        out[..., off:off + r] = v[..., off:off + r] @ latent_rotation(r)",
+                               "        out[..., off:off + r] = v[..., off:off + r] @ latent_rotation(r) if off else v[..., :r]"),
  "layer_q_from_x": ("q = round_bf16(_linear_dense_w8a8(xq, sx, layer[\"W_Q\"], layer[\"s_Q\"]))",
                     "q = round_bf16(_linear_dense_w8a8(*quantize_rows_i8(x.astype(np.float32)), layer[\"W_Q\"], layer[\"s_Q\"]))"),
 }

@@ -500,3 +500,71 @@ def test_decoder_layer_tiny_worked():
     for cache, (code, scale) in ((ck, exp["k_new"]), (cv, exp["v_new"])):
         assert int(cache.codes[0][0][1, 0]) == code
         assert np.float32(cache.scales[0][0][1]).view(np.uint32) == np.float32(float.fromhex(scale)).view(np.uint32)
+
+
+# ---------------------------------------------------------------- rotations (S1, S2)
+
+@pytest.mark.parametrize("n", [1, 2, 8, 64, 4096])
+def test_hadamard_closed_form_and_orthogonal(n):
+    """Sylvester-Hadamard entries are (-1)^popcount(i & j) / sqrt(n); the
+    matrix is symmetric and orthogonal."""
+    h = O.hadamard(n)
+    if n <= 64:
+        i = np.arange(n)[:, None]
+        j = np.arange(n)[None, :]
+        parity = np.vectorize(lambda a: bin(int(a)).count("1") & 1)(i & j)
+        np.testing.assert_array_equal(h * math.sqrt(n), np.where(parity, -1.0, 1.0))
+    np.testing.assert_allclose(h @ h.T, np.eye(n), atol=1e-12)
+    np.testing.assert_array_equal(h, h.T)
+
+
+@pytest.mark.parametrize("r,block", [(8, 8), (16, 16), (24, 8), (32, 32), (48, 16), (64, 64), (12, 4), (4, 4)])
+def test_latent_rotation_blocks(r, block):
+    s2 = O.latent_rotation(r)
+    np.testing.assert_allclose(s2 @ s2.T, np.eye(r), atol=1e-12)
+    for b0 in range(0, r, block):
+        np.testing.assert_allclose(s2[b0:b0 + block, b0:b0 + block], O.hadamard(block))
+        mask = np.ones(r, bool)
+        mask[b0:b0 + block] = False
+        assert np.all(s2[b0:b0 + block][:, mask] == 0)
+
+
+def test_rotations_leave_attention_unchanged():
+    """With the cache rotated (C S2) and the factor counter-rotated (S2^T B),
+    materialised attention is the same (no quantisation in between)."""
+    rng = np.random.default_rng(9)
+    T, r, H = 37, 24, 16
+    C, Cv = rng.standard_normal((T, r)), rng.standard_normal((T, r))
+    BK, BV = rng.standard_normal((r, H)), rng.standard_normal((r, H))
+    q = rng.standard_normal(H)
+    s2 = O.latent_rotation(r)
+    a = O.attention_materialized(q, C, Cv, BK, BV, 0.3)
+    b = O.attention_materialized(q, C @ s2, Cv @ s2, s2.T @ BK, s2.T @ BV, 0.3)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
+    x = rng.standard_normal((3, 64))
+    A = rng.standard_normal((64, 24))
+    h = O.hadamard(64)
+    np.testing.assert_allclose((x @ h) @ (h.T @ A), x @ A, atol=1e-12)
+
+
+def test_rotate_latents_and_rmsnorm_hadamard_brute_force():
+    rng = np.random.default_rng(10)
+    ranks = [24, 8, 16]
+    v = rng.standard_normal((2, sum(ranks))).astype(np.float32)
+    got = O.rotate_latents(v, ranks)
+    off = 0
+    for r in ranks:
+        n = r & -r if (r & -r) <= 64 else 64
+        for row in range(2):
+            for d in range(r):
+                blk = (d // n) * n
+                acc = sum(float(v[row, off + blk + i]) * (-1) ** bin(i & (d - blk)).count("1") for i in range(n))
+                assert got[row, off + d] == np.float32(acc / math.sqrt(n))
+        off += r
+    x = rng.standard_normal((2, 8))
+    y = O.rmsnorm_hadamard(x, 1e-5)
+    xn = x / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + 1e-5)
+    for row in range(2):
+        for j in range(8):
+            want = sum(xn[row, i] * (-1) ** bin(i & j).count("1") for i in range(8)) / math.sqrt(8)
+            assert abs(y[row, j] - want) < 1e-12
