@@ -36,7 +36,8 @@ design notes):
   of a row may be shorter when g does not divide r.  Packing: low nibble holds
   the even dim, high nibble the odd dim, both two's complement.
 * No positional encoding (neither page mentions one), so the absorbed form
-  (q B_K^T) C^T equals the materialised one.
+  (q B_K^T) C^T equals the materialised one.  The rotary extension below
+  (attention_rope) is a separate path with its own readings.
 * Attention over positions [0, len) where len already counts the token
   appended in the same step.
 """
@@ -54,6 +55,7 @@ __all__ = [
     "linear_w8a8_hybrid", "quantize_rows_i8", "rmsnorm", "swiglu",
     "per_head_svd", "round_bf16", "LatentCache", "decoder_layer_w8a8",
     "hadamard", "latent_rotation", "rotate_latents", "rmsnorm_hadamard",
+    "rope_angles", "rope", "attention_rope", "latent_attention_rope",
 ]
 
 FP16_MAX = 65504.0
@@ -418,6 +420,70 @@ def rmsnorm_hadamard(x, eps=1e-5):
     """S1 after the pre-norm: RMSNorm(x) times hadamard(k), k = the row width."""
     x = rmsnorm(x, eps)
     return x @ hadamard(x.shape[-1])
+
+
+# ---------------------------------------------------------------------------
+# Rotary positions (an extension: neither page mentions positional encoding).
+# The WSVD page's fused kernel rebuilds K_h on chip from the latent (§2C);
+# with a rotary position encoding that rebuild is required, since the
+# rotation of each key depends on its position and q can no longer be folded
+# into B_K.  Readings: rotate-half pairs (dim i with dim i + H/2), frequencies
+# theta_i = base^(-2 i / H) with base 10000, keys at their cache positions
+# 0 .. len - 1, the query at the position of the newest cached token
+# (len - 1), values not rotated (so V keeps the latent form).
+# ---------------------------------------------------------------------------
+
+def rope_angles(positions, H, base=10000.0):
+    """angle[t, i] = positions[t] * base^(-2 i / H) for i < H / 2 (float64)."""
+    i = np.arange(H // 2, dtype=np.float64)
+    theta = float(base) ** (-2.0 * i / H)
+    return np.asarray(positions, np.float64)[:, None] * theta[None, :]
+
+
+def rope(x, positions, base=10000.0):
+    """Rotate-half rotary encoding of rows x [T, H] at positions [T]: for each
+    i < H/2 the pair (x_i, x_{i+H/2}) is turned by angle[t, i]."""
+    x = np.asarray(x, np.float64)
+    H = x.shape[-1]
+    h = H // 2
+    ang = rope_angles(positions, H, base)
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = x[:, :h], x[:, h:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=1)
+
+
+def attention_rope(q, Ck_hat, Cv_hat, B_K, B_V, softmax_scale, q_pos, base=10000.0, k_pos0=0):
+    """Attention of one (batch, head) with rotary keys and query.
+
+    K = Ck_hat B_K rebuilt, each row t rotated at position k_pos0 + t; q
+    rotated at q_pos; s = K_rot q_rot * scale; o = softmax(s) (Cv_hat B_V).
+    """
+    K = np.asarray(Ck_hat, np.float64) @ np.asarray(B_K, np.float64)   # rebuilt keys [T, H]
+    V = np.asarray(Cv_hat, np.float64) @ np.asarray(B_V, np.float64)   # values [T, H]
+    T = K.shape[0]
+    K_rot = rope(K, k_pos0 + np.arange(T), base)
+    q_rot = rope(np.asarray(q, np.float64)[None, :], [q_pos], base)[0]
+    s = (K_rot @ q_rot) * float(softmax_scale)
+    s = s - np.max(s)
+    p = np.exp(s)
+    p = p / np.sum(p)
+    return p @ V
+
+
+def latent_attention_rope(q, cache_k, cache_v, B_K_heads, B_V_heads, softmax_scale, base=10000.0):
+    """attention_rope for every (b, h) over the whole cache; the query of row
+    b sits at position len_b - 1.  Returns o: [B, n_h, H] float64."""
+    q = np.asarray(q, np.float64)
+    Bsz, n_h, H = q.shape
+    out = np.zeros((Bsz, n_h, H), np.float64)
+    for b in range(Bsz):
+        T = cache_k.length(b)
+        if T == 0:
+            continue
+        for h in range(n_h):
+            out[b, h] = attention_rope(q[b, h], cache_k.dequant(b, h), cache_v.dequant(b, h),
+                                       B_K_heads[h], B_V_heads[h], softmax_scale, T - 1, base)
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -47,6 +47,13 @@ MUTANTS = {
  "rotation_block_cap_32": ("    while r % (2 * n) == 0 and 2 * n <= 64:", "    while r % (2 * n) == 0 and 2 * n <= 32:"),
  "rotate_latents_skips_head": ("        out[..., off:off + r] = v[..., off:off + r] @ latent_rotation(r)",
                                "        out[..., off:off + r] = v[..., off:off + r] @ latent_rotation(r) if off else v[..., :r]"),
+ "rope_interleaved_pairs": ("    x1, x2 = x[:, :h], x[:, h:]\n    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=1)",
+                            "    x1, x2 = x[:, 0::2], x[:, 1::2]\n    return np.stack([x1 * c - x2 * s, x2 * c + x1 * s], axis=2).reshape(x.shape)"),
+ "rope_sign": ("x2 * c + x1 * s], axis=1)", "x2 * c - x1 * s], axis=1)"),
+ "rope_freq_exponent": ("theta = float(base) ** (-2.0 * i / H)", "theta = float(base) ** (-1.0 * i / H)"),
+ "rope_query_unrotated": ("    q_rot = rope(np.asarray(q, np.float64)[None, :], [q_pos], base)[0]",
+                          "    q_rot = np.asarray(q, np.float64)"),
+ "rope_query_at_len": ("softmax_scale, T - 1, base)", "softmax_scale, T, base)"),
  "layer_q_from_x": ("q = round_bf16(_linear_dense_w8a8(xq, sx, layer[\"W_Q\"], layer[\"s_Q\"]))",
                     "q = round_bf16(_linear_dense_w8a8(*quantize_rows_i8(x.astype(np.float32)), layer[\"W_Q\"], layer[\"s_Q\"]))"),
 }

@@ -568,3 +568,102 @@ def test_rotate_latents_and_rmsnorm_hadamard_brute_force():
         for j in range(8):
             want = sum(xn[row, i] * (-1) ** bin(i & j).count("1") for i in range(8)) / math.sqrt(8)
             assert abs(y[row, j] - want) < 1e-12
+
+
+# ---------------------------------------------------------------- rotary positions (extension)
+
+def test_rope_unit_vectors_closed_form():
+    """H = 8, base 10000: theta_i = 10^-i.  e_i at position p turns into
+    cos(p theta_i) e_i + sin(p theta_i) e_{i+4}; e_{i+4} into
+    cos(p theta_i) e_{i+4} - sin(p theta_i) e_i."""
+    H, p = 8, 3
+    for i in range(4):
+        th = 10.0 ** (-i)
+        e = np.zeros((1, H))
+        e[0, i] = 1.0
+        want = np.zeros(H)
+        want[i], want[i + 4] = math.cos(p * th), math.sin(p * th)
+        np.testing.assert_allclose(O.rope(e, [p])[0], want, atol=1e-15)
+        e = np.zeros((1, H))
+        e[0, i + 4] = 1.0
+        want = np.zeros(H)
+        want[i + 4], want[i] = math.cos(p * th), -math.sin(p * th)
+        np.testing.assert_allclose(O.rope(e, [p])[0], want, atol=1e-15)
+    # position 0 is the identity
+    x = np.random.default_rng(1).standard_normal((3, 16))
+    np.testing.assert_array_equal(O.rope(x, [0, 0, 0]), x)
+
+
+def test_rope_scores_depend_on_offset_only():
+    """<R_m q, R_n k> = <q, R_{n-m} k>: block rotation matrices built
+    explicitly (2 x 2 per frequency pair), positions shifted together leave
+    every score unchanged, and the rotation keeps norms."""
+    rng = np.random.default_rng(2)
+    H = 16
+    q, k = rng.standard_normal(H), rng.standard_normal(H)
+
+    def rot(pos):
+        R = np.zeros((H, H))
+        for i in range(H // 2):
+            a = pos * 10000.0 ** (-2.0 * i / H)
+            R[i, i], R[i, i + H // 2] = math.cos(a), -math.sin(a)
+            R[i + H // 2, i], R[i + H // 2, i + H // 2] = math.sin(a), math.cos(a)
+        return R
+
+    for m, n in ((0, 5), (7, 3), (1000, 16383)):
+        s = O.rope(q[None], [m])[0] @ O.rope(k[None], [n])[0]
+        assert abs(s - q @ (rot(n - m) @ k)) < 1e-9 * (1 + abs(s))
+        np.testing.assert_allclose(O.rope(k[None], [n])[0], rot(n) @ k, atol=1e-12)
+        assert abs(np.linalg.norm(O.rope(k[None], [n])[0]) - np.linalg.norm(k)) < 1e-12
+
+
+def test_attention_rope_brute_force_and_shift_invariance():
+    rng = np.random.default_rng(3)
+    T, r, H = 5, 4, 8
+    Ck, Cv = rng.standard_normal((T, r)), rng.standard_normal((T, r))
+    BK, BV = rng.standard_normal((r, H)), rng.standard_normal((r, H))
+    q = rng.standard_normal(H)
+    got = O.attention_rope(q, Ck, Cv, BK, BV, 0.4, q_pos=T - 1)
+    # brute force: explicit per-pair rotations, scores, softmax, weighted V rows
+    scores = []
+    for t in range(T):
+        kt = Ck[t] @ BK
+        acc = 0.0
+        for i in range(H // 2):
+            th = 10000.0 ** (-2.0 * i / H)
+            ck, sk = math.cos(t * th), math.sin(t * th)
+            cq, sq = math.cos((T - 1) * th), math.sin((T - 1) * th)
+            k1, k2 = kt[i] * ck - kt[i + 4] * sk, kt[i + 4] * ck + kt[i] * sk
+            q1, q2 = q[i] * cq - q[i + 4] * sq, q[i + 4] * cq + q[i] * sq
+            acc += k1 * q1 + k2 * q2
+        scores.append(0.4 * acc)
+    w = [math.exp(s - max(scores)) for s in scores]
+    want = sum(wt * (Cv[t] @ BV) for t, wt in enumerate(w)) / sum(w)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    # shifting every position by the same amount changes nothing
+    shifted = O.attention_rope(q, Ck, Cv, BK, BV, 0.4, q_pos=T - 1 + 700, k_pos0=700)
+    np.testing.assert_allclose(shifted, got, rtol=1e-9, atol=1e-12)
+    # one token: the output is its value row whatever the rotation
+    np.testing.assert_allclose(O.attention_rope(q, Ck[:1], Cv[:1], BK, BV, 0.4, q_pos=9), Cv[0] @ BV, atol=1e-12)
+
+
+def test_latent_attention_rope_query_at_last_position():
+    rng = np.random.default_rng(4)
+    ranks, H = [8, 16], 16
+    lens = [6, 0, 3]
+    ck, cv = O.LatentCache(3, ranks, "i8", 32), O.LatentCache(3, ranks, "i8", 32)
+    for b, L in enumerate(lens):
+        ck.append(b, [O.quantize_i8(rng.standard_normal((L, r)).astype(np.float32)) for r in ranks])
+        cv.append(b, [O.quantize_i8(rng.standard_normal((L, r)).astype(np.float32)) for r in ranks])
+    BK = [rng.standard_normal((r, H)) for r in ranks]
+    BV = [rng.standard_normal((r, H)) for r in ranks]
+    q = rng.standard_normal((3, 2, H))
+    out = O.latent_attention_rope(q, ck, cv, BK, BV, 0.25)
+    assert np.all(out[1] == 0)
+    for b in (0, 2):
+        for h in range(2):
+            want = O.attention_rope(q[b, h], ck.dequant(b, h), cv.dequant(b, h), BK[h], BV[h], 0.25, lens[b] - 1)
+            np.testing.assert_array_equal(out[b, h], want)
+            # at position 0 of a one-token-shorter window the scores differ: the query position matters
+            other = O.attention_rope(q[b, h], ck.dequant(b, h), cv.dequant(b, h), BK[h], BV[h], 0.25, 0)
+            assert not np.allclose(other, want)
