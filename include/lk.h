@@ -109,7 +109,21 @@ typedef struct {
   const int32_t* ranks; /* HOST [n_heads]                                   */
   void* codes;          /* device, 256-byte aligned                        */
   void* scales;         /* device, 256-byte aligned                        */
+  int32_t rotation;     /* 0 or 1; see below                                */
 } lk_latent_cache;
+
+/*
+ * rotation = 1 (WSVD §2C: an orthogonal S2 applied to the latent smooths its
+ * outlier channels before round-to-nearest): lk_latent_project_append
+ * multiplies each head's fp32 latent v^h by S2_h before quantising it, where
+ * S2_h is block diagonal with normalised Walsh-Hadamard blocks of order n =
+ * the largest power of two dividing r_h, capped at 64 (S2_h = S2_h^T =
+ * S2_h^-1).  The cache then holds codes of v^h S2_h; since
+ * (v S2)(S2 B) = v B, the decode entry points stay unchanged when they are
+ * given the counter-rotated factors S2_h B_K^h and S2_h B_V^h.  Folding S2
+ * into A offline (A^h S2_h) gives the same cache without this flag.  Only
+ * the append reads the flag; 0 is the plain cache.
+ */
 
 /* Bytes the caller must allocate for a cache's code and scale planes. */
 lk_status lk_latent_cache_bytes(const lk_latent_cache* cache, size_t* codes_bytes,
@@ -134,7 +148,7 @@ lk_status lk_latent_cache_bytes(const lk_latent_cache* cache, size_t* codes_byte
  *   n_new once every token is written.  seq_len_host: HOST copy of the same
  *   values, used for the capacity check seq_len + n_new <= capacity.
  * workspace: lk_latent_project_workspace_bytes(...) bytes, 256-B aligned;
- *   its first 256 bytes are an arrival counter that must be zero before the
+ *   its first 2048 bytes are arrival counters that must be zero before the
  *   first call and that every completed call leaves zero.
  */
 lk_status lk_latent_project_append(const lk_latent_cache* k_cache, const lk_latent_cache* v_cache,
@@ -271,12 +285,54 @@ lk_status lk_dense_decode_attn(const void* q, const void* K, const void* V, int3
 size_t lk_dense_decode_workspace_bytes(int32_t batch, int32_t n_heads, int32_t head_dim, int32_t max_seq_len);
 
 /*
+ * Rotary positions (an extension: neither page uses a positional encoding).
+ *
+ * lk_rope_table: table[t][i] = (cos a, sin a), a = t * base^(-2 i / head_dim),
+ * for t < max_pos and i < head_dim / 2, computed in float64 and stored fp32
+ * ([max_pos][head_dim / 2][2], device, written on `stream`).  base > 1.
+ *
+ * lk_latent_decode_attn_rope: latent decode attention for a model that
+ * rotates keys and queries (rotate-half pairs (i, i + H/2)).  The rotation
+ * of a key depends on its position, so q cannot be absorbed into B_K: each
+ * key is rebuilt from its latent code on chip (the WSVD page's fused kernel
+ * rebuilds K_h on chip, technical summary §2C).  For batch row b, head h,
+ * positions t < len = min(seq_len[b], max_seq_len):
+ *   K_t = dequant(c_K[t]) B_K^h, rotated by the table row t;
+ *   q rotated by the table row len - 1 (the newest cached position);
+ *   s_t = (rot q) . (rot K_t) * softmax_scale;  p = softmax(s);
+ *   out = (sum_t p_t dequant(c_V[t])) B_V^h   (values are not rotated).
+ * Caches and their layouts as for lk_latent_decode_attn (the rotation flag
+ * of a cache is not read here).  q: [B, n_heads, head_dim] LK_F32 or
+ * LK_BF16; B_K, B_V: bf16 (b_dtype LK_BF16), packed per head as for
+ * lk_latent_decode_attn; head_dim a multiple of 32 (<= LK_MAX_HEAD_DIM);
+ * rope_table: an lk_rope_table table of the same head_dim with at least
+ * max_seq_len rows; q, B_K, B_V, rope_table 16-byte aligned.  out:
+ * [B, n_heads, head_dim] LK_F32 or LK_BF16; rows with len = 0 are zero.
+ * workspace: lk_latent_decode_rope_workspace_bytes(...) bytes, 256-byte
+ * aligned, its first round_up(4 * B * n_heads, 256) bytes zero at entry
+ * (left zero by every completed call).  The keys are rebuilt with exact
+ * bf16 products summed in fp32; everything after is fp32.
+ */
+lk_status lk_rope_table(int32_t head_dim, int32_t max_pos, float base, float* table, lk_stream_t stream);
+lk_status lk_latent_decode_attn_rope(const lk_latent_cache* k_cache, const lk_latent_cache* v_cache,
+                                     const void* q, lk_dtype q_dtype, const void* B_K, const void* B_V,
+                                     lk_dtype b_dtype, int32_t head_dim, const int32_t* seq_len,
+                                     int32_t max_seq_len, const float* rope_table, float softmax_scale,
+                                     void* out, lk_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                     lk_stream_t stream);
+size_t lk_latent_decode_rope_workspace_bytes(const lk_latent_cache* k_cache, const lk_latent_cache* v_cache,
+                                             int32_t head_dim, int32_t max_seq_len);
+
+/*
  * The naive low-rank path the WSVD page contrasts with its fused kernel
  * (technical summary §1: rebuilding K and V from the factors through
  * memory costs more than it saves): for positions [0, seq_len[b]),
  *   K_out[b, h, t, :] = dequant(c_K[b, h, t]) B_K^h,  V_out likewise,
  * stored bf16 [B, n_heads, capacity, head_dim] (rows past seq_len[b] are not
- * written).  Caches, B_K / B_V and their layouts as for lk_latent_decode_attn.
+ * written).  Caches and their layouts as for lk_latent_decode_attn; B_K and
+ * B_V bf16 (b_dtype LK_BF16, else LK_ERR_DTYPE), 16-byte aligned; head_dim a
+ * multiple of 16.  Each value is the fp32 sum of exact code x factor
+ * products (per scale group, times the group's scale), rounded once to bf16.
  * Attending the result with lk_dense_decode_attn gives the same output as
  * lk_latent_decode_attn up to the bf16 rounding of K and V.
  */
@@ -345,6 +401,18 @@ lk_status lk_quantize_rows_i8(const void* x, lk_dtype x_dtype, int32_t m, int32_
 /* RMSNorm with unit weight, y = x / sqrt(mean(x^2) + eps), then per-row int8
  * quantisation of y (fp32).  x: [m, k] LK_F32 or LK_BF16. */
 lk_status lk_rmsnorm_quant_i8(const void* x, lk_dtype x_dtype, int32_t m, int32_t k, float eps,
+                              int8_t* x_q, float* x_scale, lk_stream_t stream);
+
+/* S1 on the input of the latent projection (WSVD §2C: S1 is a Hadamard
+ * matrix applied to the input to smooth its outlier channels):
+ * y = RMSNorm(x) H_k with H_k the normalised Walsh-Hadamard matrix of order
+ * k (k a power of two, <= 32768), then per-row int8 quantisation of y as in
+ * lk_quantize_rows_i8.  The projection weight must then be H_k A (H_k is
+ * symmetric and orthogonal), so y (H_k A) = RMSNorm(x) A.  The transform is
+ * fp32 butterflies (log2 k adds per element, then one multiply by
+ * fl32(1 / sqrt(k))).  x: [m, k] LK_F32 or LK_BF16; x_q int8 [m, k];
+ * x_scale fp32 [m].  LK_ERR_SHAPE when k is not a power of two. */
+lk_status lk_rmsnorm_hadamard_quant_i8(const void* x, lk_dtype x_dtype, int32_t m, int32_t k, float eps,
                               int8_t* x_q, float* x_scale, lk_stream_t stream);
 
 /* SwiGLU h = silu(gate) * up in fp32 (LASER §4 fuses it into the FFN), then

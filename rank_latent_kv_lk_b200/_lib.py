@@ -40,6 +40,7 @@ class LatentCacheDesc(C.Structure):
         ("ranks", C.POINTER(C.c_int32)),
         ("codes", C.c_void_p),
         ("scales", C.c_void_p),
+        ("rotation", C.c_int32),
     ]
 
 
@@ -97,11 +98,16 @@ def _load():
         "lk_dense_decode_attn": (C.c_int, [P, P, P, I32, I32, I32, I32, P, I32, C.c_float, P, C.c_int, P, SZ, P]),
         "lk_dense_decode_workspace_bytes": (SZ, [I32, I32, I32, I32]),
         "lk_latent_reconstruct_kv": (C.c_int, [CP, CP, P, P, C.c_int, I32, P, I32, P, P, P]),
+        "lk_rope_table": (C.c_int, [I32, I32, C.c_float, P, P]),
+        "lk_latent_decode_attn_rope": (C.c_int, [CP, CP, P, C.c_int, P, P, C.c_int, I32, P, I32, P, C.c_float, P,
+                                                 C.c_int, P, SZ, P]),
+        "lk_latent_decode_rope_workspace_bytes": (SZ, [CP, CP, I32, I32]),
         "lk_lowrank_linear": (C.c_int, [WP, P, P, I32, P, P, C.c_int, P, P, P, SZ, P]),
         "lk_lowrank_workspace_bytes": (SZ, [WP, I32]),
         "lk_quantize_latent": (C.c_int, [P, I32, I32, C.c_int, I32, P, P, P]),
         "lk_quantize_rows_i8": (C.c_int, [P, C.c_int, I32, I32, P, P, P]),
         "lk_rmsnorm_quant_i8": (C.c_int, [P, C.c_int, I32, I32, C.c_float, P, P, P]),
+        "lk_rmsnorm_hadamard_quant_i8": (C.c_int, [P, C.c_int, I32, I32, C.c_float, P, P, P]),
         "lk_swiglu_quant_i8": (C.c_int, [P, P, C.c_int, I32, I32, P, P, P]),
         "lk_device_status": (C.c_int, [I32]),
     }

@@ -57,8 +57,10 @@ workspaces = _WorkspacePool()
 class LatentCache:
     """Device latent cache of one layer for K or V (codes + scales planes)."""
 
-    def __init__(self, batch, ranks, capacity, kind="i8", group=32, device="cuda", role="k"):
-        """role: 'k' or 'v' -- the two caches of a layer lay codes out differently."""
+    def __init__(self, batch, ranks, capacity, kind="i8", group=32, device="cuda", role="k", rotation=False):
+        """role: 'k' or 'v' -- the two caches of a layer lay codes out differently.
+        rotation: the append multiplies each head's latent by its block-Hadamard
+        S2 before quantising (decode then takes the factors S2 B)."""
         if kind not in ("i8", "i4"):
             raise ValueError("kind must be 'i8' or 'i4'")
         self.role = role
@@ -69,7 +71,9 @@ class LatentCache:
                                   dtype=torch.float32 if kind == "i8" else torch.float16, device=device)
         self._ranks = (C.c_int32 * len(self.ranks))(*self.ranks)
         self._desc = LatentCacheDesc(batch, len(self.ranks), capacity, LK_I8 if kind == "i8" else LK_I4,
-                                     group, self._ranks, self.codes.data_ptr(), self.scales.data_ptr())
+                                     group, self._ranks, self.codes.data_ptr(), self.scales.data_ptr(),
+                                     1 if rotation else 0)
+        self.rotation = bool(rotation)
 
     @property
     def n_heads(self):
@@ -183,6 +187,32 @@ def dense_decode_attn(q, K, V, seq_len, max_seq_len, softmax_scale=None, out=Non
     return out
 
 
+def rope_table(head_dim, max_pos, base=10000.0, device="cuda", stream=None):
+    """cos / sin of t * base^(-2 i / head_dim): fp32 [max_pos, head_dim / 2, 2]."""
+    table = torch.empty((max_pos, head_dim // 2, 2), dtype=torch.float32, device=device)
+    check(lib.lk_rope_table(int(head_dim), int(max_pos), float(base), _ptr(table), _stream(stream)))
+    return table
+
+
+def latent_decode_attn_rope(k_cache, v_cache, q, B_K, B_V, seq_len, max_seq_len, table, softmax_scale=None,
+                            out=None, out_dtype=None, stream=None):
+    """Decode attention with rotary keys and query: keys rebuilt from the latent
+    codes on chip and rotated at their positions, the query at the newest
+    position (seq_len - 1); values in latent form.  B_K / B_V bf16."""
+    H = q.shape[-1]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(H)
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    need = lib.lk_latent_decode_rope_workspace_bytes(k_cache.desc(), v_cache.desc(), H, int(max_seq_len))
+    ws = workspaces.get(("rope", k_cache.batch * len(k_cache.ranks)), need, q.device)
+    check(lib.lk_latent_decode_attn_rope(
+        k_cache.desc(), v_cache.desc(), _ptr(q), _dtype_code(q), _ptr(B_K), _ptr(B_V), _dtype_code(B_K), H,
+        _ptr(seq_len), int(max_seq_len), _ptr(table), float(softmax_scale), _ptr(out), _dtype_code(out),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
 def reconstruct_kv(k_cache, v_cache, B_K, B_V, seq_len, max_seq_len, head_dim, K_out=None, V_out=None, stream=None):
     """The naive path: K, V rebuilt from the latent cache into bf16 [B, heads, capacity, H]."""
     shape = (k_cache.batch, len(k_cache.ranks), k_cache.capacity, head_dim)
@@ -250,6 +280,17 @@ def rmsnorm_quant_i8(x, eps=1e-5, stream=None):
     q = torch.empty((m, k), dtype=torch.int8, device=x.device)
     s = torch.empty((m,), dtype=torch.float32, device=x.device)
     check(lib.lk_rmsnorm_quant_i8(_ptr(x), _dtype_code(x), m, k, float(eps), _ptr(q), _ptr(s), _stream(stream)))
+    return q, s
+
+
+def rmsnorm_hadamard_quant_i8(x, eps=1e-5, stream=None):
+    """RMSNorm, then the normalised Walsh-Hadamard transform of each row (S1),
+    then per-row int8 quantisation; the row width must be a power of two."""
+    m, k = x.shape
+    q = torch.empty((m, k), dtype=torch.int8, device=x.device)
+    s = torch.empty((m,), dtype=torch.float32, device=x.device)
+    check(lib.lk_rmsnorm_hadamard_quant_i8(_ptr(x), _dtype_code(x), m, k, float(eps), _ptr(q), _ptr(s),
+                                           _stream(stream)))
     return q, s
 
 

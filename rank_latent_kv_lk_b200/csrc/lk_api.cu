@@ -1,5 +1,7 @@
 // C ABI: host-side validation and dispatch for every entry point in lk.h.
 // Nothing is launched and nothing is written unless every check passes.
+#include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -66,6 +68,7 @@ lk_status check_cache(const lk_latent_cache* c, const char* name, bool need_buff
   if (c->code_dtype == LK_I4 && (c->group < 8 || c->group % 8 != 0))
     return fail(LK_ERR_SHAPE, "%s: int4 group %d must be a positive multiple of 8", name, c->group);
   if (!c->ranks) return fail(LK_ERR_INVALID_ARG, "%s: null ranks", name);
+  if (c->rotation != 0 && c->rotation != 1) return fail(LK_ERR_INVALID_ARG, "%s: rotation must be 0 or 1", name);
   const int mult = c->code_dtype == LK_I8 ? 4 : 8;
   for (int h = 0; h < c->n_heads; ++h) {
     const int r = c->ranks[h];
@@ -182,8 +185,8 @@ lk_status lk_latent_project_append(const lk_latent_cache* k, const lk_latent_cac
   if (!aligned(workspace, 256)) return fail(LK_ERR_ALIGN, "workspace must be 256-byte aligned");
 
   lk::ProjectLaunch a{};
-  a.k = {k->codes, k->scales, k->code_dtype == LK_I8 ? 0 : 1, k->group, k->n_heads, k->capacity};
-  a.v = {v->codes, v->scales, v->code_dtype == LK_I8 ? 0 : 1, v->group, v->n_heads, v->capacity};
+  a.k = {k->codes, k->scales, k->code_dtype == LK_I8 ? 0 : 1, k->group, k->n_heads, k->capacity, k->rotation};
+  a.v = {v->codes, v->scales, v->code_dtype == LK_I8 ? 0 : 1, v->group, v->n_heads, v->capacity, v->rotation};
   a.ranks_k = k->ranks;
   a.ranks_v = v->ranks;
   a.x = x;
@@ -377,6 +380,101 @@ lk_status lk_dense_decode_attn(const void* q, const void* K, const void* V, int3
   return LK_OK;
 }
 
+lk_status lk_rope_table(int32_t head_dim, int32_t max_pos, float base, float* table, lk_stream_t stream) {
+  if (head_dim < 2 || head_dim > LK_MAX_HEAD_DIM || head_dim % 2 != 0)
+    return fail(LK_ERR_SHAPE, "head_dim %d must be even in [2, %d]", head_dim, LK_MAX_HEAD_DIM);
+  if (max_pos < 0) return fail(LK_ERR_SHAPE, "max_pos %d < 0", max_pos);
+  if (!(base > 1.0f) || !std::isfinite(base)) return fail(LK_ERR_INVALID_ARG, "base must be finite and > 1");
+  if (max_pos > 0 && !table) return fail(LK_ERR_INVALID_ARG, "null table");
+  cudaError_t e = lk::launch_rope_table(table, head_dim, max_pos, (double)base, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lk_rope_table");
+  return LK_OK;
+}
+
+namespace {
+lk_status rope_check(const lk_latent_cache* k, const lk_latent_cache* v, int32_t head_dim, int32_t max_seq_len) {
+  lk_status s;
+  if ((s = check_cache(k, "k_cache", true)) != LK_OK) return s;
+  if ((s = check_cache(v, "v_cache", true)) != LK_OK) return s;
+  if (k->batch != v->batch || k->n_heads != v->n_heads || k->capacity != v->capacity)
+    return fail(LK_ERR_SHAPE, "k and v caches differ in batch, heads or capacity");
+  if (k->code_dtype != v->code_dtype) return fail(LK_ERR_UNSUPPORTED, "k and v caches differ in code dtype");
+  if (head_dim < 32 || head_dim > LK_MAX_HEAD_DIM || head_dim % 32 != 0)
+    return fail(LK_ERR_SHAPE, "head_dim %d must be a multiple of 32 in [32, %d]", head_dim, LK_MAX_HEAD_DIM);
+  if (max_seq_len < 0 || max_seq_len > k->capacity)
+    return fail(LK_ERR_SHAPE, "max_seq_len %d outside [0, capacity]", max_seq_len);
+  return LK_OK;
+}
+int rv_max_of(const lk_latent_cache* v) {
+  int m = 0;
+  for (int h = 0; h < v->n_heads; ++h) m = std::max(m, (int)v->ranks[h]);
+  return m;
+}
+}  // namespace
+
+size_t lk_latent_decode_rope_workspace_bytes(const lk_latent_cache* k, const lk_latent_cache* v, int32_t head_dim,
+                                             int32_t max_seq_len) {
+  if (rope_check(k, v, head_dim, max_seq_len) != LK_OK) return 0;
+  return lk::rope_workspace_bytes(k->batch * k->n_heads, rv_max_of(v), max_seq_len, num_sms());
+}
+
+lk_status lk_latent_decode_attn_rope(const lk_latent_cache* k, const lk_latent_cache* v, const void* q,
+                                     lk_dtype q_dtype, const void* B_K, const void* B_V, lk_dtype b_dtype,
+                                     int32_t head_dim, const int32_t* seq_len, int32_t max_seq_len,
+                                     const float* rope_table, float softmax_scale, void* out, lk_dtype out_dtype,
+                                     void* workspace, size_t workspace_bytes, lk_stream_t stream) {
+  lk_status s;
+  if ((s = rope_check(k, v, head_dim, max_seq_len)) != LK_OK) return s;
+  if (!q || !B_K || !B_V || !out || !seq_len || !rope_table)
+    return fail(LK_ERR_INVALID_ARG, "null q, B_K, B_V, out, seq_len or rope_table");
+  if (q_dtype != LK_F32 && q_dtype != LK_BF16) return fail(LK_ERR_DTYPE, "q dtype must be LK_F32 or LK_BF16");
+  if (b_dtype != LK_BF16) return fail(LK_ERR_DTYPE, "B dtype must be LK_BF16");
+  if (out_dtype != LK_F32 && out_dtype != LK_BF16) return fail(LK_ERR_DTYPE, "out dtype must be LK_F32 or LK_BF16");
+  if (!aligned(q, 16) || !aligned(B_K, 16) || !aligned(B_V, 16) || !aligned(rope_table, 16))
+    return fail(LK_ERR_ALIGN, "q, B_K, B_V and rope_table must be 16-byte aligned");
+  if (!(softmax_scale == softmax_scale)) return fail(LK_ERR_INVALID_ARG, "softmax_scale is NaN");
+  const size_t need = lk_latent_decode_rope_workspace_bytes(k, v, head_dim, max_seq_len);
+  if (!workspace || workspace_bytes < need)
+    return fail(LK_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
+  if (!aligned(workspace, 256)) return fail(LK_ERR_ALIGN, "workspace must be 256-byte aligned");
+  lk::RopeLaunch a{};
+  a.codes_k = k->codes;
+  a.codes_v = v->codes;
+  a.scales_k = k->scales;
+  a.scales_v = v->scales;
+  a.q = q;
+  a.BK = B_K;
+  a.BV = B_V;
+  a.table = rope_table;
+  a.seq_len = seq_len;
+  a.out = out;
+  a.workspace = workspace;
+  a.ranks_k = k->ranks;
+  a.ranks_v = v->ranks;
+  a.kind = k->code_dtype == LK_I8 ? 0 : 1;
+  a.batch = k->batch;
+  a.n_heads = k->n_heads;
+  a.head_dim = head_dim;
+  a.capacity = k->capacity;
+  a.group_k = k->group;
+  a.group_v = v->group;
+  a.q_bf16 = q_dtype == LK_BF16;
+  a.out_bf16 = out_dtype == LK_BF16;
+  a.max_len = max_seq_len;
+  a.num_sms = num_sms();
+  a.softmax_scale = softmax_scale;
+  if (max_seq_len == 0) {
+    // nothing to attend: every output is zero
+    const size_t ob = (size_t)k->batch * k->n_heads * head_dim * (out_dtype == LK_BF16 ? 2 : 4);
+    cudaError_t e = cudaMemsetAsync(out, 0, ob, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "lk_latent_decode_attn_rope");
+    return LK_OK;
+  }
+  cudaError_t e = lk::launch_rope_decode(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lk_latent_decode_attn_rope");
+  return LK_OK;
+}
+
 lk_status lk_latent_reconstruct_kv(const lk_latent_cache* k, const lk_latent_cache* v, const void* B_K,
                                    const void* B_V, lk_dtype b_dtype, int32_t head_dim, const int32_t* seq_len,
                                    int32_t max_seq_len, void* K_out, void* V_out, lk_stream_t stream) {
@@ -387,12 +485,13 @@ lk_status lk_latent_reconstruct_kv(const lk_latent_cache* k, const lk_latent_cac
     return fail(LK_ERR_SHAPE, "k and v caches differ in batch, heads or capacity");
   if (k->code_dtype != v->code_dtype) return fail(LK_ERR_UNSUPPORTED, "k and v caches differ in code dtype");
   if (!B_K || !B_V || !seq_len || !K_out || !V_out) return fail(LK_ERR_INVALID_ARG, "null B_K, B_V, seq_len or outputs");
-  if (b_dtype != LK_F32 && b_dtype != LK_BF16) return fail(LK_ERR_DTYPE, "B dtype must be LK_F32 or LK_BF16");
-  if (head_dim < 8 || head_dim > LK_MAX_HEAD_DIM || head_dim % 8 != 0)
-    return fail(LK_ERR_SHAPE, "head_dim %d must be a multiple of 8 in [8, %d]", head_dim, LK_MAX_HEAD_DIM);
+  if (b_dtype != LK_BF16) return fail(LK_ERR_DTYPE, "B dtype must be LK_BF16");
+  if (head_dim < 16 || head_dim > LK_MAX_HEAD_DIM || head_dim % 16 != 0)
+    return fail(LK_ERR_SHAPE, "head_dim %d must be a multiple of 16 in [16, %d]", head_dim, LK_MAX_HEAD_DIM);
   if (max_seq_len < 0 || max_seq_len > k->capacity)
     return fail(LK_ERR_SHAPE, "max_seq_len %d outside [0, capacity]", max_seq_len);
   if (!aligned(K_out, 16) || !aligned(V_out, 16)) return fail(LK_ERR_ALIGN, "K_out and V_out must be 16-byte aligned");
+  if (!aligned(B_K, 16) || !aligned(B_V, 16)) return fail(LK_ERR_ALIGN, "B_K and B_V must be 16-byte aligned");
   lk::ReconLaunch a{};
   a.codes[0] = k->codes;
   a.codes[1] = v->codes;
@@ -514,6 +613,13 @@ lk_status lk_rmsnorm_quant_i8(const void* x, lk_dtype x_dtype, int32_t m, int32_
                               float* x_scale, lk_stream_t stream) {
   if (!(eps >= 0.0f)) return fail(LK_ERR_INVALID_ARG, "eps must be >= 0");
   return rowquant(1, x, nullptr, x_dtype, m, k, eps, x_q, x_scale, stream, "lk_rmsnorm_quant_i8");
+}
+
+lk_status lk_rmsnorm_hadamard_quant_i8(const void* x, lk_dtype x_dtype, int32_t m, int32_t k, float eps,
+                                       int8_t* x_q, float* x_scale, lk_stream_t stream) {
+  if (!(eps >= 0.0f)) return fail(LK_ERR_INVALID_ARG, "eps must be >= 0");
+  if (k < 1 || (k & (k - 1)) != 0) return fail(LK_ERR_SHAPE, "lk_rmsnorm_hadamard_quant_i8: k %d not a power of two", k);
+  return rowquant(3, x, nullptr, x_dtype, m, k, eps, x_q, x_scale, stream, "lk_rmsnorm_hadamard_quant_i8");
 }
 
 lk_status lk_swiglu_quant_i8(const void* gate, const void* up, lk_dtype dtype, int32_t m, int32_t n, int8_t* h_q,

@@ -212,3 +212,44 @@ static constexpr uint64_t LK_WAIT_LIMIT_NS = 2000000000ull;  // 2 s
 // kernel be scheduled early.
 LK_DEVICE void lk_grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 LK_DEVICE void lk_grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+// ---------------------------------------------------------------- warp-level bf16 tensor-core products
+// D = A B + D for a 16 x 16 (m16n8k16) or 16 x 8 (m16n8k8) bf16 A and a
+// 16 x 8 / 8 x 8 bf16 B, fp32 accumulators.  Fragments (gid = lane / 4,
+// tig = lane % 4): a0 = (row gid, k 2 tig, 2 tig + 1), a1 = row gid + 8,
+// a2 / a3 = the same rows at k + 8; b0 = (k 2 tig, 2 tig + 1, column gid),
+// b1 = k + 8; c0, c1 = (row gid, columns 2 tig, 2 tig + 1), c2, c3 = row
+// gid + 8.  The k8 form takes a0, a1 and b0 only.
+LK_DEVICE void lk_mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                 uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+LK_DEVICE void lk_mma_bf16_1688(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+// Four 8 x 8 b16 matrices from shared memory: lanes 8 i .. 8 i + 7 give the
+// row addresses of matrix i (16 bytes each); lane l receives, of matrix i,
+// row l / 4, elements 2 (l % 4) and 2 (l % 4) + 1 (.trans: the transpose).
+LK_DEVICE void lk_ldmatrix_x4(uint32_t (&r)[4], const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(lk_smem_addr(row_addr)));
+}
+LK_DEVICE void lk_ldmatrix_x4_trans(uint32_t (&r)[4], const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(lk_smem_addr(row_addr)));
+}
+// Two values as packed bf16 (first in the low half), round to nearest even.
+LK_DEVICE uint32_t lk_pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}

@@ -263,25 +263,38 @@ __global__ void __launch_bounds__(kDThreads) dense_decode_kernel(const __grid_co
 
 // ---------------------------------------------------------------- naive reconstruction
 // K[b, h, t, :] = dequant(c_K[t]) B_K^h for t < seq_len[b] (and V likewise),
-// stored bf16 [B, n_heads, capacity, H].  A CTA takes 64 tokens of one
-// (b, h, K-or-V): B^h staged in shared memory as fp32, the 64 code rows and
-// scales read from the cache layout, each thread 8 outputs of a row.
+// stored bf16 [B, n_heads, capacity, H], on the tensor cores: a CTA takes
+// kRTok tokens of one (b, h, K-or-V).  The codes of those tokens (one
+// contiguous byte range of the cache plane in either layout) are expanded to
+// bf16 rows [token][dim] in shared memory (exact: |code| <= 127), B^h is
+// staged as bf16 [dim][H]; each warp takes 16-token tiles and, per pair of
+// 8-dim output columns, runs m16n8k16 products over the latent dims (int4
+// with several scale groups: m16n8k8 products, one accumulator per group,
+// each group's sum scaled by the token's group scale), then scales by the
+// token's scale, rounds to bf16 once and stores.  The code and factor
+// products are exact; the only rounding besides the fp32 sums is the final
+// one to bf16.
 struct ReconParams {
   const uint8_t* codes[2];
   const uint8_t* scales[2];
-  const void* Bf[2];
+  const uint16_t* Bf[2];
   uint16_t* dst[2];
   const int32_t* seq_len;
-  int kind, n_heads, H, capacity, b_bf16, max_len;
+  int kind, n_heads, H, capacity, max_len;
   int tot_rb[2], tot_ng[2];
   uint8_t rank[2][LK_MAX_HEADS], group[2][LK_MAX_HEADS];
   uint16_t pref_rb[2][LK_MAX_HEADS], pref_ng[2][LK_MAX_HEADS], pref_r[2][LK_MAX_HEADS];
 };
 
-constexpr int kRTok = 64;
+constexpr int kRTok = 256;      // tokens per CTA
+constexpr int kRWarps = 8;
 
-__global__ void __launch_bounds__(256) reconstruct_kernel(const __grid_constant__ ReconParams p) {
-  extern __shared__ __align__(16) float rsmem[];  // B^h [r][H] fp32, then codes [kRTok][r] fp32 (dequantised)
+// Shared-memory strides (bf16 elements): rows padded by 8 so that the eight
+// 16-byte rows an ldmatrix reads fall in distinct banks.
+LK_DEVICE int recon_cstride(int r16) { return r16 + 8; }
+
+__global__ void __launch_bounds__(kRWarps * 32) reconstruct_kernel(const __grid_constant__ ReconParams p) {
+  extern __shared__ __align__(16) uint8_t rsm[];
   const int which = blockIdx.z;  // 0: K, 1: V
   const int bh = blockIdx.y;
   const int b = bh / p.n_heads, h = bh - b * p.n_heads;
@@ -289,72 +302,173 @@ __global__ void __launch_bounds__(256) reconstruct_kernel(const __grid_constant_
   const int len = max(0, min(p.seq_len[b], p.max_len));
   if (t0 >= len) return;
   const int r = p.rank[which][h], H = p.H;
+  const int r16 = (r + 15) & ~15;
   const int rb = p.kind == 0 ? r : r / 2;
-  float* Bs = rsmem;
-  float* Cs = rsmem + r * H;
-  const int64_t boff = (int64_t)p.pref_r[which][h] * H;
-  for (int i = threadIdx.x; i < r * H; i += blockDim.x) {
-    Bs[i] = p.b_bf16 ? lk_bf16_to_f32(static_cast<const uint16_t*>(p.Bf[which])[boff + i])
-                     : static_cast<const float*>(p.Bf[which])[boff + i];
+  const int g = p.group[which][h], ng = (r + g - 1) / g;
+  const int cst = recon_cstride(r16), bst = H + 8;
+  uint16_t* Cs = reinterpret_cast<uint16_t*>(rsm);              // [kRTok][cst]
+  uint16_t* Bs = Cs + kRTok * cst;                              // [r16][bst]
+  float* Ss = reinterpret_cast<float*>(Bs + r16 * bst);         // [kRTok][ng]
+  const int ntok = min(kRTok, len - t0);
+  const int ntok16 = (ntok + 15) & ~15;                         // whole 16-token blocks (the cache holds them)
+  // B^h rows, zero rows up to r16
+  const uint16_t* Bg = p.Bf[which] + (int64_t)p.pref_r[which][h] * H;
+  for (int i = threadIdx.x; i < r16 * (H / 8); i += blockDim.x) {
+    const int d = i / (H / 8), c8 = i - d * (H / 8);
+    const uint4 v = d < r ? *reinterpret_cast<const uint4*>(Bg + (int64_t)d * H + 8 * c8) : make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(Bs + d * bst + 8 * c8) = v;
   }
+  // code dims r .. r16 - 1 are zero
+  for (int i = threadIdx.x; i < ntok16 * (r16 - r); i += blockDim.x) {
+    const int t = i / (r16 - r), d = r + i - t * (r16 - r);
+    Cs[t * cst + d] = 0;
+  }
+  // codes: the plane's bytes of tokens t0 .. t0 + ntok16, read as words
   const uint8_t* plane = p.codes[which] + ((int64_t)b * p.tot_rb[which] + p.pref_rb[which][h]) * p.capacity;
-  const int g = p.kind == 0 ? r : min((int)p.group[which][h], r), ng = (r + g - 1) / g;
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(plane + (int64_t)t0 * rb);
+  const int nwords = ntok16 * rb / 4;
   const int cs = lk_chunk_bytes(rb);
-  for (int i = threadIdx.x; i < kRTok * r; i += blockDim.x) {
-    const int tl = i / r, d = i - tl * r;
-    const int t = t0 + tl;
-    float val = 0.0f;
-    if (t < len) {
-      int code;
+  for (int i = threadIdx.x; i < nwords; i += blockDim.x) {
+    const uint32_t w = __ldg(src + i);
+    const int o = 4 * i;
+    const int blk = o / (16 * rb), rem = o - blk * 16 * rb;
+    if (which == 0) {  // token-major chunks: the word is consecutive bytes of one token
+      const int ch = rem / (16 * cs), rem2 = rem - ch * 16 * cs;
+      const int t = blk * 16 + rem2 / cs, byte0 = ch * cs + rem2 % cs;
+      uint16_t* row = Cs + t * cst;
       if (p.kind == 0) {
-        const int64_t off = which == 0 ? lk_code_offset(t, d, rb, cs) : (int64_t)(t >> 4) * 16 * rb + d * 16 + (t & 15);
-        code = (int)(int8_t)plane[off];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) row[byte0 + k] = __bfloat16_as_ushort(__int2bfloat16_rn((int)(int8_t)(w >> (8 * k))));
       } else {
-        int nib;
-        if (which == 0) {
-          const uint8_t byte = plane[lk_code_offset(t, d >> 1, rb, cs)];
-          nib = (d & 1) ? (byte >> 4) : (byte & 0xF);
-        } else {
-          const uint8_t byte = plane[(int64_t)(t >> 4) * 16 * rb + d * 8 + ((t & 15) >> 1)];
-          nib = (t & 1) ? (byte >> 4) : (byte & 0xF);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int nib = (int)((w >> (4 * k)) & 0xF);
+          row[2 * byte0 + k] = __bfloat16_as_ushort(__int2bfloat16_rn(nib >= 8 ? nib - 16 : nib));
         }
-        code = nib >= 8 ? nib - 16 : nib;
       }
-      float scale;
-      if (p.kind == 0) {
-        scale = reinterpret_cast<const float*>(p.scales[which])[((int64_t)b * p.n_heads + h) * p.capacity + t];
-      } else {
-        const uint16_t* sp = reinterpret_cast<const uint16_t*>(p.scales[which]) +
-                             ((int64_t)b * p.tot_ng[which] + p.pref_ng[which][h]) * p.capacity;
-        scale = lk_f16_to_f32(sp[(int64_t)t * ng + d / g]);
+    } else if (p.kind == 0) {  // dimension-major: the word is 4 consecutive tokens of one dim
+      const int d = rem / 16, tt = rem % 16;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        Cs[(blk * 16 + tt + k) * cst + d] = __bfloat16_as_ushort(__int2bfloat16_rn((int)(int8_t)(w >> (8 * k))));
+    } else {                   // int4 dimension-major: 8 consecutive tokens of one dim
+      const int d = rem / 8, tt = 2 * (rem % 8);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int nib = (int)((w >> (4 * k)) & 0xF);
+        Cs[(blk * 16 + tt + k) * cst + d] = __bfloat16_as_ushort(__int2bfloat16_rn(nib >= 8 ? nib - 16 : nib));
       }
-      val = (float)code * scale;
     }
-    Cs[tl * r + d] = val;
+  }
+  // scales as fp32 [token][group]
+  if (p.kind == 0) {
+    const float* sp = reinterpret_cast<const float*>(p.scales[which]) + ((int64_t)b * p.n_heads + h) * p.capacity + t0;
+    for (int i = threadIdx.x; i < ntok16; i += blockDim.x) Ss[i] = sp[i];
+  } else {
+    const uint16_t* sp = reinterpret_cast<const uint16_t*>(p.scales[which]) +
+                         ((int64_t)b * p.tot_ng[which] + p.pref_ng[which][h]) * p.capacity + (int64_t)t0 * ng;
+    for (int i = threadIdx.x; i < ntok16 * ng; i += blockDim.x) Ss[i] = lk_f16_to_f32(sp[i]);
   }
   __syncthreads();
-  uint16_t* out = p.dst[which] + ((int64_t)bh * p.capacity) * H;
-  const int chunks = H / 8;
-  for (int i = threadIdx.x; i < kRTok * chunks; i += blockDim.x) {
-    const int tl = i / chunks, c8 = i - tl * chunks;
-    const int t = t0 + tl;
-    if (t >= len) continue;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int d = 0; d < r; ++d) {
-      const float cv = Cs[tl * r + d];
-      const float4 b0 = *reinterpret_cast<const float4*>(Bs + d * H + 8 * c8);
-      const float4 b1 = *reinterpret_cast<const float4*>(Bs + d * H + 8 * c8 + 4);
-      acc[0] = fmaf(cv, b0.x, acc[0]); acc[1] = fmaf(cv, b0.y, acc[1]);
-      acc[2] = fmaf(cv, b0.z, acc[2]); acc[3] = fmaf(cv, b0.w, acc[3]);
-      acc[4] = fmaf(cv, b1.x, acc[4]); acc[5] = fmaf(cv, b1.y, acc[5]);
-      acc[6] = fmaf(cv, b1.z, acc[6]); acc[7] = fmaf(cv, b1.w, acc[7]);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int nks = r16 / 16;
+  const bool grouped = ng > 1;  // int4 with several groups (groups are multiples of 8 dims)
+  uint16_t* out = p.dst[which] + (int64_t)bh * p.capacity * H;
+  // a warp takes two 16-token tiles at a time, so that each B fragment read
+  // from shared memory feeds both
+  for (int tb0 = 32 * warp; tb0 < ntok16; tb0 += 32 * kRWarps) {
+    const int nmt = tb0 + 16 < ntok16 ? 2 : 1;
+    // A fragments of each tile and k step: matrices (rows 0-7, k 0-7),
+    // (rows 8-15, k 0-7), (rows 0-7, k 8-15), (rows 8-15, k 8-15)
+    uint32_t af[2][4][4];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        if (m < nmt && ks < nks) {
+          const int row = tb0 + 16 * m + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int col = 16 * ks + (lane >> 4) * 8;
+          lk_ldmatrix_x4(af[m][ks], Cs + row * cst + col);
+        } else {
+          af[m][ks][0] = af[m][ks][1] = af[m][ks][2] = af[m][ks][3] = 0u;
+        }
+      }
     }
-    uint4 o;
-    o.x = (uint32_t)lk_f32_to_bf16(acc[0]) | ((uint32_t)lk_f32_to_bf16(acc[1]) << 16);
-    o.y = (uint32_t)lk_f32_to_bf16(acc[2]) | ((uint32_t)lk_f32_to_bf16(acc[3]) << 16);
-    o.z = (uint32_t)lk_f32_to_bf16(acc[4]) | ((uint32_t)lk_f32_to_bf16(acc[5]) << 16);
-    o.w = (uint32_t)lk_f32_to_bf16(acc[6]) | ((uint32_t)lk_f32_to_bf16(acc[7]) << 16);
-    *reinterpret_cast<uint4*>(out + (int64_t)t * H + 8 * c8) = o;
+    for (int n0 = 0; n0 < H; n0 += 16) {
+      // [tile][column octet][fragment]
+      float acc[2][2][4], o[2][2][4];
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[m][n][e] = o[m][n][e] = 0.0f;
+      int cur = 0;  // scale group of the open accumulators
+      auto fold = [&](int gi) {
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          const int tl = tb0 + 16 * m + gid;
+          const float sl = Ss[tl * ng + gi], sh = Ss[(tl + 8) * ng + gi];
+#pragma unroll
+          for (int n = 0; n < 2; ++n) {
+            o[m][n][0] = fmaf(sl, acc[m][n][0], o[m][n][0]);
+            o[m][n][1] = fmaf(sl, acc[m][n][1], o[m][n][1]);
+            o[m][n][2] = fmaf(sh, acc[m][n][2], o[m][n][2]);
+            o[m][n][3] = fmaf(sh, acc[m][n][3], o[m][n][3]);
+            acc[m][n][0] = acc[m][n][1] = acc[m][n][2] = acc[m][n][3] = 0.0f;
+          }
+        }
+      };
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        if (ks < nks) {
+          // B fragments for columns n0 .. n0 + 15: matrices (k 0-7, n 0-7),
+          // (k 8-15, n 0-7), (k 0-7, n 8-15), (k 8-15, n 8-15), transposed
+          uint32_t bfr[4];
+          const int krow = 16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int ncol = n0 + (lane >> 4) * 8;
+          lk_ldmatrix_x4_trans(bfr, Bs + krow * bst + ncol);
+          if (!grouped) {
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+              lk_mma_bf16_16816(acc[m][0], af[m][ks][0], af[m][ks][1], af[m][ks][2], af[m][ks][3], bfr[0], bfr[1]);
+              lk_mma_bf16_16816(acc[m][1], af[m][ks][0], af[m][ks][1], af[m][ks][2], af[m][ks][3], bfr[2], bfr[3]);
+            }
+          } else {
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              const int d0 = 16 * ks + 8 * hf;
+              if (d0 < r) {
+                const int gi = d0 / g;
+                if (gi != cur) {  // the previous group is complete
+                  fold(cur);
+                  cur = gi;
+                }
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                  lk_mma_bf16_1688(acc[m][0], af[m][ks][2 * hf], af[m][ks][2 * hf + 1], bfr[hf]);
+                  lk_mma_bf16_1688(acc[m][1], af[m][ks][2 * hf], af[m][ks][2 * hf + 1], bfr[2 + hf]);
+                }
+              }
+            }
+          }
+        }
+      }
+      fold(cur);  // (one group: o = sigma * acc)
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int t_lo = t0 + tb0 + 16 * m + gid, t_hi = t_lo + 8;
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+          const int col = n0 + 8 * n + 2 * tig;
+          if (m < nmt && t_lo < len)
+            *reinterpret_cast<uint32_t*>(out + (int64_t)t_lo * H + col) = lk_pack_bf16x2(o[m][n][0], o[m][n][1]);
+          if (m < nmt && t_hi < len)
+            *reinterpret_cast<uint32_t*>(out + (int64_t)t_hi * H + col) = lk_pack_bf16x2(o[m][n][2], o[m][n][3]);
+        }
+      }
+    }
   }
 }
 
@@ -414,14 +528,14 @@ cudaError_t launch_reconstruct_kv(const ReconLaunch& a, cudaStream_t stream) {
   p.n_heads = a.n_heads;
   p.H = a.head_dim;
   p.capacity = a.capacity;
-  p.b_bf16 = a.b_bf16;
+  if (!a.b_bf16) return cudaErrorInvalidValue;  // the factors are bf16 tensor-core operands
   p.max_len = a.max_len;
   p.seq_len = a.seq_len;
   int r_max = 0;
   for (int c = 0; c < 2; ++c) {
     p.codes[c] = static_cast<const uint8_t*>(a.codes[c]);
     p.scales[c] = static_cast<const uint8_t*>(a.scales[c]);
-    p.Bf[c] = a.B[c];
+    p.Bf[c] = static_cast<const uint16_t*>(a.B[c]);
     p.dst[c] = static_cast<uint16_t*>(a.out[c]);
     int prb = 0, png = 0, pr = 0;
     for (int h = 0; h < a.n_heads; ++h) {
@@ -440,12 +554,16 @@ cudaError_t launch_reconstruct_kv(const ReconLaunch& a, cudaStream_t stream) {
     p.tot_rb[c] = prb;
     p.tot_ng[c] = png;
   }
-  const int smem = (r_max * a.head_dim + kRTok * r_max) * 4;
+  int ng_max = 1;
+  for (int c = 0; c < 2; ++c)
+    for (int h = 0; h < a.n_heads; ++h) ng_max = std::max(ng_max, (a.ranks[c][h] + p.group[c][h] - 1) / p.group[c][h]);
+  const int r16 = (r_max + 15) & ~15;
+  const int smem = (kRTok * (r16 + 8) + r16 * (a.head_dim + 8)) * 2 + kRTok * ng_max * 4;
   cudaError_t e = cudaFuncSetAttribute(reconstruct_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)((a.max_len + kRTok - 1) / kRTok), (unsigned)(a.batch * a.n_heads), 2);
   if (grid.x == 0) return cudaSuccess;
-  reconstruct_kernel<<<grid, 256, smem, stream>>>(p);
+  reconstruct_kernel<<<grid, kRWarps * 32, smem, stream>>>(p);
   count_launch();
   return cudaGetLastError();
 }

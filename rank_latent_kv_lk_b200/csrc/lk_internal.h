@@ -48,6 +48,29 @@ size_t decode_workspace_bytes(int units, int rv_max, int max_len, int n_split);
 cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream);
 
 
+// ---------------------------------------------------------------- rotary-position decode
+struct RopeLaunch {
+  const void* codes_k;
+  const void* codes_v;
+  const void* scales_k;
+  const void* scales_v;
+  const void* q;
+  const void* BK;  // bf16
+  const void* BV;  // bf16
+  const float* table;
+  const int32_t* seq_len;
+  void* out;
+  void* workspace;
+  const int32_t* ranks_k;  // host
+  const int32_t* ranks_v;  // host
+  int kind, batch, n_heads, head_dim, capacity, group_k, group_v;
+  int q_bf16, out_bf16, max_len, num_sms;
+  float softmax_scale;
+};
+size_t rope_workspace_bytes(int units, int rv_max, int max_len, int num_sms);
+cudaError_t launch_rope_decode(const RopeLaunch& a, cudaStream_t stream);
+cudaError_t launch_rope_table(float* table, int head_dim, int max_pos, double base, cudaStream_t stream);
+
 // ---------------------------------------------------------------- dense comparison points
 struct DenseLaunch {
   const void* q;  // bf16 [B, n_heads, H]
@@ -85,6 +108,7 @@ struct CacheView {
   int group;
   int n_heads;
   int capacity;
+  int rotation;  // 1: each head's latent is rotated by its S2 before quantisation
 };
 
 struct ProjectLaunch {
@@ -132,7 +156,8 @@ cudaError_t launch_lowrank_linear(const LowrankLaunch& a, cudaStream_t stream);
 // ---------------------------------------------------------------- quantisers / elementwise
 cudaError_t launch_quantize_latent(const float* v, int m, int r, int kind, int group, void* codes,
                                    void* scales, cudaStream_t stream);
-// mode 0: quantise x; 1: RMSNorm then quantise; 2: SwiGLU(x, x2) then quantise
+// mode 0: quantise x; 1: RMSNorm then quantise; 2: SwiGLU(x, x2) then quantise;
+// 3: RMSNorm, then the normalised Walsh-Hadamard transform (k a power of two), then quantise
 cudaError_t launch_rowquant(int mode, const void* x, const void* x2, int x_bf16, int m, int k,
                             float eps, int8_t* x_q, float* x_scale, cudaStream_t stream);
 

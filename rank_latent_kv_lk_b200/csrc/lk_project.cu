@@ -128,6 +128,7 @@ LK_DEVICE void append_values(const FinalizeParams& p, int grow, int j, float v0,
   const lk::CacheView& cv = is_k ? p.k : p.v;
   const int hh = is_k ? j : j - p.k.n_heads;
   const int r = p.rank[j];
+  if (cv.rotation) lk_rotate_latent_warp(v0, v1, r);
   const LkQRow qr = lk_quantize_row_warp(v0, v1, r, cv.kind, cv.group);
   const int64_t pos = (int64_t)p.seq_len[b] + t;
   const int cap = cv.capacity;
@@ -207,9 +208,9 @@ __global__ void __launch_bounds__(128) proj_finalize_kernel(const __grid_constan
 }
 
 // ---------------------------------------------------------------- decode: one cluster per head
-// A thread-block cluster of kClusterE CTAs owns one head: CTA q reduces the
-// q-th slice of E for every latent column of the head and every row; the
-// cluster's rank 0 sums the kClusterE partials over distributed shared memory,
+// A thread-block cluster of CE CTAs owns one head: CTA q reduces the q-th
+// slice of E for every latent column of the head and every row; the
+// cluster's rank 0 sums the CE partials over distributed shared memory,
 // quantises and appends.  No partials leave the SMs and nobody waits on a
 // global counter; the last head to finish advances seq_len (atomic ticket).
 //
@@ -222,7 +223,11 @@ __global__ void __launch_bounds__(128) proj_finalize_kernel(const __grid_constan
 // and the rows of x (converted once to fp32 in shared memory) are broadcast
 // loads.  The four lanes' sums meet by two shuffles, the warps of a tile in
 // shared memory in a fixed order (the result does not depend on timing).
-constexpr int kClusterE = 8;  // CTAs per head (portable cluster size): each reduces 1/8 of E
+// CTAs per head: 8 (the portable cluster size) for 3..8 token rows; 4 for one
+// or two rows, whose CTAs finish sooner and leave more of the GPU to an
+// attention launch that overlaps them (decode step)
+constexpr int kClusterMax = 8;
+int cluster_for_rows(int rows) { return rows <= 2 ? 4 : 8; }
 constexpr int kProjWarps = kGemvThreads / 32;
 
 struct ClusterProjParams {
@@ -234,7 +239,7 @@ struct ClusterProjParams {
   int off_x, off_red;  // shared-memory offsets: x slice (fp32, or int8 for int8 inputs), warp partials
 };
 
-template <int XT, int MT>
+template <int XT, int MT, int CE>
 __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid_constant__ ClusterProjParams p) {
   lk_grid_dep_launch();  // a decode launched next may start its set-up now
   using T = typename XTraits<XT>::T;
@@ -390,11 +395,11 @@ __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid
           if (INT) {
             int acc = 0;
 #pragma unroll
-            for (int q = 0; q < kClusterE; ++q) acc += (int)part[((size_t)q * LK_MAX_RANK + d) * M + m];
+            for (int q = 0; q < CE; ++q) acc += (int)part[((size_t)q * LK_MAX_RANK + d) * M + m];
             val = __fmul_rn(__fmul_rn((float)acc, f.x_scale[m]), lk_f16_to_f32(f.a_scale[nn]));
           } else {
 #pragma unroll
-            for (int q = 0; q < kClusterE; ++q) val += __uint_as_float(part[((size_t)q * LK_MAX_RANK + d) * M + m]);
+            for (int q = 0; q < CE; ++q) val += __uint_as_float(part[((size_t)q * LK_MAX_RANK + d) * M + m]);
           }
         }
         vals[q2] = val;
@@ -414,18 +419,173 @@ __global__ void __launch_bounds__(kGemvThreads) proj_cluster_kernel(const __grid
   }
 }
 
+// ---------------------------------------------------------------- decode, bf16: tensor-core GEMV
+// v^T = A x^T for up to 32 token rows of bf16 inputs, one launch.  A CTA owns
+// 16 latent columns (one m16 tile) over all of E; its 8 warps split E.  Per
+// 64-element k block a lane loads 16 consecutive k of two weight rows (gid,
+// gid + 8) and of its token rows (gid, gid + 8, ...), and the block's four
+// m16n8k16 products take their k slots from those registers: product s uses
+// k = 16 tig + 4 s + {0, 1} for the slots 2 tig, 2 tig + 1 and 16 tig + 4 s +
+// {2, 3} for 2 tig + 8, 2 tig + 9, for A and x alike, so every k of the block
+// meets its own x once and the sum is the plain dot product.  Each weight is
+// read once (16-byte loads, L1 bypassed); the tensor cores only keep the
+// instruction count per byte low, the launch is bound by HBM.  The warps'
+// sums meet in shared memory in a fixed order, go to the workspace, and the
+// CTA that completes a head's last column block (ticket per head) quantises
+// and appends that head for every row; the last head advances seq_len.
+constexpr int kMmaWarps = 8;
+constexpr int kMmaMaxRows = 32;
+
+struct MmaProjParams {
+  FinalizeParams f;
+  const uint16_t* x;
+  const uint16_t* A;
+  int M, E;
+  int32_t* done_cnt;
+  int32_t* head_cnt;  // [heads] column blocks of the head done in this launch
+};
+
+LK_DEVICE uint4 ldg_stream16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+LK_DEVICE uint32_t word_of(const uint4 (&v)[2], int w) {
+  const uint4& q = v[w >> 2];
+  return (w & 3) == 0 ? q.x : (w & 3) == 1 ? q.y : (w & 3) == 2 ? q.z : q.w;
+}
+
+template <int NT>  // n8 tiles of token rows: M <= 8 NT
+__global__ void __launch_bounds__(kMmaWarps * 32) proj_mma_kernel(const __grid_constant__ MmaProjParams p) {
+  lk_grid_dep_launch();  // a decode launched next may start its set-up now
+  constexpr int BR = NT == 1 ? 4 : (NT == 2 ? 2 : 1);  // k blocks whose loads are in flight together
+  __shared__ float red[kMmaWarps][16][8 * NT + 1];
+  __shared__ int fin[16];  // heads whose last column block this CTA completed
+  __shared__ int nfin;
+  const FinalizeParams& f = p.f;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int col0 = blockIdx.x * 16;
+  const int M = p.M, E = p.E;
+  const int nb = (E + 63) / 64;
+  const int kb0 = warp * nb / kMmaWarps, kb1 = (warp + 1) * nb / kMmaWarps;
+  // columns past n_tot (last tile) repeat the last row: computed, never stored
+  const uint16_t* A0 = p.A + (int64_t)min(col0 + gid, f.n_tot - 1) * E;
+  const uint16_t* A1 = p.A + (int64_t)min(col0 + gid + 8, f.n_tot - 1) * E;
+  if (threadIdx.x == 0) nfin = 0;
+  // The CTA's weight rows are one contiguous range: ask for all of it in L2
+  // at once (bulk prefetches, 16 KB each), so HBM streams at full rate while
+  // the warps' own loads, whose number in flight the register budget caps,
+  // find their lines in L2.
+  if (threadIdx.x < 32) {
+    const int nrows = min(16, f.n_tot - col0);
+    const char* base = reinterpret_cast<const char*>(p.A + (int64_t)col0 * E);
+    const int64_t bytes = (int64_t)nrows * E * 2;
+    for (int64_t off = (int64_t)threadIdx.x * 16384; off < bytes; off += 32 * 16384) {
+      const uint32_t n = (uint32_t)min((int64_t)16384, bytes - off);
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + off), "r"(n) : "memory");
+    }
+  }
+  float c[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) c[t][0] = c[t][1] = c[t][2] = c[t][3] = 0.0f;
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  for (int kb = kb0; kb < kb1; kb += BR) {
+    uint4 wa[BR][2], wb[BR][2], xv[BR][NT][2];
+#pragma unroll
+    for (int u = 0; u < BR; ++u) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int k = (kb + u) * 64 + 16 * tig + 8 * h;
+        const bool ok = kb + u < kb1 && k < E;  // E is a multiple of 8
+        wa[u][h] = ok ? ldg_stream16(A0 + k) : z;
+        wb[u][h] = ok ? ldg_stream16(A1 + k) : z;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const int m = 8 * t + gid;
+          // (volatile like the weight loads, so that all of a round's loads are
+          // issued before the first product waits on one)
+          xv[u][t][h] = ok && m < M ? ldg_stream16(p.x + (int64_t)m * E + k) : z;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < BR; ++u) {
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const uint32_t a0 = word_of(wa[u], 2 * s), a2 = word_of(wa[u], 2 * s + 1);
+        const uint32_t a1 = word_of(wb[u], 2 * s), a3 = word_of(wb[u], 2 * s + 1);
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+          lk_mma_bf16_16816(c[t], a0, a1, a2, a3, word_of(xv[u][t], 2 * s), word_of(xv[u][t], 2 * s + 1));
+      }
+    }
+  }
+  // D fragment: c0, c1 = (column gid, rows 2 tig, 2 tig + 1), c2, c3 = column gid + 8
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    red[warp][gid][8 * t + 2 * tig] = c[t][0];
+    red[warp][gid][8 * t + 2 * tig + 1] = c[t][1];
+    red[warp][gid + 8][8 * t + 2 * tig] = c[t][2];
+    red[warp][gid + 8][8 * t + 2 * tig + 1] = c[t][3];
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < 16 * M; idx += kMmaWarps * 32) {
+    const int cc = idx / M, m = idx - cc * M;
+    const int n = col0 + cc;
+    if (n < f.n_tot) {
+      float s = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kMmaWarps; ++w) s += red[w][cc][m];
+      f.ws[(int64_t)m * f.n_tot + n] = __float_as_uint(s);
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  const int nh = f.k.n_heads + f.v.n_heads;
+  for (int j = threadIdx.x; j < nh; j += kMmaWarps * 32) {
+    const int h0 = f.col[j], h1 = h0 + f.rank[j];
+    if (h0 < col0 + 16 && h1 > col0) {
+      const int nblk = (h1 - 1) / 16 - h0 / 16 + 1;
+      if (atomicAdd(&p.head_cnt[j], 1) == nblk - 1) fin[atomicAdd(&nfin, 1)] = j;
+    }
+  }
+  __syncthreads();
+  const int nf = nfin;
+  if (nf == 0) return;
+  __threadfence();  // the other blocks' columns of these heads are visible
+  for (int it = warp; it < nf * M; it += kMmaWarps) {
+    const int j = fin[it / M], m = it - (it / M) * M;
+    append_head(f, m, m, j);
+  }
+  __syncthreads();  // every append of these heads is written
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nf; ++i) p.head_cnt[fin[i]] = 0;  // ready for the next call
+    __threadfence();
+    if (atomicAdd(p.done_cnt, nf) == nh - nf) {  // every head appended: advance the rows
+      __threadfence();
+      for (int b = 0; b < f.batch; ++b) f.seq_len[b] += f.n_new;
+      *p.done_cnt = 0;
+    }
+  }
+}
+
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 // E-slice of each cluster CTA for the decode kernel (16-byte multiple).
-int cluster_slice(int E, int xtype) {
+int cluster_slice(int E, int xtype, int ce) {
   const int ve = xtype == lk::X_F32 ? 4 : (xtype == lk::X_BF16 ? 8 : 16);
-  return round_up((E + kClusterE - 1) / kClusterE, ve);
+  return round_up((E + ce - 1) / ce, ve);
 }
 
 int x_size(int xtype) { return xtype == lk::X_F32 ? 4 : (xtype == lk::X_BF16 ? 2 : 1); }
 
 constexpr int kPrefillRowChunk = 8192;
-constexpr size_t kWsHeader = 2048;  // done counter at 0, head counters at 256
+constexpr size_t kWsHeader = 2048;  // done counter at 0, per-head counters from byte 256 on
+constexpr int kHeadCntOffset = 256;
 
 }  // namespace
 
@@ -436,7 +596,9 @@ namespace lk {
 size_t project_workspace_bytes(int rows, int n_tot, int embed_dim, int xtype, int num_sms) {
   (void)num_sms;
   size_t body;
-  if (rows <= kGemvMaxRows) {
+  if (xtype == X_BF16 && rows <= kMmaMaxRows) {
+    body = (size_t)rows * n_tot * 4;  // the column sums, read back by each head's finishing CTA
+  } else if (rows <= kGemvMaxRows) {
     body = 0;  // partials stay in the cluster's shared memory
   } else {
     body = (size_t)std::min(rows, kPrefillRowChunk) * n_tot * 4;
@@ -482,6 +644,28 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
   const int heads_tot = a.k.n_heads + a.v.n_heads;
   cudaError_t e;
 
+  if (a.xtype == X_BF16 && rows <= kMmaMaxRows) {
+    MmaProjParams d{};
+    f.n_ksplit = 1;
+    f.ws_rows = rows;
+    f.row0 = 0;
+    f.rows = rows;
+    f.do_update = 1;
+    d.f = f;
+    d.x = static_cast<const uint16_t*>(a.x);
+    d.A = static_cast<const uint16_t*>(a.A);
+    d.M = rows;
+    d.E = a.embed_dim;
+    d.done_cnt = static_cast<int32_t*>(a.workspace);
+    d.head_cnt = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(a.workspace) + kHeadCntOffset);
+    const unsigned grid = (unsigned)((a.n_tot + 15) / 16);
+    if (rows <= 8) proj_mma_kernel<1><<<grid, kMmaWarps * 32, 0, stream>>>(d);
+    else if (rows <= 16) proj_mma_kernel<2><<<grid, kMmaWarps * 32, 0, stream>>>(d);
+    else proj_mma_kernel<4><<<grid, kMmaWarps * 32, 0, stream>>>(d);
+    count_launch();
+    return cudaGetLastError();
+  }
+
   if (rows <= kGemvMaxRows) {
     ClusterProjParams d{};
     f.n_ksplit = 1;
@@ -494,32 +678,38 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
     d.A = a.A;
     d.M = rows;
     d.E = a.embed_dim;
-    d.slice = cluster_slice(a.embed_dim, a.xtype);
     d.done_cnt = static_cast<int32_t*>(a.workspace);
     const size_t xelem = a.xtype == X_I8 ? 1 : 4;  // x slice in shared memory: int8 or fp32
-    d.off_x = round_up(kClusterE * LK_MAX_RANK * rows * 4, 128);
+    const int ce = cluster_for_rows(rows);
+    d.slice = cluster_slice(a.embed_dim, a.xtype, ce);
+    d.off_x = round_up(kClusterMax * LK_MAX_RANK * rows * 4, 128);
     d.off_red = d.off_x + round_up((int)(rows * d.slice * xelem), 128);
     const int mt = rows <= 1 ? 1 : (rows <= 2 ? 2 : (rows <= 4 ? 4 : 8));
     const size_t smem = (size_t)d.off_red + (size_t)kProjWarps * 8 * mt * 4;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kClusterE, heads_tot, 1);
+    cfg.gridDim = dim3(ce, heads_tot, 1);
     cfg.blockDim = dim3(kGemvThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kClusterE;
+    attr[0].val.clusterDim.x = ce;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-#define LK_PROJ_LAUNCH(XTV, MTV)                                                                        \
-  do {                                                                                                \
-    e = cudaFuncSetAttribute(proj_cluster_kernel<XTV, MTV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             (int)smem);                                                             \
-    if (e != cudaSuccess) return e;                                                                   \
-    e = cudaLaunchKernelEx(&cfg, proj_cluster_kernel<XTV, MTV>, d);                                  \
-    if (e == cudaSuccess) count_launch();                                                             \
+#define LK_PROJ_LAUNCH3(XTV, MTV, CEV)                                                                      \
+  do {                                                                                                     \
+    e = cudaFuncSetAttribute(proj_cluster_kernel<XTV, MTV, CEV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             (int)smem);                                                                  \
+    if (e != cudaSuccess) return e;                                                                        \
+    e = cudaLaunchKernelEx(&cfg, proj_cluster_kernel<XTV, MTV, CEV>, d);                                  \
+    if (e == cudaSuccess) count_launch();                                                                  \
+  } while (0)
+#define LK_PROJ_LAUNCH(XTV, MTV)                 \
+  do {                                           \
+    if (ce == 4) LK_PROJ_LAUNCH3(XTV, MTV, 4);   \
+    else LK_PROJ_LAUNCH3(XTV, MTV, 8);           \
   } while (0)
 #define LK_PROJ_MT(XTV)                          \
   do {                                           \
@@ -533,6 +723,7 @@ cudaError_t launch_project_append(const ProjectLaunch& a, cudaStream_t stream) {
     else LK_PROJ_MT(X_I8);
 #undef LK_PROJ_MT
 #undef LK_PROJ_LAUNCH
+#undef LK_PROJ_LAUNCH3
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }

@@ -59,7 +59,8 @@ LK_DEVICE float block_reduce(float v, float* scratch, bool is_max) {
 }
 
 // One CTA per row: y = f(x) kept in shared memory, then int8 absmax codes.
-// mode 0: y = x; 1: y = x / sqrt(mean(x^2) + eps); 2: y = silu(x) * x2.
+// mode 0: y = x; 1: y = x / sqrt(mean(x^2) + eps); 2: y = silu(x) * x2;
+// 3: mode 1, then the normalised Walsh-Hadamard transform of the row.
 template <bool BF16>
 __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(int mode, const void* __restrict__ x,
                                                               const void* __restrict__ x2, int k, float eps,
@@ -111,10 +112,26 @@ __global__ void __launch_bounds__(kRowThreads) rowquant_kernel(int mode, const v
       ss = fmaf(a, a, ss);
     }
   }
-  if (mode == 1) {
+  if (mode == 1 || mode == 3) {
     const float tot = block_reduce(ss, scratch, false);
     const float denom = sqrtf(__fdiv_rn(tot, (float)k) + eps);
     for (int i = threadIdx.x; i < k; i += kRowThreads) ys[i] = __fdiv_rn(ys[i], denom);
+  }
+  if (mode == 3) {
+    // S1 (WSVD page §2C): the normalised Walsh-Hadamard transform of the
+    // row (k a power of two), butterflies in shared memory
+    for (int h = 1; h < k; h <<= 1) {
+      __syncthreads();
+      for (int i = threadIdx.x; i < k / 2; i += kRowThreads) {
+        const int i0 = (i / h) * 2 * h + (i % h), i1 = i0 + h;
+        const float a = ys[i0], b = ys[i1];
+        ys[i0] = __fadd_rn(a, b);
+        ys[i1] = __fsub_rn(a, b);
+      }
+    }
+    __syncthreads();
+    const float c = __double2float_rn(1.0 / sqrt((double)k));  // fl32(1 / sqrt(k))
+    for (int i = threadIdx.x; i < k; i += kRowThreads) ys[i] = __fmul_rn(ys[i], c);
   }
   __syncthreads();
   float a = 0.0f;

@@ -4,6 +4,36 @@
 
 #include "lk_common.cuh"
 
+// S2 of one head's latent (WSVD page §2C: an orthogonal rotation of the
+// latent before RTN smooths outlier dims): block diagonal, each block the
+// normalised Walsh-Hadamard matrix of order n = the largest power of two
+// dividing r (at most 64).  Lane l holds v0 = dim l and v1 = dim l + 32;
+// in place, y_j = sum_i v_i (-1)^popcount(i & j) / sqrt(n) over each block
+// (butterflies across lanes by shuffles; the order-64 stage combines v0 and
+// v1 of the same lane).
+LK_DEVICE void lk_rotate_latent_warp(float& v0, float& v1, int r) {
+  const int lane = threadIdx.x & 31;
+  int n = 1;
+  while (r % (2 * n) == 0 && 2 * n <= 64) n *= 2;
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+    if (h < n) {
+      const float p0 = __shfl_xor_sync(0xffffffffu, v0, h);
+      const float p1 = __shfl_xor_sync(0xffffffffu, v1, h);
+      v0 = (lane & h) ? __fsub_rn(p0, v0) : __fadd_rn(v0, p0);
+      v1 = (lane & h) ? __fsub_rn(p1, v1) : __fadd_rn(v1, p1);
+    }
+  }
+  if (n == 64) {
+    const float a = v0, b = v1;
+    v0 = __fadd_rn(a, b);
+    v1 = __fsub_rn(a, b);
+  }
+  const float c = __double2float_rn(1.0 / sqrt((double)n));  // fl32(1 / sqrt(n))
+  v0 = __fmul_rn(v0, c);
+  v1 = __fmul_rn(v1, c);
+}
+
 // One row of r <= 64 latent values; lane l holds v0 = row[l] and
 // v1 = row[l + 32] (ignored past r).  Returns each element's code and the
 // scale of the group it belongs to.

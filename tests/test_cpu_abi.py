@@ -158,6 +158,9 @@ def test_quantizer_validation(L):
     assert L.lib.lk_quantize_rows_i8(None, L.LK_F32, 1, 40000, None, None, None) == L.LK_ERR_SHAPE
     assert L.lib.lk_quantize_rows_i8(None, L.LK_I8, 1, 4, None, None, None) == L.LK_ERR_DTYPE
     assert L.lib.lk_rmsnorm_quant_i8(None, L.LK_F32, 1, 4, -1.0, None, None, None) == L.LK_ERR_INVALID_ARG
+    assert L.lib.lk_rmsnorm_hadamard_quant_i8(None, L.LK_F32, 1, 48, 1e-5, None, None, None) == L.LK_ERR_SHAPE
+    assert L.lib.lk_rmsnorm_hadamard_quant_i8(None, L.LK_F32, 1, 65536, 1e-5, None, None, None) == L.LK_ERR_SHAPE
+    assert L.lib.lk_rmsnorm_hadamard_quant_i8(None, L.LK_F32, 1, 64, 1e-5, None, None, None) == L.LK_ERR_INVALID_ARG
     assert L.lib.lk_swiglu_quant_i8(C.c_void_p(FAKE), None, L.LK_F32, 1, 4, C.c_void_p(FAKE),
                                     C.c_void_p(FAKE), None) == L.LK_ERR_INVALID_ARG
 
@@ -170,3 +173,45 @@ def test_cache_bytes(L):
     k4 = cache(L, batch=2, heads=2, cap=32, kind=L.LK_I4, group=16, ranks=(24, 64))
     assert L.lib.lk_latent_cache_bytes(C.byref(k4), C.byref(cb), C.byref(sb)) == L.LK_OK
     assert cb.value == 2 * (12 + 32) * 32 and sb.value == 2 * (2 + 4) * 32 * 2
+    k.rotation = 1
+    assert L.lib.lk_latent_cache_bytes(C.byref(k), C.byref(cb), C.byref(sb)) == L.LK_OK
+    k.rotation = 2
+    assert L.lib.lk_latent_cache_bytes(C.byref(k), C.byref(cb), C.byref(sb)) == L.LK_ERR_INVALID_ARG
+
+
+def rope(L, k, v, max_len=32, ws_bytes=1 << 20, ws=FAKE + 0x200000, H=64, table=FAKE + 0xC00000, bdt=None):
+    return L.lib.lk_latent_decode_attn_rope(C.byref(k), C.byref(v), C.c_void_p(FAKE + 0x300000), L.LK_BF16,
+                                            C.c_void_p(FAKE + 0x400000), C.c_void_p(FAKE + 0x500000),
+                                            L.LK_BF16 if bdt is None else bdt, H, C.c_void_p(FAKE + 0x600000),
+                                            max_len, C.c_void_p(table), 0.125, C.c_void_p(FAKE + 0x700000),
+                                            L.LK_F32, C.c_void_p(ws), ws_bytes, None)
+
+
+def test_rope_validation(L):
+    k, v = cache(L), cache(L)
+    assert L.lib.lk_rope_table(7, 16, 10000.0, C.c_void_p(FAKE), None) == L.LK_ERR_SHAPE
+    assert L.lib.lk_rope_table(64, -1, 10000.0, C.c_void_p(FAKE), None) == L.LK_ERR_SHAPE
+    assert L.lib.lk_rope_table(64, 16, 1.0, C.c_void_p(FAKE), None) == L.LK_ERR_INVALID_ARG
+    assert L.lib.lk_rope_table(64, 16, 10000.0, None, None) == L.LK_ERR_INVALID_ARG
+    assert rope(L, k, v, H=48) == L.LK_ERR_SHAPE                              # not a multiple of 32
+    assert rope(L, k, v, bdt=L.LK_F32) == L.LK_ERR_DTYPE                      # factors are bf16 operands
+    assert rope(L, k, v, table=0) == L.LK_ERR_INVALID_ARG
+    assert rope(L, k, v, table=FAKE + 8) == L.LK_ERR_ALIGN
+    assert rope(L, k, v, max_len=65) == L.LK_ERR_SHAPE
+    assert rope(L, k, v, ws_bytes=16) == L.LK_ERR_WORKSPACE
+    assert rope(L, k, cache(L, kind=L.LK_I4)) == L.LK_ERR_UNSUPPORTED
+    assert L.lib.lk_latent_decode_rope_workspace_bytes(C.byref(k), C.byref(v), 64, 32) > 256
+    assert L.lib.lk_latent_decode_rope_workspace_bytes(C.byref(k), C.byref(v), 48, 32) == 0
+
+
+def test_reconstruct_validation(L):
+    k, v = cache(L), cache(L)
+
+    def rec(bdt=None, H=64, max_len=32, bk=FAKE + 0x400000):
+        return L.lib.lk_latent_reconstruct_kv(C.byref(k), C.byref(v), C.c_void_p(bk), C.c_void_p(FAKE + 0x500000),
+                                              L.LK_BF16 if bdt is None else bdt, H, C.c_void_p(FAKE + 0x600000),
+                                              max_len, C.c_void_p(FAKE + 0x700000), C.c_void_p(FAKE + 0x800000), None)
+    assert rec(bdt=L.LK_F32) == L.LK_ERR_DTYPE
+    assert rec(H=40) == L.LK_ERR_SHAPE                                       # not a multiple of 16
+    assert rec(max_len=65) == L.LK_ERR_SHAPE
+    assert rec(bk=FAKE + 0x400008) == L.LK_ERR_ALIGN

@@ -7,8 +7,13 @@
   bf16 ulp) for bf16 outputs.
 * lk_latent_reconstruct_kv: the naive path's K = dequant(C_K) B_K and V,
   stored bf16: each value within one bf16 rounding of the oracle's float64
-  product; then attending them with the dense kernel matches the latent
-  decode within the bf16 tolerance.
+  product.  Attending them with the dense kernel matches the oracle's
+  attention over its own bf16-rounded K and V within 1e-3 * RMS (a value
+  whose fp32 sum straddles a bf16 rounding boundary may land one ulp off).
+  Against the latent decode the naive path differs by what storing K and V
+  in bf16 costs: float64 attention over bf16-rounded K, V moves these cases'
+  outputs by up to 1.6% (int8 codes) and 2.7% (int4) of their RMS, so that
+  comparison allows 4e-2 * RMS.
 """
 import math
 
@@ -73,18 +78,23 @@ def test_dense_decode_matches_oracle(B, nh, H, lens, cap, out_dtype):
             assert np.all(got[b] == 0)
 
 
-@pytest.mark.parametrize("kind,ranks_k,ranks_v", [("i8", [16, 32, 8, 64], [32, 8, 64, 16]),
-                                                  ("i4", [24, 16, 32, 64], [16, 32, 24, 8])])
-def test_reconstruct_then_dense_equals_latent(kind, ranks_k, ranks_v):
+@pytest.mark.parametrize("kind,ranks_k,ranks_v,group", [
+    ("i8", [16, 32, 8, 64], [32, 8, 64, 16], 32),
+    ("i8", [12, 20, 4, 36], [44, 60, 28, 52], 32),   # ranks not multiples of 16 (zero-padded k steps)
+    ("i4", [24, 16, 32, 64], [16, 32, 24, 8], 32),   # one or two scale groups per token
+    ("i4", [48, 16, 24, 64], [40, 8, 56, 16], 8),    # groups of 8: two groups inside each 16-dim step
+    ("i4", [48, 24, 40, 64], [56, 8, 24, 16], 24),   # groups of 24 straddling the 16-dim steps
+])
+def test_reconstruct_then_dense_equals_latent(kind, ranks_k, ranks_v, group):
     lk = _lk()
     lens = [700, 33, 2049]
     B, H, cap = len(lens), 128, 2064
     rng = np.random.default_rng(5)
     lat_k = [[(rng.standard_normal((lens[b], r)) * 1.3).astype(np.float32) for r in ranks_k] for b in range(B)]
     lat_v = [[(rng.standard_normal((lens[b], r)) * 1.3).astype(np.float32) for r in ranks_v] for b in range(B)]
-    ok, ov, (rk_rows, rk_sc), (rv_rows, rv_sc) = build_caches(lat_k, lat_v, ranks_k, ranks_v, kind, 32)
-    ck = lk.LatentCache(B, ranks_k, cap, kind, 32)
-    cv = lk.LatentCache(B, ranks_v, cap, kind, 32, role="v")
+    ok, ov, (rk_rows, rk_sc), (rv_rows, rv_sc) = build_caches(lat_k, lat_v, ranks_k, ranks_v, kind, group)
+    ck = lk.LatentCache(B, ranks_k, cap, kind, group)
+    cv = lk.LatentCache(B, ranks_v, cap, kind, group, role="v")
     ck.load(rk_rows, rk_sc)
     cv.load(rv_rows, rv_sc)
     g = torch.Generator().manual_seed(6)
@@ -99,15 +109,23 @@ def test_reconstruct_then_dense_equals_latent(kind, ranks_k, ranks_v):
     offv = np.concatenate([[0], np.cumsum(ranks_v)])
     BKf, BVf = BK.double().numpy(), BV.double().numpy()
     Kc, Vc = Kr.float().cpu().numpy(), Vr.float().cpu().numpy()
+    nh = len(ranks_k)
+    want_naive = np.zeros((B, nh, H))
+    eye = np.eye(H)
     for b in range(B):
-        for h in range(len(ranks_k)):
+        for h in range(nh):
             T = lens[b]
             wk = ok.dequant(b, h) @ BKf[offk[h]:offk[h + 1]]
             wv = ov.dequant(b, h) @ BVf[offv[h]:offv[h + 1]]
             for got, want in ((Kc[b, h, :T], wk), (Vc[b, h, :T], wv)):
                 # one bf16 rounding of an fp32 sum: |err| <= 2^-8 |value| + fp32 slack
                 assert np.all(np.abs(got - want) <= 2.0 ** -8 * np.abs(want) + 1e-5 * np.abs(want).max())
+            kb = torch.from_numpy(wk).to(torch.bfloat16).double().numpy()
+            vb = torch.from_numpy(wv).to(torch.bfloat16).double().numpy()
+            want_naive[b, h] = O.attention_materialized(q[b, h].double().numpy(), kb, vb, eye, eye,
+                                                        1.0 / math.sqrt(H))
     dense = lk.dense_decode_attn(q.cuda(), Kr, Vr, seq, max(lens), out_dtype=torch.float32)
     latent = lk.latent_decode_attn(ck, cv, q.cuda(), BK.cuda(), BV.cuda(), seq, max(lens), out_dtype=torch.float32)
     torch.cuda.synchronize()
-    assert_close_bf16(dense.cpu().numpy(), latent.cpu().numpy(), 1e-2, "naive path vs latent decode")
+    assert_close_rms(dense.cpu().numpy(), want_naive, 1e-3, "naive path vs oracle on bf16 K, V")
+    assert_close_rms(dense.cpu().numpy(), latent.cpu().numpy(), 4e-2, "naive path vs latent decode")
