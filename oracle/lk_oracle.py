@@ -56,6 +56,7 @@ __all__ = [
     "per_head_svd", "round_bf16", "LatentCache", "decoder_layer_w8a8",
     "hadamard", "latent_rotation", "rotate_latents", "rmsnorm_hadamard",
     "rope_angles", "rope", "attention_rope", "latent_attention_rope",
+    "linear_w8a8_outsplit", "ffn_gate_up_swiglu",
 ]
 
 FP16_MAX = 65504.0
@@ -302,6 +303,16 @@ def latent_attention(q, cache_k, cache_v, B_K_heads, B_V_heads, softmax_scale, m
 # LASER hybrid dense + low-rank linear (LASER page §3), W8A8
 # ---------------------------------------------------------------------------
 
+def _requant_latent(acc_U, sx, s_U):
+    """The low-rank latent t = fl32(fl32(fl32(acc_U) * s_x) * s_U), requantised
+    per token with the int8 absmax rule: returns (t_q, s_t)."""
+    t = np.asarray(acc_U).astype(np.float32)
+    t = (t.astype(np.float64) * sx[:, None]).astype(np.float32)
+    t = (t.astype(np.float64)
+         * np.asarray(s_U, np.float16).astype(np.float32)[None, :]).astype(np.float32)
+    return quantize_rows_i8(t)
+
+
 def linear_w8a8_hybrid(x_q, x_scale, dense_idx, lr_idx, W_D, s_D, U, s_U, V, s_V,
                        residual=None):
     """y = x_q[:, D] W_D (dense branch) + requant(x_q[:, not D] U) V (low-rank branch).
@@ -329,17 +340,58 @@ def linear_w8a8_hybrid(x_q, x_scale, dense_idx, lr_idx, W_D, s_D, U, s_U, V, s_V
     s_t = np.zeros((M,), np.float32)
     if len(lr_idx):
         acc_U = x[:, np.asarray(lr_idx)] @ np.asarray(U, np.int64)
-        t = acc_U.astype(np.float32)
-        t = (t.astype(np.float64) * sx[:, None]).astype(np.float32)
-        t = (t.astype(np.float64)
-             * np.asarray(s_U, np.float16).astype(np.float32)[None, :]).astype(np.float32)
-        t_q, s_t = quantize_rows_i8(t)
+        t_q, s_t = _requant_latent(acc_U, sx, s_U)
         acc_V = t_q.astype(np.int64) @ np.asarray(V, np.int64)
         y += (acc_V.astype(np.float64) * s_t.astype(np.float64)[:, None]
               * np.asarray(s_V, np.float16).astype(np.float64)[None, :])
     if residual is not None:
         y += np.asarray(residual, np.float64)
     return y, t_q, s_t
+
+
+def linear_w8a8_outsplit(x_q, x_scale, dense_out, lr_out, W_D, s_D, U, s_U, V, s_V):
+    """The hybrid linear split on OUTPUT channels (LASER page §3 read as: the
+    selected hidden channels of a projection keep dense weights, the rest come
+    from the SVD factors).
+
+    x_q int8 [M, K] with per-token float32 scale s_x [M]; dense_out and
+    lr_out are disjoint sorted output-channel lists covering [0, N);
+    W_D int8 [K, |dense_out|] with fp16 scale s_D [|dense_out|]; U int8 [K, R]
+    with fp16 scale s_U [R]; V int8 [R, |lr_out|] with fp16 scale s_V
+    [|lr_out|].  Same rules as linear_w8a8_hybrid: the latent
+    t = fl32(fl32(fl32(x_q U) * s_x) * s_U) is requantised per token (t_q, s_t);
+    y[:, dense_out] = acc_D * s_x * s_D, y[:, lr_out] = acc_V * s_t * s_V
+    (float64).  Returns (y [M, N] float64, t_q, s_t).
+    """
+    x = np.asarray(x_q, np.int64)
+    sx = np.asarray(x_scale, np.float32)
+    M = x.shape[0]
+    N = len(dense_out) + len(lr_out)
+    y = np.zeros((M, N), np.float64)
+    if len(dense_out):
+        acc_D = x @ np.asarray(W_D, np.int64)
+        s_dense = np.asarray(s_D, np.float16).astype(np.float64)
+        y[:, np.asarray(dense_out)] = acc_D.astype(np.float64) * sx.astype(np.float64)[:, None] * s_dense[None, :]
+    t_q = np.zeros((M, 0), np.int8)
+    s_t = np.zeros((M,), np.float32)
+    if len(lr_out):
+        acc_U = x @ np.asarray(U, np.int64)
+        t_q, s_t = _requant_latent(acc_U, sx, s_U)
+        acc_V = t_q.astype(np.int64) @ np.asarray(V, np.int64)
+        s_lr = np.asarray(s_V, np.float16).astype(np.float64)
+        y[:, np.asarray(lr_out)] = (acc_V.astype(np.float64) * s_t.astype(np.float64)[:, None]
+                                    * s_lr[None, :])
+    return y, t_q, s_t
+
+
+def ffn_gate_up_swiglu(x_q, x_scale, gate, up):
+    """silu(gate(x)) * up(x) with both projections split on output channels
+    (linear_w8a8_outsplit; gate and up are dicts of its weight arguments).
+    Reading: gate and up keep the same hidden channels dense, so channel j of
+    both comes from the same kind of branch.  Returns [M, N] float64."""
+    g, _, _ = linear_w8a8_outsplit(x_q, x_scale, **gate)
+    u, _, _ = linear_w8a8_outsplit(x_q, x_scale, **up)
+    return swiglu(g, u)
 
 
 def swiglu(gate, up):

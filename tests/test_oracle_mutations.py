@@ -28,7 +28,8 @@ MUTANTS = {
  "scale_swap": ("* np.asarray(s_D, np.float16).astype(np.float64)[None, :])", "* np.asarray(s_V if s_V is not None else s_D, np.float16).astype(np.float64)[None, :])"),
  "nibble_swap": ("return (lo | (hi << 4)).astype(np.uint8)", "return (hi | (lo << 4)).astype(np.uint8)"),
  "i4_div8": ("s32 = _fl32_div(absmax, np.float32(7.0))", "s32 = _fl32_div(absmax, np.float32(8.0))"),
- "no_requant_sU": ("* np.asarray(s_U, np.float16).astype(np.float32)[None, :]).astype(np.float32)\n        t_q", "* 1.0).astype(np.float32)\n        t_q"),
+ "no_requant_sU": ("* np.asarray(s_U, np.float16).astype(np.float32)[None, :]).astype(np.float32)\n    return quantize_rows_i8(t)",
+                   "* 1.0).astype(np.float32)\n    return quantize_rows_i8(t)"),
  "rms_eps_out": ("np.mean(x * x, axis=-1, keepdims=True) + eps)", "np.mean(x * x, axis=-1, keepdims=True)) + eps"),
  "drop_residual": ("    if residual is not None:\n        y += np.asarray(residual, np.float64)", "    pass"),
  "v_not_BV": ("V = np.asarray(Cv_hat, np.float64) @ np.asarray(B_V, np.float64)   # [T, H]", "V = np.asarray(Cv_hat, np.float64) @ np.asarray(B_K, np.float64)   # [T, H]"),
@@ -54,6 +55,10 @@ MUTANTS = {
  "rope_query_unrotated": ("    q_rot = rope(np.asarray(q, np.float64)[None, :], [q_pos], base)[0]",
                           "    q_rot = np.asarray(q, np.float64)"),
  "rope_query_at_len": ("softmax_scale, T - 1, base)", "softmax_scale, T, base)"),
+ "outsplit_lr_scaled_by_sx": ("        y[:, np.asarray(lr_out)] = (acc_V.astype(np.float64) * s_t.astype(np.float64)[:, None]",
+                              "        y[:, np.asarray(lr_out)] = (acc_V.astype(np.float64) * sx.astype(np.float64)[:, None]"),
+ "outsplit_dense_inputs_reversed": ("        acc_D = x @ np.asarray(W_D, np.int64)", "        acc_D = x[:, ::-1] @ np.asarray(W_D, np.int64)"),
+ "ffn_gate_up_swapped": ("    return swiglu(g, u)", "    return swiglu(u, g)"),
  "layer_q_from_x": ("q = round_bf16(_linear_dense_w8a8(xq, sx, layer[\"W_Q\"], layer[\"s_Q\"]))",
                     "q = round_bf16(_linear_dense_w8a8(*quantize_rows_i8(x.astype(np.float32)), layer[\"W_Q\"], layer[\"s_Q\"]))"),
 }

@@ -667,3 +667,59 @@ def test_latent_attention_rope_query_at_last_position():
             # at position 0 of a one-token-shorter window the scores differ: the query position matters
             other = O.attention_rope(q[b, h], ck.dequant(b, h), cv.dequant(b, h), BK[h], BV[h], 0.25, 0)
             assert not np.allclose(other, want)
+
+
+# ---------------------------------------------------------------- hybrid linear split on output channels
+
+def _outsplit_tiny():
+    """K = 2 inputs, N = 3 outputs: output 1 dense, outputs 0 and 2 low-rank (R = 1)."""
+    return dict(dense_out=[1], lr_out=[0, 2], W_D=np.array([[3], [1]], np.int8), s_D=np.array([0.25], np.float16),
+                U=np.array([[3], [1]], np.int8), s_U=np.array([1.0], np.float16),
+                V=np.array([[2, -1]], np.int8), s_V=np.array([0.5, 0.25], np.float16))
+
+
+def test_outsplit_worked_example():
+    """x = [2, -1], s_x = 0.5.  Dense output 1: (2*3 - 1*1) * 0.5 * 0.25 = 0.625.
+    Latent: (2*3 - 1*1) * 0.5 * 1 = 2.5 -> s_t = fl32(2.5 / 127), code 127.
+    Low-rank outputs: 127 * 2 * s_t * 0.5 and 127 * (-1) * s_t * 0.25."""
+    x = np.array([[2, -1]], np.int8)
+    y, t_q, s_t = O.linear_w8a8_outsplit(x, np.array([0.5], np.float32), **_outsplit_tiny())
+    st = float(np.float32(2.5) / np.float32(127.0))
+    assert t_q.tolist() == [[127]] and float(s_t[0]) == st
+    np.testing.assert_array_equal(y[0], [127 * 2 * st * 0.5, 0.625, -127 * st * 0.25])
+    # gate = this projection, up = a dense projection with hand-computed outputs [1, -0.5, 1]
+    up = dict(dense_out=[0, 1, 2], lr_out=[], W_D=np.array([[1, 0, 1], [0, 1, 0]], np.int8),
+              s_D=np.array([1.0, 1.0, 1.0], np.float16), U=None, s_U=None, V=None, s_V=None)
+    m = O.ffn_gate_up_swiglu(x, np.array([0.5], np.float32), _outsplit_tiny(), up)
+    g = y[0]
+    want = [g[j] / (1.0 + math.exp(-g[j])) * u for j, u in enumerate([1.0, -0.5, 1.0])]
+    np.testing.assert_allclose(m[0], want, rtol=1e-15)
+
+
+def test_outsplit_reduces_to_the_input_split_at_the_extremes():
+    """All outputs dense = the all-dense input split (a plain int8 GEMM); no
+    outputs dense = the all-low-rank input split: the same numbers exactly."""
+    rng = np.random.default_rng(21)
+    M, K, N, R = 5, 64, 24, 16
+    x = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    sx = (rng.random(M) * 0.01 + 0.001).astype(np.float32)
+    W = rng.integers(-127, 128, (K, N)).astype(np.int8)
+    sW = (rng.random(N) * 0.01 + 0.001).astype(np.float16)
+    U = rng.integers(-127, 128, (K, R)).astype(np.int8)
+    sU = (rng.random(R) * 0.01 + 0.001).astype(np.float16)
+    V = rng.integers(-127, 128, (R, N)).astype(np.int8)
+    sV = (rng.random(N) * 0.01 + 0.001).astype(np.float16)
+    allc, none = list(range(N)), []
+    y1, _, _ = O.linear_w8a8_outsplit(x, sx, allc, none, W, sW, U, sU, V, sV)
+    y2, _, _ = O.linear_w8a8_hybrid(x, sx, list(range(K)), [], W, sW, None, None, None, None)
+    np.testing.assert_array_equal(y1, y2)
+    y3, tq3, st3 = O.linear_w8a8_outsplit(x, sx, none, allc, W, sW, U, sU, V, sV)
+    y4, tq4, st4 = O.linear_w8a8_hybrid(x, sx, [], list(range(K)), None, None, U, sU, V, sV)
+    np.testing.assert_array_equal(y3, y4)
+    np.testing.assert_array_equal(tq3, tq4)
+    # a split in between: each output channel equals the extreme it belongs to
+    D = sorted(rng.choice(N, 6, replace=False).tolist())
+    L = [j for j in range(N) if j not in D]
+    y5, _, _ = O.linear_w8a8_outsplit(x, sx, D, L, W[:, D], sW[D], U, sU, V[:, L], sV[L])
+    np.testing.assert_array_equal(y5[:, D], y1[:, D])
+    np.testing.assert_array_equal(y5[:, L], y3[:, L])
