@@ -58,6 +58,13 @@ def parse_args(argv=None):
     ap.add_argument("--attn-only", action="store_true",
                     help="time the latent decode attention alone on one layer of the workload, "
                          "its cache filled with seeded random codes (no prefill)")
+    ap.add_argument("--proj-only", action="store_true",
+                    help="time the decode-step latent projection + quantise + append alone on one layer of the "
+                         "workload (one new token per row; seq_len rewound outside the timed region)")
+    ap.add_argument("--ffn-compare", action="store_true",
+                    help="time the FFN input side (gate, up, SwiGLU, int8 requant) of the W8A8 layer shape with the "
+                         "hybrid split on input channels (two hybrid linears + SwiGLU) and on output channels "
+                         "(lk_ffn_gate_up_swiglu + requant)")
     ap.add_argument("--all-layers", action="store_true",
                     help="kept for old command lines: multi-layer workloads always time every layer")
     ap.add_argument("--no-extra", action="store_true",
@@ -230,6 +237,7 @@ class DecodeState:
 KERNEL_SOURCES = {
     "decode_attn_kernel": ["lk_decode.cu", "lk_common.cuh", "lk_internal.h"],
     "proj_cluster_kernel": ["lk_project.cu", "lk_common.cuh", "lk_quant.cuh", "lk_internal.h"],
+    "proj_mma_kernel": ["lk_project.cu", "lk_common.cuh", "lk_quant.cuh", "lk_internal.h"],
 }
 
 
@@ -802,7 +810,8 @@ def run_single(args, w):
         _finish(world)
         return 0
     hbm, peak_kind = peaks()
-    dominant = "decode_attn_kernel" if r["attn_us_per_launch"] >= r["proj_us_per_call"] else "proj_cluster_kernel"
+    dominant = "decode_attn_kernel" if r["attn_us_per_launch"] >= r["proj_us_per_call"] else (
+        "proj_mma_kernel" if w.act == "bf16" else "proj_cluster_kernel")
     ach = r["attn_gbs"] if dominant == "decode_attn_kernel" else r["proj_gbs"]
     line = {
         "metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": r["steps"],
@@ -830,6 +839,144 @@ def run_single(args, w):
     print(json.dumps(line), flush=True)
     _finish(world)
     return 0
+
+
+def run_proj_only(args):
+    """The decode-step latent projection + quantise + append alone on one layer
+    of a workload (one new token per batch row), L2 flushed before every call."""
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    import rank_latent_kv_lk_b200 as lk
+    from rank_latent_kv_lk_b200 import synth
+    from rank_latent_kv_lk_b200.configs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    rk, rv = synth.ranks(w)
+    rk, rv = rk[0], rv[0]
+    A, _, _ = synth.factors(w, 0, rk, rv)
+    A = A.to(device)
+    cap = 64
+    ck = lk.LatentCache(w.batch, rk, cap, w.kind, w.group, device)
+    cv = lk.LatentCache(w.batch, rv, cap, w.kind, w.group, device, role="v")
+    seq = torch.zeros(w.batch, dtype=torch.int32, device=device)
+    x = synth.decode_tokens(w, 0)[0].to(device)
+    if x.dtype != A.dtype:
+        x = x.to(A.dtype)
+    x_scale = a_scale = None
+    if w.act == "i8":
+        raise SystemExit("--proj-only covers the float workloads (1-4)")
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    hl = [0] * w.batch
+    for _ in range(max(3, args.warmup)):
+        seq.zero_()
+        lk.latent_project_append(ck, cv, x, A, seq, hl, x_scale, a_scale)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(1e8))
+    with ClockSampler(local) as clocks:
+        for i in range(K):
+            seq.zero_()
+            flush.fill_(1)
+            ev[i][0].record(stream)
+            lk.latent_project_append(ck, cv, x, A, seq, hl, x_scale, a_scale)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    lk.device_status()
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), world, device)
+    us = total_ms / K * 1e3
+    esz = A.element_size()
+    rb = lambda r: r if w.kind == "i8" else r // 2
+    sb = lambda r: 4 if w.kind == "i8" else 2 * (-(-r // min(w.group, r)))
+    new_bytes = w.batch * (sum(rb(r) + sb(r) for r in rk) + sum(rb(r) + sb(r) for r in rv))
+    nbytes = A.numel() * esz + x.numel() * x.element_size() + new_bytes
+    gbs = nbytes / (us * 1e-6) / 1e9
+    hbm, peak_kind = peaks()
+    kernel = "proj_mma_kernel" if w.act == "bf16" else "proj_cluster_kernel"
+    if rank == 0:
+        print(json.dumps({
+            "mode": "proj-only", "metric": "latent-projection HBM GB/s", "value": gbs * world, "unit": "GB/s",
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "us_per_call": us, "higher_is_better": True,
+            "scaling": "weak", "dtype": w.act,
+            "data": "synthetic (seeded: the workload's decode tokens and factors)",
+            "config": {"workload": w.name, "layer": 0, "batch": w.batch, "n_tot": int(A.shape[0]),
+                       "embed_dim": w.embed_dim, "l2": "flushed before every call (256 MiB write, untimed)"},
+            "algorithmic_bytes_per_call": nbytes,
+            "roofline": {"kernel": kernel, "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": gbs / hbm, "peak_kind": peak_kind,
+                         "traffic": profiled_traffic(kernel, f"{w.key}-proj")},
+            "clocks": clocks.summary(),
+        }))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_ffn_compare(args):
+    """FFN input side at the W8A8 layer shape, the two channel splits side by side."""
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    import rank_latent_kv_lk_b200 as lk
+    from rank_latent_kv_lk_b200 import synth
+    from rank_latent_kv_lk_b200.configs import WORKLOADS
+    from rank_latent_kv_lk_b200.layer import hybrid_weight
+    w = WORKLOADS[5]
+    rk, rv = synth.ranks(w)
+    lw = synth.layer_weights_w8a8(w, rk[0], rv[0])
+    gate_in = hybrid_weight(lw["gate"], w.embed_dim, w.ffn_inter, device)
+    up_in = hybrid_weight(lw["up"], w.embed_dim, w.ffn_inter, device)
+    d = synth.ffn_outsplit_weights(w)
+    ffn = lk.OutsplitFfn(d, device)
+    g = torch.Generator().manual_seed(5)
+    xq = torch.clamp(torch.round(torch.randn(w.batch, w.embed_dim, generator=g) * 40), -127, 127).to(torch.int8)
+    xq = xq.to(device)
+    sx = (torch.rand(w.batch, generator=g) * 0.01 + 0.002).to(device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def split_in():
+        gg = lk.lowrank_linear(gate_in, xq, sx)
+        uu = lk.lowrank_linear(up_in, xq, sx)
+        return lk.swiglu_quant_i8(gg, uu)
+
+    def split_out():
+        return lk.quantize_rows_i8(ffn(xq, sx))
+
+    def timed(fn, K):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        l0 = lk.kernel_launches()
+        for i in range(K):
+            flush.fill_(1)
+            ev[i][0].record()
+            fn()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        return sum(e[0].elapsed_time(e[1]) for e in ev) / K * 1e3, (lk.kernel_launches() - l0) / K
+
+    K = args.steps
+    us_in, n_in = timed(split_in, K)
+    us_out, n_out = timed(split_out, K)
+    nbytes = lambda dd: sum(v.numel() * v.element_size() for k in ("gate", "up") for v in dd[k].values())
+    b_in = sum(t.numel() * t.element_size() for name in ("gate", "up")
+               for t in (lw[name]["W_D"], lw[name]["U"], lw[name]["V"]))
+    b_out = nbytes(d)
+    hbm, peak_kind = peaks()
+    if rank == 0:
+        print(json.dumps({
+            "mode": "ffn-compare", "workload": w.name, "batch": w.batch, "hidden": w.ffn_inter,
+            "l2": "flushed before every call (256 MiB write, untimed)",
+            "input_split": {"us": us_in, "launches": n_in, "weight_bytes": b_in, "gbs": b_in / us_in / 1e3},
+            "output_split_fused": {"us": us_out, "launches": n_out, "weight_bytes": b_out,
+                                   "gbs": b_out / us_out / 1e3},
+            "peak_gbs": hbm, "peak_kind": peak_kind,
+        }))
 
 
 def run_attn_only(args):
@@ -1122,6 +1269,10 @@ def main(argv=None):
         return run_reference(args)
     if args.attn_only:
         return run_attn_only(args)
+    if args.proj_only:
+        return run_proj_only(args)
+    if args.ffn_compare:
+        return run_ffn_compare(args)
     if args.layer:
         return run_layer(args)
     if args.dense_compare:

@@ -380,6 +380,45 @@ lk_status lk_lowrank_linear(const lk_lowrank_weight* w, const int8_t* x_q, const
 size_t lk_lowrank_workspace_bytes(const lk_lowrank_weight* w, int32_t m);
 
 /*
+ * The FFN input side with the hybrid split on OUTPUT (hidden) channels
+ * (LASER technical summary §3: the selected hidden channels keep dense
+ * weights, the rest come from the SVD factors; §4: the input projections,
+ * the latent activation and SwiGLU fused), W8A8.  Gate and up keep the same
+ * hidden channels dense: dense_out (device int32 [n_dense]) lists them, in
+ * the order of the W_D rows, and lr_out (device int32 [n_out - n_dense]) the
+ * others, in the order of the V rows; together they cover [0, n_out) once.
+ * For each token row m and projection P in {gate, up}:
+ *   channel dense_out[i]: P = fl32(fl32(acc * s_x[m]) * s_D[i]),
+ *                         acc = x_q[m] . W_D[i]                (exact int32)
+ *   latent:   t = fl32(fl32(fl32(x_q[m] . U[k]) * s_x[m]) * s_U[k]), k < rank,
+ *             requantised per token with the int8 absmax rule -> (t_q, s_t)
+ *   channel lr_out[i]:    P = fl32(fl32(acc * s_t[m]) * s_V[i]), acc = t_q . V[i]
+ *   out[m][j] = silu(gate_j) * up_j = gate_j / (1 + exp(-gate_j)) * up_j  (fp32)
+ * Launches: the two latent products (tcgen05 int8 GEMM), one requantisation
+ * of both, then one launch for gate, up and SwiGLU together.
+ * Weights (per projection): W_D int8 [n_dense][k_in], U int8 [rank][k_in],
+ * V int8 [n_out - n_dense][rank] (rows contiguous along the contraction),
+ * fp16 scales; all 16-byte aligned.  k_in and rank multiples of 16; rank > 0
+ * exactly when n_dense < n_out.  x_q int8 [m][k_in] (16-byte aligned),
+ * x_scale fp32 [m]; out fp32 [m][n_out].  workspace:
+ * lk_ffn_gate_up_swiglu_workspace_bytes(...) bytes, 256-byte aligned.
+ */
+typedef struct {
+  const int8_t* W_D;
+  const uint16_t* s_D;
+  const int8_t* U;
+  const uint16_t* s_U;
+  const int8_t* V;
+  const uint16_t* s_V;
+} lk_outsplit_weight;
+
+lk_status lk_ffn_gate_up_swiglu(const lk_outsplit_weight* gate, const lk_outsplit_weight* up, int32_t k_in,
+                                int32_t n_out, int32_t n_dense, int32_t rank, const int32_t* dense_out,
+                                const int32_t* lr_out, const int8_t* x_q, const float* x_scale, int32_t m,
+                                float* out, void* workspace, size_t workspace_bytes, lk_stream_t stream);
+size_t lk_ffn_gate_up_swiglu_workspace_bytes(int32_t rank, int32_t m);
+
+/*
  * Stand-alone latent quantiser (the rule lk_latent_project_append applies),
  * exposed for bit-exact testing.  v: fp32 [m, r].
  *  LK_I8: scale = fl32(absmax / 127); code = clamp(rint(fl32(v / scale)),

@@ -9,7 +9,7 @@ import importlib
 _API = ("LatentCache", "LowrankWeight", "device_status", "latent_decode_attn", "latent_decode_step",
         "latent_project_append", "lowrank_linear", "quantize_latent", "quantize_rows_i8", "rmsnorm_quant_i8",
         "rmsnorm_hadamard_quant_i8", "swiglu_quant_i8", "workspaces", "kernel_launches", "dense_decode_attn", "reconstruct_kv",
-        "rope_table", "latent_decode_attn_rope")
+        "rope_table", "latent_decode_attn_rope", "OutsplitFfn")
 
 
 def __getattr__(name):

@@ -61,6 +61,17 @@ class LowrankWeightDesc(C.Structure):
     ]
 
 
+class OutsplitWeightDesc(C.Structure):
+    _fields_ = [
+        ("W_D", C.c_void_p),
+        ("s_D", C.c_void_p),
+        ("U", C.c_void_p),
+        ("s_U", C.c_void_p),
+        ("V", C.c_void_p),
+        ("s_V", C.c_void_p),
+    ]
+
+
 class LkError(RuntimeError):
     def __init__(self, status, message):
         super().__init__(f"{message} (status {status})")
@@ -99,6 +110,9 @@ def _load():
         "lk_dense_decode_workspace_bytes": (SZ, [I32, I32, I32, I32]),
         "lk_latent_reconstruct_kv": (C.c_int, [CP, CP, P, P, C.c_int, I32, P, I32, P, P, P]),
         "lk_rope_table": (C.c_int, [I32, I32, C.c_float, P, P]),
+        "lk_ffn_gate_up_swiglu": (C.c_int, [C.POINTER(OutsplitWeightDesc), C.POINTER(OutsplitWeightDesc), I32, I32,
+                                            I32, I32, P, P, P, P, I32, P, P, SZ, P]),
+        "lk_ffn_gate_up_swiglu_workspace_bytes": (SZ, [I32, I32]),
         "lk_latent_decode_attn_rope": (C.c_int, [CP, CP, P, C.c_int, P, P, C.c_int, I32, P, I32, P, C.c_float, P,
                                                  C.c_int, P, SZ, P]),
         "lk_latent_decode_rope_workspace_bytes": (SZ, [CP, CP, I32, I32]),

@@ -10,7 +10,8 @@ import math
 
 import torch
 
-from ._lib import LK_BF16, LK_F16, LK_F32, LK_I4, LK_I8, LatentCacheDesc, LowrankWeightDesc, check, lib
+from ._lib import (LK_BF16, LK_F16, LK_F32, LK_I4, LK_I8, LatentCacheDesc, LowrankWeightDesc, OutsplitWeightDesc,
+                   check, lib)
 from .layout import CacheGeometry
 
 _DT = {torch.float32: LK_F32, torch.bfloat16: LK_BF16, torch.float16: LK_F16, torch.int8: LK_I8}
@@ -185,6 +186,37 @@ def dense_decode_attn(q, K, V, seq_len, max_seq_len, softmax_scale=None, out=Non
                                    float(softmax_scale), _ptr(out), _dtype_code(out), _ptr(ws), ws.numel(),
                                    _stream(stream)))
     return out
+
+
+class OutsplitFfn:
+    """Device gate and up weights of the FFN split on output channels (int8,
+    fp16 scales; see lk_ffn_gate_up_swiglu).  d: a dict as from
+    synth.ffn_outsplit_weights."""
+
+    def __init__(self, d, device="cuda"):
+        self.k_in, self.n_out, self.rank, self.n_dense = d["k_in"], d["n_out"], d["rank"], d["n_dense"]
+        self.dense_out = d["dense_out"].to(device)
+        self.lr_out = d["lr_out"].to(device)
+        self._keep = []
+        self._desc = []
+        for name in ("gate", "up"):
+            t = {k: v.to(device) for k, v in d[name].items()}
+            self._keep.append(t)
+            self._desc.append(OutsplitWeightDesc(*[t[k].data_ptr() if t[k].numel() else None
+                                                   for k in ("W_D", "s_D", "U", "s_U", "V", "s_V")]))
+
+    def __call__(self, x_q, x_scale, out=None, stream=None):
+        """silu(gate(x)) * up(x): fp32 [m, n_out]."""
+        m = x_q.shape[0]
+        if out is None:
+            out = torch.empty((m, self.n_out), dtype=torch.float32, device=x_q.device)
+        need = lib.lk_ffn_gate_up_swiglu_workspace_bytes(self.rank, m)
+        ws = workspaces.get("ffn_outsplit", need, x_q.device)
+        check(lib.lk_ffn_gate_up_swiglu(C.byref(self._desc[0]), C.byref(self._desc[1]), self.k_in, self.n_out,
+                                        self.n_dense, self.rank, _ptr(self.dense_out), _ptr(self.lr_out),
+                                        _ptr(x_q), _ptr(x_scale), m, _ptr(out), _ptr(ws), ws.numel(),
+                                        _stream(stream)))
+        return out
 
 
 def rope_table(head_dim, max_pos, base=10000.0, device="cuda", stream=None):

@@ -380,6 +380,54 @@ lk_status lk_dense_decode_attn(const void* q, const void* K, const void* V, int3
   return LK_OK;
 }
 
+size_t lk_ffn_gate_up_swiglu_workspace_bytes(int32_t rank, int32_t m) {
+  if (rank < 0 || m < 0) return 0;
+  return lk::ffn_workspace_bytes(m, rank);
+}
+
+lk_status lk_ffn_gate_up_swiglu(const lk_outsplit_weight* gate, const lk_outsplit_weight* up, int32_t k_in,
+                                int32_t n_out, int32_t n_dense, int32_t rank, const int32_t* dense_out,
+                                const int32_t* lr_out, const int8_t* x_q, const float* x_scale, int32_t m,
+                                float* out, void* workspace, size_t workspace_bytes, lk_stream_t stream) {
+  if (!gate || !up) return fail(LK_ERR_INVALID_ARG, "null weight descriptor");
+  if (k_in < 16 || k_in % 16 || n_out < 1 || n_dense < 0 || n_dense > n_out || rank < 0 || rank % 16)
+    return fail(LK_ERR_SHAPE, "bad k_in %d / n_out %d / n_dense %d / rank %d", k_in, n_out, n_dense, rank);
+  if ((n_dense < n_out) != (rank > 0))
+    return fail(LK_ERR_SHAPE, "rank %d must be > 0 exactly when some channels are low-rank", rank);
+  if (m < 0 || m > 65535) return fail(LK_ERR_SHAPE, "m %d outside [0, 65535]", m);
+  if (m > 0 && (!x_q || !x_scale || !out)) return fail(LK_ERR_INVALID_ARG, "null x_q, x_scale or out");
+  for (const lk_outsplit_weight* w : {gate, up}) {
+    if (n_dense > 0 && (!w->W_D || !w->s_D || !dense_out))
+      return fail(LK_ERR_INVALID_ARG, "null dense weights, scales or channel list");
+    if (n_dense < n_out && (!w->U || !w->s_U || !w->V || !w->s_V || !lr_out))
+      return fail(LK_ERR_INVALID_ARG, "null low-rank weights, scales or channel list");
+    if (!aligned(w->W_D, 16) || !aligned(w->U, 16) || !aligned(w->V, 16))
+      return fail(LK_ERR_ALIGN, "weights must be 16-byte aligned");
+  }
+  if (!aligned(x_q, 16)) return fail(LK_ERR_ALIGN, "x_q must be 16-byte aligned");
+  const size_t need = lk::ffn_workspace_bytes(m, rank);
+  if (!workspace || workspace_bytes < need)
+    return fail(LK_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
+  if (!aligned(workspace, 256)) return fail(LK_ERR_ALIGN, "workspace must be 256-byte aligned");
+  lk::FfnLaunch a{};
+  a.gate = {gate->W_D, gate->s_D, gate->U, gate->s_U, gate->V, gate->s_V};
+  a.up = {up->W_D, up->s_D, up->U, up->s_U, up->V, up->s_V};
+  a.dense_out = dense_out;
+  a.lr_out = lr_out;
+  a.x_q = x_q;
+  a.x_scale = x_scale;
+  a.out = out;
+  a.workspace = workspace;
+  a.m = m;
+  a.k_in = k_in;
+  a.n_out = n_out;
+  a.n_dense = n_dense;
+  a.rank = rank;
+  cudaError_t e = lk::launch_ffn_gate_up(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lk_ffn_gate_up_swiglu");
+  return LK_OK;
+}
+
 lk_status lk_rope_table(int32_t head_dim, int32_t max_pos, float base, float* table, lk_stream_t stream) {
   if (head_dim < 2 || head_dim > LK_MAX_HEAD_DIM || head_dim % 2 != 0)
     return fail(LK_ERR_SHAPE, "head_dim %d must be even in [2, %d]", head_dim, LK_MAX_HEAD_DIM);

@@ -48,6 +48,28 @@ size_t decode_workspace_bytes(int units, int rv_max, int max_len, int n_split);
 cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream);
 
 
+// ---------------------------------------------------------------- FFN input side split on output channels
+struct OutsplitWeights {
+  const int8_t* W_D;    // [n_dense][k_in]
+  const uint16_t* s_D;  // fp16 [n_dense]
+  const int8_t* U;      // [rank][k_in]
+  const uint16_t* s_U;  // fp16 [rank]
+  const int8_t* V;      // [n_out - n_dense][rank]
+  const uint16_t* s_V;  // fp16 [n_out - n_dense]
+};
+struct FfnLaunch {
+  OutsplitWeights gate, up;
+  const int32_t* dense_out;  // device [n_dense]
+  const int32_t* lr_out;     // device [n_out - n_dense]
+  const int8_t* x_q;
+  const float* x_scale;
+  float* out;
+  void* workspace;
+  int m, k_in, n_out, n_dense, rank;
+};
+size_t ffn_workspace_bytes(int m, int rank);
+cudaError_t launch_ffn_gate_up(const FfnLaunch& a, cudaStream_t stream);
+
 // ---------------------------------------------------------------- rotary-position decode
 struct RopeLaunch {
   const void* codes_k;

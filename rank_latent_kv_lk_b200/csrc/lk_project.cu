@@ -476,19 +476,6 @@ __global__ void __launch_bounds__(kMmaWarps * 32) proj_mma_kernel(const __grid_c
   const uint16_t* A0 = p.A + (int64_t)min(col0 + gid, f.n_tot - 1) * E;
   const uint16_t* A1 = p.A + (int64_t)min(col0 + gid + 8, f.n_tot - 1) * E;
   if (threadIdx.x == 0) nfin = 0;
-  // The CTA's weight rows are one contiguous range: ask for all of it in L2
-  // at once (bulk prefetches, 16 KB each), so HBM streams at full rate while
-  // the warps' own loads, whose number in flight the register budget caps,
-  // find their lines in L2.
-  if (threadIdx.x < 32) {
-    const int nrows = min(16, f.n_tot - col0);
-    const char* base = reinterpret_cast<const char*>(p.A + (int64_t)col0 * E);
-    const int64_t bytes = (int64_t)nrows * E * 2;
-    for (int64_t off = (int64_t)threadIdx.x * 16384; off < bytes; off += 32 * 16384) {
-      const uint32_t n = (uint32_t)min((int64_t)16384, bytes - off);
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + off), "r"(n) : "memory");
-    }
-  }
   float c[NT][4];
 #pragma unroll
   for (int t = 0; t < NT; ++t) c[t][0] = c[t][1] = c[t][2] = c[t][3] = 0.0f;

@@ -147,6 +147,29 @@ def layer_weights_w8a8(w, ranks_k, ranks_v):
     return out
 
 
+def ffn_outsplit_weights(w, k_in=None, n_out=None, rank=None, dense_frac=None, seed_purpose=None):
+    """Gate and up weights of the FFN split on output channels (CPU), with the
+    workload's int8 recipe: a seeded dense_frac of the hidden channels (a
+    multiple of 16) keep dense rows W_D [n_dense, k_in], the others come from
+    U [rank, k_in] and V [n_out - n_dense, rank].  Gate and up share the split."""
+    g = generator(w, WEIGHTS if seed_purpose is None else seed_purpose)
+    k_in = w.embed_dim if k_in is None else k_in
+    n_out = w.ffn_inter if n_out is None else n_out
+    rank = w.ffn_rank if rank is None else rank
+    frac = w.ffn_dense_frac if dense_frac is None else dense_frac
+    n_dense = int(round(frac * n_out / 16)) * 16
+    perm = torch.randperm(n_out, generator=g)
+    dense_out = torch.sort(perm[:n_dense]).values.to(torch.int32)
+    lr_out = torch.sort(perm[n_dense:]).values.to(torch.int32)
+    out = dict(dense_out=dense_out, lr_out=lr_out, k_in=k_in, n_out=n_out, rank=rank, n_dense=n_dense)
+    for name in ("gate", "up"):
+        W_D, s_D = int8_weight(g, n_dense, k_in)
+        U, s_U = int8_weight(g, rank, k_in)
+        V, s_V = int8_weight(g, n_out - n_dense, rank)
+        out[name] = dict(W_D=W_D, s_D=s_D, U=U, s_U=s_U, V=V, s_V=s_V)
+    return out
+
+
 def as_numpy(t):
     """Exact host copy of a tensor as numpy (bf16 values widened to float32)."""
     t = t.detach().cpu()

@@ -215,3 +215,22 @@ def test_reconstruct_validation(L):
     assert rec(H=40) == L.LK_ERR_SHAPE                                       # not a multiple of 16
     assert rec(max_len=65) == L.LK_ERR_SHAPE
     assert rec(bk=FAKE + 0x400008) == L.LK_ERR_ALIGN
+
+
+def test_ffn_outsplit_validation(L):
+    w = L.OutsplitWeightDesc(FAKE, FAKE + 0x1000, FAKE + 0x2000, FAKE + 0x3000, FAKE + 0x4000, FAKE + 0x5000)
+
+    def ffn(k_in=256, n_out=64, n_dense=16, rank=32, m=4, ws_bytes=1 << 24, wd=None):
+        return L.lib.lk_ffn_gate_up_swiglu(C.byref(w if wd is None else wd), C.byref(w), k_in, n_out, n_dense, rank,
+                                           C.c_void_p(FAKE + 0x6000), C.c_void_p(FAKE + 0x7000),
+                                           C.c_void_p(FAKE + 0x8000), C.c_void_p(FAKE + 0x9000), m,
+                                           C.c_void_p(FAKE + 0xA000), C.c_void_p(FAKE + 0x100000), ws_bytes, None)
+    assert ffn(k_in=250) == L.LK_ERR_SHAPE
+    assert ffn(rank=24) == L.LK_ERR_SHAPE
+    assert ffn(n_dense=65) == L.LK_ERR_SHAPE
+    assert ffn(n_dense=64, rank=32) == L.LK_ERR_SHAPE          # no low-rank channel but a rank
+    assert ffn(n_dense=16, rank=0) == L.LK_ERR_SHAPE
+    assert ffn(ws_bytes=16) == L.LK_ERR_WORKSPACE
+    bad = L.OutsplitWeightDesc(FAKE + 4, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert ffn(wd=bad) == L.LK_ERR_ALIGN
+    assert L.lib.lk_ffn_gate_up_swiglu_workspace_bytes(512, 32) >= 2 * 32 * 512 * 4
