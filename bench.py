@@ -65,6 +65,9 @@ def parse_args(argv=None):
                     help="time the FFN input side (gate, up, SwiGLU, int8 requant) of the W8A8 layer shape with the "
                          "hybrid split on input channels (two hybrid linears + SwiGLU) and on output channels "
                          "(lk_ffn_gate_up_swiglu + requant)")
+    ap.add_argument("--rope", action="store_true",
+                    help="time the rotary-position decode (keys rebuilt on chip) against the absorbed latent decode "
+                         "on one layer of workloads 2-4 (the same caches)")
     ap.add_argument("--all-layers", action="store_true",
                     help="kept for old command lines: multi-layer workloads always time every layer")
     ap.add_argument("--no-extra", action="store_true",
@@ -1175,6 +1178,68 @@ def run_layer(args):
     return 0
 
 
+def run_rope(args):
+    """The rotary-position decode (lk_latent_decode_attn_rope: keys rebuilt on
+    chip, rotated) against the absorbed decode on the same caches, one layer
+    of workloads 2-4, L2 flushed before every launch."""
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    import rank_latent_kv_lk_b200 as lk
+    from rank_latent_kv_lk_b200 import synth
+    from rank_latent_kv_lk_b200.configs import WORKLOADS
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+        for e in ev:
+            flush.fill_(1)
+            e[0].record()
+            fn()
+            e[1].record()
+        torch.cuda.synchronize()
+        return statistics.median(e[0].elapsed_time(e[1]) * 1e3 for e in ev)
+
+    hbm, peak_kind = peaks()
+    lines = []
+    for key in (2, 3, 4):
+        w = WORKLOADS[key]
+        rk, rv = synth.ranks(w)
+        rk, rv = rk[0], rv[0]
+        _, BK, BV = synth.factors(dataclasses.replace(w, act="bf16"), 0, rk, rv)
+        BK, BV = BK.to(device), BV.to(device)
+        T = w.context + 1
+        g = torch.Generator(device=device)
+        g.manual_seed(synth.seed_for(w, synth.CONTEXT))
+        ck = lk.LatentCache(w.batch, rk, w.capacity, w.kind, w.group, device)
+        cv = lk.LatentCache(w.batch, rv, w.capacity, w.kind, w.group, device, role="v")
+        for c in (ck, cv):
+            c.codes.copy_(torch.randint(0, 256, c.codes.shape, dtype=torch.uint8, device=device, generator=g))
+            c.scales.copy_((torch.rand(c.scales.shape, device=device, generator=g) * 0.02 + 0.01).to(c.scales.dtype))
+        q = torch.randn(w.batch, w.n_heads, w.head_dim, generator=g, device=device).to(torch.bfloat16)
+        seq = torch.full((w.batch,), T, dtype=torch.int32, device=device)
+        out = torch.empty(w.batch, w.n_heads, w.head_dim, dtype=torch.bfloat16, device=device)
+        table = lk.rope_table(w.head_dim, w.capacity)
+        absorbed_us = timed(lambda: lk.latent_decode_attn(ck, cv, q, BK, BV, seq, T, out=out), args.steps)
+        rope_us = timed(lambda: lk.latent_decode_attn_rope(ck, cv, q, BK, BV, seq, T, table, out=out), args.steps)
+        rb = lambda r: r if w.kind == "i8" else r // 2
+        sb = lambda r: 4 if w.kind == "i8" else 2 * (-(-r // min(w.group, r)))
+        cache_bytes = w.batch * T * (sum(rb(r) + sb(r) for r in rk) + sum(rb(r) + sb(r) for r in rv))
+        flops = 2.0 * w.batch * T * sum(rk) * w.head_dim  # the key rebuild on the tensor cores
+        lines.append({"workload": w.name, "batch": w.batch, "tokens": T, "absorbed_us": absorbed_us,
+                      "rope_us": rope_us, "rope_cache_gbs": cache_bytes / rope_us / 1e3,
+                      "rope_frac_of_measured_hbm": cache_bytes / rope_us / 1e3 / hbm,
+                      "rope_key_rebuild_tflops": flops / rope_us / 1e6, "rope_over_absorbed": rope_us / absorbed_us})
+        del ck, cv
+        torch.cuda.empty_cache()
+    if rank == 0:
+        print(json.dumps({"mode": "rope", "l2": "flushed before every launch (256 MiB write, untimed)",
+                          "peak_gbs": hbm, "peak_kind": peak_kind, "results": lines}))
+
+
 def run_dense_compare(args):
     """The decode speed-up the pages report (latent attention vs flash decoding
     over dense K/V; the naive path that rebuilds K and V through memory), per
@@ -1273,6 +1338,8 @@ def main(argv=None):
         return run_proj_only(args)
     if args.ffn_compare:
         return run_ffn_compare(args)
+    if args.rope:
+        return run_rope(args)
     if args.layer:
         return run_layer(args)
     if args.dense_compare:

@@ -306,7 +306,9 @@ size_t lk_dense_decode_workspace_bytes(int32_t batch, int32_t n_heads, int32_t h
  * LK_BF16; B_K, B_V: bf16 (b_dtype LK_BF16), packed per head as for
  * lk_latent_decode_attn; head_dim a multiple of 32 (<= LK_MAX_HEAD_DIM);
  * rope_table: an lk_rope_table table of the same head_dim with at least
- * max_seq_len rows; q, B_K, B_V, rope_table 16-byte aligned.  out:
+ * max(max_seq_len, 16) rows (the kernel takes the angles of positions inside
+ * a 16-token block from the block's row and rows 0..15 by the angle-sum
+ * identities, in fp32); q, B_K, B_V, rope_table 16-byte aligned.  out:
  * [B, n_heads, head_dim] LK_F32 or LK_BF16; rows with len = 0 are zero.
  * workspace: lk_latent_decode_rope_workspace_bytes(...) bytes, 256-byte
  * aligned, its first round_up(4 * B * n_heads, 256) bytes zero at entry

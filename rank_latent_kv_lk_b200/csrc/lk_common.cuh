@@ -253,3 +253,16 @@ LK_DEVICE uint32_t lk_pack_bf16x2(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+
+// ---------------------------------------------------------------- cp.async (16 bytes, L1 bypassed)
+// Copies 16 bytes from global to shared memory asynchronously (both 16-byte
+// aligned).  lk_cp_async_commit closes a group; lk_cp_async_wait<N> waits
+// until at most N of this thread's groups are pending.
+LK_DEVICE void lk_cp_async16(void* dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(lk_smem_addr(dst_smem)), "l"(src) : "memory");
+}
+LK_DEVICE void lk_cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+LK_DEVICE void lk_cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}

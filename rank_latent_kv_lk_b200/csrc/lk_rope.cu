@@ -11,7 +11,9 @@
 //   s_t = <rot(K_t, t), rot(q, len - 1)> * softmax_scale
 //   u = sum_t softmax(s)_t sigma_V[t] c_V[t];  out = u B_V^h   (V not rotated)
 // rot turns the pairs (i, i + H/2) by t * base^(-2 i / H), with cos / sin
-// read from a table the library builds once (lk_rope_table).
+// from a table the library builds once (lk_rope_table): per 16-token block
+// one table row, and for the positions inside the block the angle-sum
+// identities with the table's rows 0..15.
 //
 // Work split: each (b, h) unit's positions are cut into pieces of a fixed
 // number of 128-token tiles; a CTA of 8 warps takes one piece.  Per tile the
@@ -62,24 +64,30 @@ struct RopeParams {
 };
 
 struct Smem {
-  int off_kc, off_vc, off_ks, off_vs, off_bk, off_q, off_wst, off_cta, total;
+  int off_kc, off_raw, raw_bytes, r_vc, r_ks, r_vs, r_ang, off_bk, off_q, off_wst, off_cta, off_to, total;
 };
 
-// Shared-memory plan (bytes) for ranks up to rk16 / rv and group counts up
-// to ngk / ngv: bf16 key codes [kTile][rk16 + 8], raw value codes, fp32
-// scales, bf16 B_K [rk16][H + 8], the rotated query, per-warp states.
-Smem smem_plan(int rk16, int rvb_max, int ngk, int ngv, int H) {
+// Shared-memory plan (bytes): bf16 key codes [kTile][rk16 + 8] (converted
+// per tile); two raw staging slots, each holding one tile's key codes, value
+// codes, both scale planes and the table rows of its 16-token blocks (filled
+// by cp.async one tile ahead); bf16 B_K [rk16][H + 8]; the rotated query;
+// per-warp states; the table rows of positions 0..15.
+Smem smem_plan(int rk16, int rbk_max, int rvb_max, int ngk, int ngv, int ssz, int H) {
   auto up = [](int x) { return (x + 15) & ~15; };
   Smem s;
   s.off_kc = 0;
-  s.off_vc = s.off_kc + up(kTile * (rk16 + 8) * 2);
-  s.off_ks = s.off_vc + up(kTile * rvb_max);
-  s.off_vs = s.off_ks + up(kTile * ngk * 4);
-  s.off_bk = s.off_vs + up(kTile * ngv * 4);
+  s.off_raw = up(kTile * (rk16 + 8) * 2);
+  s.r_vc = up(kTile * rbk_max);
+  s.r_ks = s.r_vc + up(kTile * rvb_max);
+  s.r_vs = s.r_ks + up(kTile * ngk * ssz);
+  s.r_ang = s.r_vs + up(kTile * ngv * ssz);
+  s.raw_bytes = s.r_ang + up((kTile / 16) * (H / 2) * 8);
+  s.off_bk = s.off_raw + 2 * s.raw_bytes;
   s.off_q = s.off_bk + up(rk16 * (H + 8) * 2);
   s.off_wst = s.off_q + up(H * 4);
   s.off_cta = s.off_wst + up(kWarps * (2 + kMaxR) * 4);
-  s.total = s.off_cta + up((2 + kMaxR) * 4 + 16);
+  s.off_to = s.off_cta + up((2 + kMaxR) * 4 + 16);
+  s.total = s.off_to + up(16 * (H / 2) * 8);
   return s;
 }
 
@@ -93,8 +101,7 @@ LK_DEVICE float scale_at(const uint8_t* base, int64_t i, int kind) {
 }
 
 __global__ void __launch_bounds__(kThreads, 2) rope_decode_kernel(const __grid_constant__ RopeParams p,
-                                                                   int off_kc, int off_vc, int off_ks, int off_vs,
-                                                                   int off_bk, int off_q, int off_wst, int off_cta) {
+                                                                   const __grid_constant__ Smem L) {
   extern __shared__ __align__(16) uint8_t sm[];
   const int u = blockIdx.y, piece = blockIdx.x;
   const int b = u / p.n_heads, h = u - b * p.n_heads;
@@ -110,15 +117,13 @@ __global__ void __launch_bounds__(kThreads, 2) rope_decode_kernel(const __grid_c
   const int gk = p.gk[h], gv = p.gv[h];
   const int ngk = (rk + gk - 1) / gk, ngv = (rv + gv - 1) / gv;
   const int cst = rk16 + 8, bst = H + 8;
-  uint16_t* Kc = reinterpret_cast<uint16_t*>(sm + off_kc);
-  uint8_t* Vc = sm + off_vc;
-  float* Ks = reinterpret_cast<float*>(sm + off_ks);
-  float* Vs = reinterpret_cast<float*>(sm + off_vs);
-  uint16_t* Bs = reinterpret_cast<uint16_t*>(sm + off_bk);
-  float* qr = reinterpret_cast<float*>(sm + off_q);
-  float* wst = reinterpret_cast<float*>(sm + off_wst);
-  float* cta = reinterpret_cast<float*>(sm + off_cta);
+  uint16_t* Kc = reinterpret_cast<uint16_t*>(sm + L.off_kc);
+  uint16_t* Bs = reinterpret_cast<uint16_t*>(sm + L.off_bk);
+  float* qr = reinterpret_cast<float*>(sm + L.off_q);
+  float* wst = reinterpret_cast<float*>(sm + L.off_wst);
+  float* cta = reinterpret_cast<float*>(sm + L.off_cta);
   int* ticket = reinterpret_cast<int*>(cta + 2 + kMaxR);
+  float2* ang_off = reinterpret_cast<float2*>(sm + L.off_to);  // [j < 16][half]: (cos, sin) of position j
 
   float m_run = -INFINITY, l_run = 0.0f;
   float u0 = 0.0f, u1 = 0.0f;  // latent value sums of dims lane and lane + 32
@@ -138,6 +143,7 @@ __global__ void __launch_bounds__(kThreads, 2) rope_decode_kernel(const __grid_c
       const uint4 v = d < rk ? *reinterpret_cast<const uint4*>(Bg + (int64_t)d * H + 8 * c8) : make_uint4(0, 0, 0, 0);
       *reinterpret_cast<uint4*>(Bs + d * bst + 8 * c8) = v;
     }
+    for (int i = threadIdx.x; i < 16 * half; i += kThreads) ang_off[i] = reinterpret_cast<const float2*>(p.table)[i];
     // key code dims rk .. rk16 stay zero for every tile
     for (int i = threadIdx.x; i < kTile * (rk16 - rk); i += kThreads) {
       const int t = i / (rk16 - rk);
@@ -151,15 +157,50 @@ __global__ void __launch_bounds__(kThreads, 2) rope_decode_kernel(const __grid_c
   const int csk = lk_chunk_bytes(rbk);
   const int nks = rk16 / 16;
 
-  for (int t0 = t_begin; t0 < t_end; t0 += kTile) {
+  const int ssz = p.kind == 0 ? 4 : 2;
+  const int ntiles = t_begin < t_end ? (t_end - t_begin + kTile - 1) / kTile : 0;
+  // raw copies of tile ti into staging slot `slot` (16-byte cp.async chunks;
+  // every region is a whole number of chunks: tiles are whole 16-token blocks)
+  auto issue = [&](int ti, int slot) {
+    const int t0 = t_begin + ti * kTile;
+    const int n16 = (min(kTile, t_end - t0) + 15) & ~15;
+    uint8_t* r = sm + L.off_raw + slot * L.raw_bytes;
+    const uint8_t* srcs[4] = {kplane + (int64_t)t0 * rbk, vplane + (int64_t)t0 * rbv,
+                              p.scales_k + (ks_base + (int64_t)t0 * ngk) * ssz,
+                              p.scales_v + (vs_base + (int64_t)t0 * ngv) * ssz};
+    const int offs[4] = {0, L.r_vc, L.r_ks, L.r_vs};
+    const int bytes[4] = {n16 * rbk, n16 * rbv, n16 * ngk * ssz, n16 * ngv * ssz};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      for (int i = threadIdx.x; i < bytes[q] / 16; i += kThreads) lk_cp_async16(r + offs[q] + 16 * i, srcs[q] + 16 * i);
+    const int rowc = half / 2;  // 16-byte chunks of one table row
+    for (int i = threadIdx.x; i < (n16 / 16) * rowc; i += kThreads) {
+      const int blk = i / rowc, c = i - blk * rowc;
+      lk_cp_async16(r + L.r_ang + (blk * rowc + c) * 16,
+                    reinterpret_cast<const uint8_t*>(p.table) + ((int64_t)(t0 + 16 * blk) * half * 2) * 4 + 16 * c);
+    }
+  };
+  if (ntiles > 0) issue(0, 0);
+  lk_cp_async_commit();
+
+  for (int ti = 0; ti < ntiles; ++ti) {
+    const int t0 = t_begin + ti * kTile;
     const int ntok = min(kTile, t_end - t0);
     const int ntok16 = (ntok + 15) & ~15;  // whole 16-token blocks (inside the capacity)
-    __syncthreads();  // the previous tile's buffers are free
+    if (ti + 1 < ntiles) issue(ti + 1, (ti + 1) & 1);  // the next tile streams in while this one is computed
+    lk_cp_async_commit();
+    lk_cp_async_wait<1>();  // this tile's copies (issued by this thread) have landed
+    __syncthreads();        // ... and every thread's
+    const uint8_t* raw = sm + L.off_raw + (ti & 1) * L.raw_bytes;
+    const uint8_t* Vc = raw + L.r_vc;
+    const uint8_t* Ks = raw + L.r_ks;
+    const uint8_t* Vs = raw + L.r_vs;
+    const float2* ang_blk = reinterpret_cast<const float2*>(raw + L.r_ang);  // [block][half]: its first position
     // key codes -> bf16 rows (token-major chunks: each word is 4 bytes of one token)
     {
-      const uint32_t* src = reinterpret_cast<const uint32_t*>(kplane + (int64_t)t0 * rbk);
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(raw);
       for (int i = threadIdx.x; i < ntok16 * rbk / 4; i += kThreads) {
-        const uint32_t w = __ldg(src + i);
+        const uint32_t w = src[i];
         const int o = 4 * i;
         const int blk = o / (16 * rbk), rem = o - blk * 16 * rbk;
         const int ch = rem / (16 * csk), rem2 = rem - ch * 16 * csk;
@@ -177,14 +218,6 @@ __global__ void __launch_bounds__(kThreads, 2) rope_decode_kernel(const __grid_c
         }
       }
     }
-    // value codes as they are (dimension-major 16-token blocks), 16-byte words
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(vplane + (int64_t)t0 * rbv);
-      uint4* dst = reinterpret_cast<uint4*>(Vc);
-      for (int i = threadIdx.x; i < ntok16 * rbv / 16; i += kThreads) dst[i] = __ldg(src + i);
-    }
-    for (int i = threadIdx.x; i < ntok16 * ngk; i += kThreads) Ks[i] = scale_at(p.scales_k, ks_base + (int64_t)t0 * ngk + i, p.kind);
-    for (int i = threadIdx.x; i < ntok16 * ngv; i += kThreads) Vs[i] = scale_at(p.scales_v, vs_base + (int64_t)t0 * ngv + i, p.kind);
     __syncthreads();
 
     const int tb = 16 * warp;  // this warp's tokens within the tile
@@ -214,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 2) rope_decode_kernel(const __grid_c
             for (int e = 0; e < 4; ++e) acc[a][n][e] = kv[a][n][e] = 0.0f;
         int cur = 0;
         auto fold = [&](int gi) {
-          const float sl = Ks[tl_lo * ngk + gi], sh = Ks[tl_hi * ngk + gi];
+          const float sl = scale_at(Ks, tl_lo * ngk + gi, p.kind), sh = scale_at(Ks, tl_hi * ngk + gi, p.kind);
 #pragma unroll
           for (int a = 0; a < 2; ++a)
 #pragma unroll
@@ -268,9 +301,15 @@ __global__ void __launch_bounds__(kThreads, 2) rope_decode_kernel(const __grid_c
           const float q1a = qr[d], q1b = qr[d + 1], q2a = qr[d + half], q2b = qr[d + half + 1];
 #pragma unroll
           for (int row = 0; row < 2; ++row) {
-            const int64_t pos = row == 0 ? pos_lo : pos_hi;
-            const float4 cs = pos < t_end ? *reinterpret_cast<const float4*>(p.table + (pos * half + d) * 2)
-                                          : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            const int tl = row == 0 ? tl_lo : tl_hi;
+            // angle of position t0 + tl: its block's first position plus tl % 16
+            const float4 cb = *reinterpret_cast<const float4*>(ang_blk + (tl >> 4) * half + d);
+            const float4 co = *reinterpret_cast<const float4*>(ang_off + (tl & 15) * half + d);
+            float4 cs;
+            cs.x = cb.x * co.x - cb.y * co.y;
+            cs.y = cb.y * co.x + cb.x * co.y;
+            cs.z = cb.z * co.z - cb.w * co.w;
+            cs.w = cb.w * co.z + cb.z * co.w;
             const float k1a = kv[0][n][2 * row], k1b = kv[0][n][2 * row + 1];
             const float k2a = kv[1][n][2 * row], k2b = kv[1][n][2 * row + 1];
             float s = fmaf(q1a, k1a * cs.x - k2a * cs.y, q2a * (k2a * cs.x + k1a * cs.y));
@@ -328,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 2) rope_decode_kernel(const __grid_c
           for (int j = 0; j < 16; ++j) {
             const float pj = __shfl_sync(0xffffffffu, j < 8 ? p_lo : p_hi, 4 * (j & 7));
             // (positions past the row's length carry p = 0 and whatever the cache holds)
-            const float wj = pj == 0.0f ? 0.0f : pj * Vs[(tb + j) * ngv + gi];
+            const float wj = pj == 0.0f ? 0.0f : pj * scale_at(Vs, (tb + j) * ngv + gi, p.kind);
             acc = fmaf(wj, (float)codes[j], acc);
           }
           if (q2 == 0) u0 += acc;
@@ -336,6 +375,7 @@ __global__ void __launch_bounds__(kThreads, 2) rope_decode_kernel(const __grid_c
         }
       }
     }
+    __syncthreads();  // the slot and the key rows are free for the tile after next / the next conversion
   }
   // ---- merge the warps, then the pieces of the unit
   __syncthreads();
@@ -502,12 +542,13 @@ cudaError_t launch_rope_decode(const RopeLaunch& a, cudaStream_t stream) {
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
   p.counters = reinterpret_cast<int32_t*>(ws);
   p.partials = reinterpret_cast<float*>(ws + ((size_t)units * 4 + 255) / 256 * 256);
-  const Smem s = smem_plan((rk_max + 15) & ~15, rvb_max, ngk_max, ngv_max, a.head_dim);
+  const int rbk_max = a.kind == 0 ? rk_max : rk_max / 2;
+  const Smem s = smem_plan((rk_max + 15) & ~15, rbk_max, rvb_max, ngk_max, ngv_max, a.kind == 0 ? 4 : 2,
+                           a.head_dim);
   cudaError_t e = cudaFuncSetAttribute(rope_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s.total);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)p.pieces, (unsigned)units);
-  rope_decode_kernel<<<grid, kThreads, s.total, stream>>>(p, s.off_kc, s.off_vc, s.off_ks, s.off_vs, s.off_bk,
-                                                          s.off_q, s.off_wst, s.off_cta);
+  rope_decode_kernel<<<grid, kThreads, s.total, stream>>>(p, s);
   count_launch();
   return cudaGetLastError();
 }
