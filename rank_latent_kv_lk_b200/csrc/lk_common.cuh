@@ -159,21 +159,6 @@ LK_DEVICE bool lk_mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
-// As lk_mbar_try_wait, but the thread may sleep in hardware for up to
-// `hint_ns` nanoseconds (waking when the phase completes) instead of
-// returning at once, so waiting warps do not occupy issue slots.
-LK_DEVICE bool lk_mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(lk_smem_addr(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return done != 0;
-}
-
 LK_DEVICE uint64_t lk_globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -181,13 +166,17 @@ LK_DEVICE uint64_t lk_globaltimer_ns() {
 }
 
 // Waits for the mbarrier phase with the given parity to complete; gives up
-// after `limit_ns` nanoseconds and returns false.
+// after `limit_ns` nanoseconds and returns false.  Each try_wait (no time
+// hint) suspends the thread in hardware until the phase completes or a
+// system-dependent limit passes, so the loop costs few issue slots.  (A
+// try_wait with a suspend-time hint measured late wake-ups, about 2-3 us
+// after the phase completed, and is not used.)
 LK_DEVICE bool lk_mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (lk_mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = lk_globaltimer_ns();
   for (uint32_t i = 0;; ++i) {
-    if (lk_mbar_try_wait_sleep(bar, parity, 20000u)) return true;
-    if ((i & 15u) == 15u && lk_globaltimer_ns() - t0 > limit_ns) return false;
+    if (lk_mbar_try_wait(bar, parity)) return true;
+    if ((i & 7u) == 7u && lk_globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 
