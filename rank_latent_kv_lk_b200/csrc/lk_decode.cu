@@ -233,6 +233,9 @@ constexpr float kInv254cu = 1.0f / (254.0f * 254.0f * 254.0f);
 // instruction is needed (those share a pipe with exp2).
 // (Explicitly rounded operations: a product contracted into the rounding
 // add would round the exact product instead of the stored one.)
+// WT = 3 stops after t2 (t3 = 0): x is then kept to 1/(2 * 254^2), a
+// relative 6e-8 of the largest weight (the bf16-output path).
+template <int WT>
 LK_DEVICE uint32_t expand_weight(float x) {
   x = fminf(x, 127.0f);
   const float m0 = __fadd_rn(x, kMagic);
@@ -240,10 +243,13 @@ LK_DEVICE uint32_t expand_weight(float x) {
   const float m1 = __fadd_rn(x, kMagic);
   x = __fmul_rn(__fsub_rn(x, __fsub_rn(m1, kMagic)), 254.0f);
   const float m2 = __fadd_rn(x, kMagic);
-  x = __fmul_rn(__fsub_rn(x, __fsub_rn(m2, kMagic)), 254.0f);
-  const float m3 = __fadd_rn(x, kMagic);
+  uint32_t m3 = 0u;
+  if constexpr (WT == 4) {
+    x = __fmul_rn(__fsub_rn(x, __fsub_rn(m2, kMagic)), 254.0f);
+    m3 = __float_as_uint(__fadd_rn(x, kMagic));
+  }
   const uint32_t lo = __byte_perm(__float_as_uint(m0), __float_as_uint(m1), 0x0040u);
-  const uint32_t hi = __byte_perm(__float_as_uint(m2), __float_as_uint(m3), 0x0040u);
+  const uint32_t hi = __byte_perm(__float_as_uint(m2), m3, 0x0040u);
   return __byte_perm(lo, hi, 0x5410u);
 }
 
@@ -323,7 +329,8 @@ LK_DEVICE void token_score2(const uint8_t* kc, const uint8_t* ks, const HeadGeom
     int a0 = 0, a1 = 0, a2 = 0, b0 = 0, b1 = 0, b2 = 0;
 #pragma unroll
     for (int c = 0; c < MAXCH; ++c) {
-      if (c < nch) {
+      if (c >= nch) break;  // (uniform; the chunks left hold no codes)
+      {
         Chunk<CS> ca, cb;
         ca.load(kc, g.rbk, tl, c);
         if constexpr (TG == 2) cb.load(kc, g.rbk, tb, c);
@@ -357,7 +364,8 @@ LK_DEVICE void token_score2(const uint8_t* kc, const uint8_t* ks, const HeadGeom
     // odd dims); groups are multiples of 8 dims
 #pragma unroll
     for (int c = 0; c < MAXCH; ++c) {
-      if (c < nch) {
+      if (c >= nch) break;  // (uniform; the chunks left hold no codes)
+      {
         Chunk<CS> ca, cb;
         ca.load(kc, g.rbk, tl, c);
         if constexpr (TG == 2) cb.load(kc, g.rbk, tb, c);
@@ -611,7 +619,7 @@ LK_DEVICE void absorb_q(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
 // CTA's next stage, carried across units.  NM = ceil(r_V / 8) V products per
 // stage, fixed at compile time (runtime bounds on these loops cost more
 // instructions than the products themselves).
-template <int KIND, int CSK, int NM, bool VG1, int TG>
+template <int KIND, int CSK, int NM, bool VG1, int TG, int WT>
 LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, const HeadGeom& g, int b,
                         int len, int s0, int s1, int& buf, uint32_t& phase, bool& waited) {
   const Bars B = bars_of(smem, L);
@@ -704,8 +712,8 @@ LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
         inv = 127.0f / wref;
       }
       uint32_t a0a, a2a, a0b = 0u, a2b = 0u;
-      weight_frags(expand_weight(pa * ga * inv), sel1, sel2, gid, tig, a0a, a2a);
-      if constexpr (TG == 2) weight_frags(expand_weight(pb * gb * inv), sel1, sel2, gid, tig, a0b, a2b);
+      weight_frags(expand_weight<WT>(pa * ga * inv), sel1, sel2, gid, tig, a0a, a2a);
+      if constexpr (TG == 2) weight_frags(expand_weight<WT>(pb * gb * inv), sel1, sel2, gid, tig, a0b, a2b);
       // c. acc[jm] += terms x codes of dims 8 jm .. 8 jm + 7, each group
       //    (dims >= r_V only in the last product, when r_V % 8 != 0)
 #pragma unroll
@@ -735,12 +743,12 @@ LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
       for (int gi = 0; gi < g.ngv; ++gi) {
         const float ga = va ? load_scale(vs, tl * g.ngv + gi, KIND) : 0.0f;
         uint32_t a0a, a2a;
-        weight_frags(expand_weight(pa * ga * inv), sel1, sel2, gid, tig, a0a, a2a);
+        weight_frags(expand_weight<WT>(pa * ga * inv), sel1, sel2, gid, tig, a0a, a2a);
         fr[(gi * 2 + 0) * 32 + lane] = make_uint2(a0a, a2a);
         if constexpr (TG == 2) {
           const float gb = vb ? load_scale(vs, (tl + 32) * g.ngv + gi, KIND) : 0.0f;
           uint32_t a0b, a2b;
-          weight_frags(expand_weight(pb * gb * inv), sel1, sel2, gid, tig, a0b, a2b);
+          weight_frags(expand_weight<WT>(pb * gb * inv), sel1, sel2, gid, tig, a0b, a2b);
           fr[(gi * 2 + 1) * 32 + lane] = make_uint2(a0b, a2b);
         }
       }
@@ -790,10 +798,10 @@ LK_DEVICE void run_unit(const DecodeParams& p, uint8_t* smem, const SmemLayout& 
   }
 }
 
-template <int KIND, int CSK, bool VG1, int TG>
+template <int KIND, int CSK, bool VG1, int TG, int WT>
 LK_DEVICE void run_unit_nm(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, const HeadGeom& g, int b,
                            int len, int s0, int s1, int& buf, uint32_t& phase, bool& waited) {
-#define LK_RUN(NMV) run_unit<KIND, CSK, NMV, VG1, TG>(p, smem, L, g, b, len, s0, s1, buf, phase, waited)
+#define LK_RUN(NMV) run_unit<KIND, CSK, NMV, VG1, TG, WT>(p, smem, L, g, b, len, s0, s1, buf, phase, waited)
   switch ((g.rv + 7) >> 3) {
     case 1: LK_RUN(1); break;
     case 2: LK_RUN(2); break;
@@ -943,7 +951,7 @@ LK_DEVICE void finish_unit(const DecodeParams& p, uint8_t* smem, const SmemLayou
   consumer_sync();
 }
 
-template <int KIND, int TG>
+template <int KIND, int TG, int WT>
 LK_DEVICE void consume(const DecodeParams& p, uint8_t* smem, const SmemLayout& L, int i0, int i1, int c) {
   int u = i0 / p.S, s = i0 - u * p.S;
   int it = i0, n = 0, buf = 0;
@@ -959,13 +967,13 @@ LK_DEVICE void consume(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
     const int len = waited ? unit_len(p, b) : p.stable_len;
     const int csk = lk_chunk_bytes(g.rbk);
     if (KIND == 0 || g.ngv == 1) {
-      if (csk == 16) run_unit_nm<KIND, 16, true, TG>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
-      else if (csk == 8) run_unit_nm<KIND, 8, true, TG>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
-      else run_unit_nm<KIND, 4, true, TG>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      if (csk == 16) run_unit_nm<KIND, 16, true, TG, WT>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      else if (csk == 8) run_unit_nm<KIND, 8, true, TG, WT>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      else run_unit_nm<KIND, 4, true, TG, WT>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
     } else if constexpr (KIND == 1) {
-      if (csk == 16) run_unit_nm<KIND, 16, false, TG>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
-      else if (csk == 8) run_unit_nm<KIND, 8, false, TG>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
-      else run_unit_nm<KIND, 4, false, TG>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      if (csk == 16) run_unit_nm<KIND, 16, false, TG, WT>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      else if (csk == 8) run_unit_nm<KIND, 8, false, TG, WT>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
+      else run_unit_nm<KIND, 4, false, TG, WT>(p, smem, L, g, b, len, s, s_end, buf, phase, waited);
     }
     finish_unit<KIND>(p, smem, L, g, b, h, u, it, seg_end, i0, c, n);
     it = seg_end;
@@ -976,7 +984,8 @@ LK_DEVICE void consume(const DecodeParams& p, uint8_t* smem, const SmemLayout& L
   if (!waited) lk_grid_dep_wait();  // this grid never completes before the previous one
 }
 
-template <int KIND, int TG>
+// WT: int8 terms of the value weights (4 for fp32 outputs, 3 for bf16 outputs)
+template <int KIND, int TG, int WT>
 __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const SmemLayout L = smem_layout(p);
@@ -1006,7 +1015,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_attn_kernel(const __grid_c
     if (threadIdx.x == kConsumerThreads) produce<KIND>(p, smem, L, i0, i1);
     return;
   }
-  consume<KIND, TG>(p, smem, L, i0, i1, c);
+  consume<KIND, TG, WT>(p, smem, L, i0, i1, c);
   if (threadIdx.x == 0 && *bars_of(smem, L).abort_flag) lk_dev_fail(LK_DEV_TIMEOUT_PIPE);
 }
 
@@ -1020,24 +1029,28 @@ namespace {
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 using DecodeKernel = void (*)(DecodeParams);
-DecodeKernel decode_kernel(int kind, int tg) {
-  if (kind == 0) return tg == 2 ? decode_attn_kernel<0, 2> : decode_attn_kernel<0, 1>;
-  return tg == 2 ? decode_attn_kernel<1, 2> : decode_attn_kernel<1, 1>;
+DecodeKernel decode_kernel(int kind, int tg, int wt) {
+  if (wt == 3) {
+    if (kind == 0) return tg == 2 ? decode_attn_kernel<0, 2, 3> : decode_attn_kernel<0, 1, 3>;
+    return tg == 2 ? decode_attn_kernel<1, 2, 3> : decode_attn_kernel<1, 1, 3>;
+  }
+  if (kind == 0) return tg == 2 ? decode_attn_kernel<0, 2, 4> : decode_attn_kernel<0, 1, 4>;
+  return tg == 2 ? decode_attn_kernel<1, 2, 4> : decode_attn_kernel<1, 1, 4>;
 }
 
 // Resident CTAs per SM of the decode kernel for `smem` bytes of shared memory
 // (cached per device, kernel and size; the query costs a few microseconds).
-int decode_occupancy(int kind, int tg, int smem) {
+int decode_occupancy(int kind, int tg, int wt, int smem) {
   static std::mutex mu;
   static std::map<std::tuple<int, int, int>, int> cache;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 1;
-  const auto key = std::make_tuple(dev, kind * 4 + tg, smem);
+  const auto key = std::make_tuple(dev, kind * 16 + wt * 4 + tg, smem);
   std::lock_guard<std::mutex> lock(mu);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
   int occ = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel(kind, tg), kThreads, smem);
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel(kind, tg, wt), kThreads, smem);
   if (e != cudaSuccess || occ < 1) occ = 1;
   cache[key] = occ;
   return occ;
@@ -1167,10 +1180,12 @@ cudaError_t launch_decode_attn(const DecodeLaunch& a, cudaStream_t stream) {
     p.nstages = (int)std::max<int64_t>(2, std::min<int64_t>(p.nstages, per_cta));
   }
   const int smem = smem_bytes_for(p);
-  const DecodeKernel kernel = decode_kernel(a.kind, tg);
+  // bf16 outputs (bound 1e-2 RMS) take three value-weight terms, fp32 four
+  const int wt = a.out_bf16 ? 3 : 4;
+  const DecodeKernel kernel = decode_kernel(a.kind, tg, wt);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int resident = decode_occupancy(a.kind, tg, smem) * a.num_sms;
+  const int resident = decode_occupancy(a.kind, tg, wt, smem) * a.num_sms;
   int64_t cap = std::min(resident, kAutoCtaBound);
   // In a decode step this launch overlaps the projection kernel, whose CTAs
   // hold part of every SM's registers until it ends: only one attention CTA
